@@ -1,0 +1,369 @@
+"""Pins for the CPU oracle: closed forms, invariants, brute force, fixtures.
+
+Each test ties one oracle function to something other than itself, chosen so
+that a plausible slip (a dropped term, a wrong sign or index, a transposed
+operand, an off-by-one in a rank) fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def _bf16(a):
+    return O.bf16_round(a)
+
+
+# ---------------------------------------------------------------- a1 logits
+
+def test_router_logits_matches_fsum_and_bias():
+    r = _rng(1)
+    x = _bf16(r.standard_normal((5, 7)))
+    W = _bf16(0.1 * r.standard_normal((7, 3)))
+    b = np.array([0.5, -1.0, 0.25])
+    got = O.router_logits(x, W, b)
+    for t in range(5):
+        for e in range(3):
+            want = math.fsum(x[t, i] * W[i, e] for i in range(7)) + b[e]
+            assert abs(got[t, e] - want) < 1e-14
+    # layout pin: [d, E] (a transposed operand would not even have this shape)
+    assert got.shape == (5, 3)
+
+
+def test_dot_error_bound_holds_for_fp32_sums():
+    r = _rng(2)
+    x = _bf16(r.standard_normal((64, 512)))
+    W = _bf16(0.02 * r.standard_normal((512, 4)))
+    exact = O.router_logits(x, W)
+    bound = O.dot_error_bound(x, W)
+    x32, W32 = x.astype(np.float32), W.astype(np.float32)
+    for order in (np.arange(512), np.arange(512)[::-1], r.permutation(512)):
+        acc = np.zeros((64, 4), dtype=np.float32)
+        for i in order:
+            acc = (acc + x32[:, i:i + 1] * W32[i:i + 1, :]).astype(np.float32)
+        assert np.all(np.abs(acc.astype(np.float64) - exact) <= bound)
+
+
+# ------------------------------------------------------------- a2 top-K
+
+def test_topk_golden_ties():
+    g = json.load(open(os.path.join(GOLD, "topk_ties.json")))
+    for row, K, idx, w in zip(g["rows"], g["K"], g["idx"], g["weights_approx"]):
+        l = np.array([row], dtype=np.float32)
+        got = O.topk_select(l, K)
+        assert got[0].tolist() == idx
+        ww = O.renormalized_weights(l.astype(np.float64), got)
+        assert np.allclose(ww[0], w, rtol=0, atol=2e-7)
+
+
+def test_topk_bruteforce_small():
+    r = _rng(3)
+    for trial in range(200):
+        E = int(r.integers(1, 7))
+        K = int(r.integers(1, E + 1))
+        # coarse grid -> many exact ties
+        l = (r.integers(-3, 4, size=(1, E)) * 0.5).astype(np.float32)
+        got = O.topk_select(l, K)[0].tolist()
+        want = sorted(range(E), key=lambda e: (-float(l[0, e]), e))[:K]
+        assert got == want
+        # the chosen set dominates every unchosen value
+        rest = [e for e in range(E) if e not in got]
+        if rest:
+            assert min(l[0, got]) >= max(l[0, rest])
+
+
+def test_renormalized_weights_sum_and_special_cases():
+    r = _rng(4)
+    l = r.standard_normal((50, 8)) * 3
+    for K in range(1, 9):
+        idx = O.topk_select(l, K)
+        w = O.renormalized_weights(l, idx)
+        assert np.allclose(w.sum(axis=1), 1.0, atol=1e-15, rtol=0)
+        assert np.all(np.diff(w, axis=1) <= 1e-15)  # descending logits -> descending weights
+    # K = 1: weight exactly 1
+    assert np.all(O.renormalized_weights(l, O.topk_select(l, 1)) == 1.0)
+    # K = E: the weights are the full softmax, in selection order
+    idx = O.topk_select(l, 8)
+    w = O.renormalized_weights(l, idx)
+    p = O.softmax_rows(l)
+    assert np.allclose(w, np.take_along_axis(p, idx.astype(np.int64), 1), atol=1e-15)
+    # any K: renormalised full-softmax probabilities
+    idx = O.topk_select(l, 3)
+    ps = np.take_along_axis(p, idx.astype(np.int64), 1)
+    assert np.allclose(O.renormalized_weights(l, idx), ps / ps.sum(1, keepdims=True), atol=1e-14)
+
+
+def test_bias_shifts_selection_in_fp32():
+    l = np.array([[1.0, 0.9, 0.0]], dtype=np.float32)
+    b = np.array([0.0, 0.2, 0.0], dtype=np.float32)
+    idx, w, lb = O.route_from_logits_f32(l, 1, b)
+    assert idx.tolist() == [[1]]
+    assert lb.dtype == np.float32 and lb[0, 1] == np.float32(np.float32(0.9) + np.float32(0.2))
+    # the weights use the biased logits
+    idx, w, _ = O.route_from_logits_f32(l, 2, b)
+    assert idx.tolist() == [[1, 0]]
+    d = float(lb[0, 1]) - float(lb[0, 0])
+    assert abs(w[0, 0] - 1 / (1 + math.exp(-d))) < 1e-15
+
+
+# ------------------------------------------------------------- a3 stats
+
+def test_counts_sum_and_bincount():
+    r = _rng(5)
+    l = r.standard_normal((300, 10))
+    idx = O.topk_select(l, 3)
+    c = O.expert_counts(idx, 10)
+    assert c.sum() == 900
+    assert np.array_equal(c, np.bincount(idx.reshape(-1), minlength=10))
+
+
+def test_aux_loss_uniform_cases():
+    r = _rng(6)
+    E, T, K = 8, 64, 2
+    # W_r = 0 -> every logit 0 -> P_i = 1/E exactly, so aux = sum f_i = 1
+    probs = O.softmax_rows(np.zeros((T, E)))
+    assert np.all(probs == 1.0 / E)
+    cnt = np.array([30, 10, 20, 5, 15, 20, 10, 18])  # sums to 128 = T*K
+    f, P, aux = O.load_stats(cnt, probs, T, K)
+    assert abs(aux - 1.0) < 1e-15 and abs(f.sum() - 1) < 1e-15
+    # uniform f with arbitrary P -> aux = sum P_i = 1
+    probs = O.softmax_rows(r.standard_normal((T, E)))
+    f, P, aux = O.load_stats(np.full(E, T * K // E), probs, T, K)
+    assert abs(aux - 1.0) < 1e-14
+    # the same with f measured against the mean load: N * sum (N f_i) P_i = N
+    assert abs(E * np.sum(E * f * P) - E) < 1e-12
+    # concentrated routing raises it: all on expert 0 with P_0 = 1 -> aux = E
+    probs = np.zeros((T, E)); probs[:, 0] = 1
+    cnt = np.zeros(E, dtype=np.int64); cnt[0] = T * K
+    assert abs(O.load_stats(cnt, probs, T, K)[2] - E) < 1e-15
+
+
+# ------------------------------------------------------------- a4 dispatch
+
+def test_capacity_values():
+    assert O.capacity(8192, 4, 60, 1.0) == 547       # ceil(32768/60) = ceil(546.13)
+    assert O.capacity(60, 1, 60, 1.0) == 1
+    assert O.capacity(32, 1, 8, 1.25) == 5           # 1.25*4 = 5 exactly
+    assert O.capacity(4, 2, 3, 0.75) == 2
+    assert O.capacity(10, 1, 1, 0.5) == 5
+    assert O.capacity(7, 1, 2, 1.0) == 4             # ceil(3.5)
+    assert O.capacity(100, 2, 8, 0.0) is None
+    assert O.capacity(100, 2, 8, -1.0) is None
+
+
+def test_dispatch_golden():
+    g = json.load(open(os.path.join(GOLD, "dispatch_4tok_3exp.json")))
+    idx = np.array(g["idx"], dtype=np.int32)
+    C = O.capacity(g["T"], g["K"], g["E"], g["capacity_factor"])
+    assert C == g["capacity"]
+    d = O.dispatch(idx, g["E"], C)
+    assert d["counts"].tolist() == g["counts"]
+    assert d["kept"].tolist() == g["kept"]
+    assert d["offsets"].tolist() == g["offsets"]
+    assert d["inv"].tolist() == g["inv"]
+    assert d["src"].tolist() == g["src"]
+    assert d["n_dropped"] == g["n_dropped"]
+
+
+@pytest.mark.parametrize("C", [None, 1, 3, 7, 40])
+def test_dispatch_invariants(C):
+    r = _rng(7)
+    T, E, K = 97, 9, 3
+    idx = O.topk_select(r.standard_normal((T, E)) + np.linspace(0, 2, E), K)
+    d = O.dispatch(idx, E, C)
+    cnt = d["counts"]
+    assert cnt.sum() == T * K
+    assert np.array_equal(d["kept"], cnt if C is None else np.minimum(cnt, C))
+    assert d["n_dropped"] == (0 if C is None else int(np.maximum(cnt - C, 0).sum()))
+    off = d["offsets"]
+    assert off[0] == 0 and np.all(np.diff(off) >= 0) and off[-1] == d["kept"].sum()
+    inv, src = d["inv"], d["src"]
+    rows = inv[inv >= 0]
+    assert sorted(rows.tolist()) == list(range(int(off[-1])))  # bijection
+    for t in range(T):
+        for k in range(K):
+            if inv[t, k] >= 0:
+                r_ = int(inv[t, k])
+                assert src[r_] == t
+                e = int(idx[t, k])
+                assert off[e] <= r_ < off[e + 1]
+            assert (inv[t, k] < 0) == bool(d["drop"][t, k])
+    # brute force: each expert keeps its first C tokens in ascending order
+    for e in range(E):
+        toks = [t for t in range(T) if e in idx[t].tolist()]
+        keep = toks if C is None else toks[:C]
+        assert src[off[e]:off[e + 1]].tolist() == keep
+
+
+# ------------------------------------------------------------- a5 FFN
+
+def test_swiglu_scalar_closed_form():
+    a, b, c = 0.7, -1.3, 2.5
+    y = O.swiglu_ffn(np.array([[1.0]]), np.array([[a]]), np.array([[b]]), np.array([[c]]))
+    assert abs(y[0, 0] - (a / (1 + math.exp(-a))) * b * c) < 1e-15
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    assert abs(O.silu(np.array([-40.0]))[0]) < 1e-15
+
+
+def test_swiglu_gate_is_w1_and_down_is_w2():
+    r = _rng(8)
+    X = r.standard_normal((4, 6))
+    W1 = r.standard_normal((6, 5)); W3 = r.standard_normal((6, 5)); W2 = r.standard_normal((5, 6))
+    y = O.swiglu_ffn(X, W1, W3, W2)
+    g, u = X @ W1, X @ W3
+    want = (g / (1 + np.exp(-g)) * u) @ W2
+    assert np.allclose(y, want, atol=1e-13)
+    # swapping the roles of W1 and W3 changes the result (the gate is W1)
+    assert not np.allclose(O.swiglu_ffn(X, W3, W1, W2), y)
+    # W1 = 0 -> y = 0 exactly; doubling W2 doubles y exactly
+    assert np.all(O.swiglu_ffn(X, 0 * W1, W3, W2) == 0)
+    assert np.array_equal(O.swiglu_ffn(X, W1, W3, 2 * W2), 2 * y)
+
+
+# ------------------------------------------------------------- layer
+
+def _layer_inputs(T=24, d=16, f=12, E=4, seed=9, w=0.3):
+    r = _rng(seed)
+    x = _bf16(r.standard_normal((T, d)))
+    Wr = _bf16(w * r.standard_normal((d, E)))
+    W1 = _bf16(w * r.standard_normal((E, d, f)))
+    W3 = _bf16(w * r.standard_normal((E, d, f)))
+    W2 = _bf16(w * r.standard_normal((E, f, d)))
+    return x, Wr, W1, W3, W2
+
+
+def test_layer_E1_is_dense_ffn():
+    x, Wr, W1, W3, W2 = _layer_inputs(E=1)
+    out = O.moe_layer(x, Wr, W1, W3, W2, K=1)
+    assert np.allclose(out["y"], O.swiglu_ffn(x, W1[0], W3[0], W2[0]), atol=1e-13)
+
+
+def test_layer_identical_experts_independent_of_routing():
+    x, Wr, W1, W3, W2 = _layer_inputs(E=5)
+    W1[:] = W1[0]; W3[:] = W3[0]; W2[:] = W2[0]
+    dense = O.swiglu_ffn(x, W1[0], W3[0], W2[0])
+    for K in (1, 2, 5):
+        out = O.moe_layer(x, Wr, W1, W3, W2, K=K)
+        assert np.allclose(out["y"], dense, atol=1e-12)
+
+
+def test_layer_K_equals_E_is_full_mixture():
+    x, Wr, W1, W3, W2 = _layer_inputs(E=4)
+    out = O.moe_layer(x, Wr, W1, W3, W2, K=4)
+    p = O.softmax_rows(out["logits32"].astype(np.float64))
+    want = sum(p[:, e:e + 1] * O.swiglu_ffn(x, W1[e], W3[e], W2[e]) for e in range(4))
+    assert np.allclose(out["y"], want, atol=1e-12)
+
+
+def test_layer_unselected_expert_contributes_nothing():
+    x, Wr, W1, W3, W2 = _layer_inputs(E=6)
+    bias = np.zeros(6, dtype=np.float32)
+    bias[5] = -1e4                      # expert 5 can never be selected
+    out = O.moe_layer(x, Wr, W1, W3, W2, K=2, bias32=bias)
+    assert out["counts"][5] == 0
+    W1b, W3b, W2b = W1.copy(), W3.copy(), W2.copy()
+    W1b[5] = np.nan; W3b[5] = np.nan; W2b[5] = np.nan
+    out2 = O.moe_layer(x, Wr, W1b, W3b, W2b, K=2, bias32=bias)
+    assert np.array_equal(out2["y"], out["y"])
+
+
+def test_layer_linear_in_w2_and_zero_gate():
+    x, Wr, W1, W3, W2 = _layer_inputs()
+    a = O.moe_layer(x, Wr, W1, W3, W2, K=2)["y"]
+    b = O.moe_layer(x, Wr, W1, W3, 2 * W2, K=2)["y"]
+    assert np.array_equal(b, 2 * a)
+    assert np.all(O.moe_layer(x, Wr, 0 * W1, W3, W2, K=2)["y"] == 0)
+
+
+def test_layer_bruteforce_per_token_with_capacity():
+    x, Wr, W1, W3, W2 = _layer_inputs(T=30, E=3, seed=10)
+    T, E, K, cf = 30, 3, 2, 0.75   # C = 15 exactly
+    out = O.moe_layer(x, Wr, W1, W3, W2, K=K, capacity_factor=cf)
+    C = 15
+    l32 = (x @ Wr).astype(np.float32)
+    seen = [0] * E
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-float(l32[t, e]), e))[:K]
+        z = np.exp(np.array([float(l32[t, e]) for e in order]) - float(l32[t, order[0]]))
+        w = z / z.sum()
+        y = np.zeros(x.shape[1])
+        for j, e in enumerate(order):
+            if seen[e] < C:
+                h = x[t] @ W1[e]
+                y += w[j] * ((h / (1 + np.exp(-h))) * (x[t] @ W3[e])) @ W2[e]
+            seen[e] += 1
+        assert np.allclose(out["y"][t], y, atol=1e-12), t
+    assert out["n_dropped"] == sum(max(0, s - C) for s in seen)
+
+
+def test_layer_all_slots_dropped_gives_zero():
+    x, Wr, W1, W3, W2 = _layer_inputs(T=10, E=2, seed=11)
+    out = O.moe_layer(x, Wr, W1, W3, W2, K=2, capacity_factor=0.0625)  # C = ceil(0.625) = 1
+    assert out["capacity"] == 1
+    for t in range(10):
+        if np.all(out["inv"][t] < 0):
+            assert np.all(out["y"][t] == 0)
+    # K = E = 2: every token picks both experts, so token 0 fills both slots
+    assert np.all(out["inv"][0] >= 0)
+    assert np.all(out["inv"][1:] < 0) and np.all(out["y"][1:] == 0)
+
+
+def test_layer_token_subset_matches_full():
+    x, Wr, W1, W3, W2 = _layer_inputs(T=20, seed=12)
+    full = O.moe_layer(x, Wr, W1, W3, W2, K=2, capacity_factor=1.0)
+    part = O.moe_layer(x, Wr, W1, W3, W2, K=2, capacity_factor=1.0, tokens=[3, 7, 19])
+    assert np.array_equal(part["y"][[3, 7, 19]], full["y"][[3, 7, 19]])
+    assert np.isnan(part["y"][0]).all()
+
+
+# ------------------------------------------------------------- a7 bias
+
+def test_bias_update_closed_form_over_steps():
+    r = _rng(13)
+    E, T, K, alpha = 6, 12, 2, 1e-3   # target T*K/E = 4
+    b = np.zeros(E, dtype=np.float32)
+    under = np.zeros(E, dtype=np.int64); over = np.zeros(E, dtype=np.int64)
+    ref = np.zeros(E, dtype=np.float32)
+    a32 = np.float32(alpha)
+    for step in range(10):
+        cnt = r.multinomial(T * K, np.ones(E) / E)
+        b = O.bias_update(b, cnt, T, K, alpha)
+        for e in range(E):
+            if cnt[e] > 4:
+                over[e] += 1; ref[e] = np.float32(ref[e] - a32)
+            elif cnt[e] < 4:
+                under[e] += 1; ref[e] = np.float32(ref[e] + a32)
+        assert np.array_equal(b.view(np.uint32), ref.view(np.uint32))
+    assert np.allclose(b, alpha * (under - over), atol=1e-6)
+
+
+def test_bias_update_direction_and_equality():
+    b0 = np.array([0.5, 0.5, 0.5], dtype=np.float32)
+    b = O.bias_update(b0, np.array([5, 4, 3]), T=6, K=2, alpha=0.25)  # target 4
+    assert b.tolist() == [0.25, 0.5, 0.75]
+    # non-integer target: T*K/E = 10/3; counts 3 < 3.33 < 4
+    b = O.bias_update(np.zeros(3, np.float32), np.array([4, 3, 3]), T=5, K=2, alpha=1.0)
+    assert b.tolist() == [-1.0, 1.0, 1.0]
+
+
+def test_bf16_round_ties_to_even():
+    vals = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5])
+    got = O.bf16_round(vals)
+    assert got.tolist() == [1.0, 1.0, 1.0 + 4 * 2 ** -8, 1.0, -2.5]
+
+
+def test_capacity_uses_exact_value_of_the_double():
+    # 0.8 is stored as 0.8000000000000000444..., so 0.8*30*2/3 is just above 16
+    assert O.capacity(30, 2, 3, 0.8) == 17
+    assert O.capacity(30, 2, 3, 0.75) == 15
