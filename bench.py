@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""MoE-layer forward benchmark on B200: tokens/s and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one full moe_layer_forward (route, top-K, stats, dispatch, both
+expert GEMMs, combine, bias update where the workload has one) over one batch
+of T synthetic tokens whose inputs already sit in HBM.  Inputs (2.8 GB of
+expert weights for the default Mixtral-shaped decode workload) are larger
+than L2, so no flush is needed between steps.  With N > 1 (torchrun), every
+rank runs an independent replica of the layer (the path has no exchange
+step), timing is the max over ranks and ``value`` counts all ranks' tokens.
+
+``--impl reference`` times the CPU oracle (the plain fp64 implementation the
+tests check against) on the host cores on a bounded token sample per step;
+under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_layer_gemm_b200 import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200 (Mixtral shape decode/prefill); % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="mixtral_decode", choices=sorted(synth.workloads().keys()))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=200)
+    p.add_argument("--cpu-sample-tokens", type=int, default=32)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        loaded = [r for r in rows if r[1].replace(".", "").isdigit() and float(r[3] or 0) > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[5 + i].lower() == "active"})
+        sm_loaded = [float(r[1]) for r in loaded if r[1].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm_loaded or sm), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3])}
+
+
+def layer_algorithmic(wl, counts: np.ndarray, kept: np.ndarray):
+    """Algorithmic bytes / FLOPs of one layer step and of its expert GEMMs.
+
+    Layer: weights of every expert with >= 1 kept row (3 d f bf16) + x (bf16)
+    + y (fp32) + W_r (bf16); FLOPs 2 T d E (router) + 6 d f N_kept.
+    Expert GEMMs (gate/up + down, one kernel): the touched weights plus the
+    activations they must move: x_perm in (bf16), H out and back in (bf16),
+    y_perm out (fp32); FLOPs 6 d f N_kept.
+    """
+    T, d, f, E = wl.T, wl.d_model, wl.d_ff, wl.E
+    n_kept = int(kept.sum())
+    touched = int((kept > 0).sum())
+    wbytes = touched * 3 * d * f * 2
+    layer_bytes = wbytes + T * d * 2 + T * d * 4 + d * E * 2
+    layer_flops = 2 * T * d * E + 6 * d * f * n_kept
+    gemm_bytes = wbytes + n_kept * (d * 2 + 2 * f * 2 + d * 4)
+    gemm_flops = 6 * d * f * n_kept
+    return dict(n_kept=n_kept, touched=touched, layer_bytes=layer_bytes, layer_flops=layer_flops,
+                gemm_bytes=gemm_bytes, gemm_flops=gemm_flops)
+
+
+def profile_traffic(workload: str):
+    """DRAM bytes per step of the expert GEMMs from the committed ncu summary,
+    or None when it is missing or was taken on a different kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"grouped_gemm_{workload}.txt")
+    src = os.path.join(ROOT, "moe_layer_gemm_b200", "csrc", "gemm.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        vals = {}
+        for line in open(path):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+        if vals.get("gemm_cu_sha256_16") != h:
+            return None
+        return int(float(vals["dram_bytes_per_step"]))
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------- oracle timing
+
+def time_oracle(wl, x_h, Wr_h, W1_h, W3_h, W2_h, tokens, bias32=None, steps=1):
+    """Wall time of the CPU oracle on a token sample (routing all T tokens)."""
+    sys.path.insert(0, ROOT)
+    from oracle import moe_oracle as O
+    x64 = x_h.double().numpy()
+    Wr64 = Wr_h.double().numpy()
+
+    class Slab:
+        def __init__(self, t):
+            self.t = t
+            self.shape = tuple(t.shape)
+
+        def __getitem__(self, e):
+            return self.t[int(e)].numpy()   # fp32 view; the oracle widens to fp64
+
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        O.moe_layer(x64, Wr64, Slab(W1_h), Slab(W3_h), Slab(W2_h), wl.K, wl.capacity_factor,
+                    bias32=bias32, alpha=wl.alpha, tokens=tokens)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def host_inputs(wl, device):
+    """x, Wr, W1, W3, W2 as host fp32 tensors (generated where it is fastest)."""
+    x = synth.make_x(wl, device=device)
+    Wr = synth.make_router(wl, device=device)
+    W1, W3, W2 = synth.make_expert_weights(wl, device=device)
+    return [t.to("cpu", torch.float32) for t in (x, Wr, W1, W3, W2)]
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = synth.get_workload(args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x_h, Wr_h, W1_h, W3_h, W2_h = host_inputs(wl, dev)
+    S = min(args.cpu_sample_tokens, wl.T)
+    tokens = np.linspace(0, wl.T - 1, S).astype(int).tolist()
+    bias = np.zeros(wl.E, np.float32) if wl.use_bias else None
+    steps = max(1, min(args.steps, 5))
+    warm = min(args.warmup, 1)
+    if warm:
+        time_oracle(wl, x_h, Wr_h, W1_h, W3_h, W2_h, tokens, bias, warm)
+    times = time_oracle(wl, x_h, Wr_h, W1_h, W3_h, W2_h, tokens, bias, steps)
+    sec = statistics.mean(times)
+    value = S / sec
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": warm, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
+                   "capacity_factor": wl.capacity_factor},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{S} of {wl.T} tokens per step (routing, counts and capacity over all "
+                                   f"{wl.T}); {steps} steps after {warm} warm-up (of {args.steps}/{args.warmup} "
+                                   f"asked, bounded to minutes)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    from moe_layer_gemm_b200 import abi
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = False
+    if world > 1:
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+        pg = True
+
+    def barrier():
+        if pg:
+            torch.distributed.barrier()
+
+    wl = synth.get_workload(args.workload)
+    dims = abi.Dims(wl.T, wl.d_model, wl.d_ff, wl.E, wl.K, wl.capacity_factor)
+    x = synth.make_x(wl, device=dev)
+    Wr = synth.make_router(wl, device=dev)
+    W1, W3, W2 = synth.make_expert_weights(wl, device=dev)
+    W13p, W2p = abi.pack_weights(dims, W1, W3, W2)
+    torch.cuda.synchronize()
+    host_w = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host_w = [t.to("cpu", torch.float32) for t in (x, Wr, W1, W3, W2)]
+    del W1, W3, W2
+    torch.cuda.empty_cache()
+    ws = abi.alloc_workspace(dims, dev)
+    y = torch.empty(wl.T, wl.d_model, dtype=torch.float32, device=dev)
+    E = wl.E
+    i32 = dict(dtype=torch.int32, device=dev)
+    outs = dict(counts=torch.zeros(E, **i32), kept=torch.zeros(E, **i32), n_dropped=torch.zeros(1, **i32),
+                f=torch.zeros(E, dtype=torch.float32, device=dev), P=torch.zeros(E, dtype=torch.float32, device=dev),
+                aux=torch.zeros(1, dtype=torch.float32, device=dev))
+    bias = torch.zeros(E, dtype=torch.float32, device=dev) if wl.use_bias else None
+    alpha = float(wl.alpha) if wl.use_bias else 0.0
+
+    def step(evs=None):
+        abi.moe_layer_forward(dims, x, Wr, bias, alpha, W13p, W2p, y, ws, outs, stage_events=evs)
+
+    abi.moe_reset_device_status(ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, detail = abi.moe_get_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device-side wait ran out during warm-up (code {detail})")
+
+    # ---- timed region: K steps, per-stage events recorded live
+    K = args.steps
+    nev = abi.NUM_STAGE_EVENTS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(K)]
+    s = torch.cuda.current_stream()
+    for row in evs:      # create the underlying events before the timed region
+        for e in row:
+            e.record(s)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    start.record(s)
+    for i in range(K):
+        step(evs[i])
+    end.record(s)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = start.elapsed_time(end)
+    if pg:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / K
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in range(K)])
+    stage_ms = stage.mean(axis=0)
+    st, detail = abi.moe_get_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device-side wait ran out in the timed region (code {detail})")
+
+    counts = outs["counts"].cpu().numpy()
+    kept = outs["kept"].cpu().numpy()
+    alg = layer_algorithmic(wl, counts, kept)
+    peaks, peak_src = load_peaks()
+    gemm_ms = float(stage_ms[2] + stage_ms[3])
+    sustained = ms_total > 1000.0
+    tensor_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    bw = peaks["hbm_gbs"]
+    t_bytes = alg["layer_bytes"] / (bw * 1e9)
+    t_flops = alg["layer_flops"] / (tensor_peak * 1e12)
+    layer_bound = "hbm" if t_bytes >= t_flops else "tensor"
+    g_bytes_t = alg["gemm_bytes"] / (bw * 1e9)
+    g_flops_t = alg["gemm_flops"] / (tensor_peak * 1e12)
+    if g_bytes_t >= g_flops_t:
+        achieved = alg["gemm_bytes"] / (gemm_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": bw, "unit": "GB/s", "frac": achieved / bw}
+    else:
+        achieved = alg["gemm_flops"] / (gemm_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak}
+    traffic = profile_traffic(wl.name)
+    roof.update({"traffic": traffic, "kernel": "grouped_gemm_kernel (gate/up + down launches)",
+                 "algorithmic_per_step": alg["gemm_bytes"] if roof["bound"] == "hbm" else alg["gemm_flops"],
+                 "ms_per_step": gemm_ms, "peak_source": f"{peak_src}" + (" sustained" if sustained and roof["bound"] == "tensor" else "")})
+
+    # ---- end to end through the public API with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(wl.T, wl.d_model, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    E2E = max(1, args.e2e_steps)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        abi.moe_layer_forward(dims, x_dev, Wr, bias, alpha, W13p, W2p, y, ws, outs)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(E2E):
+        e2e_step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / E2E
+    if pg:
+        t = torch.tensor([ms_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    launches = abi.moe_layer_launch_count(dims, True, bias is not None and alpha != 0.0) * K
+
+    cpu = None
+    if host_w is not None:
+        S = min(args.cpu_sample_tokens, wl.T)
+        tokens = np.linspace(0, wl.T - 1, S).astype(int).tolist()
+        b32 = np.zeros(E, np.float32) if wl.use_bias else None
+        times = time_oracle(wl, *host_w, tokens, b32, steps=2)
+        sec = min(times)
+        cpu = {"value": S / sec, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{S} of {wl.T} tokens (routing over all {wl.T}), best of 2 runs of {sec:.1f}-"
+                         f"{max(times):.1f} s"}
+
+    if pg:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    value = wl.T * world / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
+                   "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (expert weights %.2f GB)" % (wl.E * 3 * wl.d_model * wl.d_ff * 2 / 1e9)},
+        "roofline": roof,
+        "layer_roofline": {"bound": layer_bound, "t_roof_ms": max(t_bytes, t_flops) * 1e3, "t_meas_ms": ms_step,
+                           "frac": max(t_bytes, t_flops) * 1e3 / ms_step, "bytes": alg["layer_bytes"],
+                           "flops": alg["layer_flops"]},
+        "stage_ms": {"route": stage_ms[0], "dispatch": stage_ms[1], "gemm_gate_up": stage_ms[2],
+                     "gemm_down": stage_ms[3], "combine_stats": stage_ms[4]},
+        "routing": {"n_kept": alg["n_kept"], "experts_touched": alg["touched"],
+                    "max_over_mean_load": float(counts.max() / (wl.T * wl.K / wl.E)),
+                    "count_cv": float(counts.std() / counts.mean()), "n_dropped": int(outs["n_dropped"].item())},
+        "cpu_baseline": cpu,
+        "e2e": {"value": wl.T * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,231 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) Mixture-of-Experts layer library.
+ *
+ * One MoE FFN layer forward pass on one GPU, in five steps:
+ *   route    logits = x . W_r (+ bias), top-K, softmax over the K kept logits
+ *   permute  group the (token, slot) assignments by expert (histogram, scan,
+ *            stable token-order ranks, capacity drop, row gather)
+ *   expert   per expert: H = silu(X W1) * (X W3); Y = H W2  (tcgen05 GEMMs)
+ *   combine  y[t] = sum_k w[t,k] * Y[row(t,k)]  (deterministic gather)
+ *   stats    counts, f_i, P_i, aux = E * sum f_i P_i; aux-free bias update
+ *
+ * Sources (web pages; cited by title and section):
+ *   [P1] "MoE serving essay", dpshk.com/news/3211971
+ *   [P2] "MoE computation notes", cf-1.com/news/5905749
+ *   [P3] "MoE inference engineering in practice", ybb.press/quantum-computing/18594
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers to memory the caller owns; the
+ *     library allocates nothing on these paths and keeps no pointer after a
+ *     call returns.  Scratch space is the caller's workspace (`ws`, sized by
+ *     moe_workspace_size).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns; results are ready when the stream
+ *     reaches that point.  No call synchronises the device.
+ *   - Layouts are dense row-major.  bf16 values are passed as their 16-bit
+ *     patterns (moe_bf16).  Pointers must be 16-byte aligned; d_model and
+ *     d_ff must be multiples of 16.
+ *   - Status codes are returned (MOE_OK = 0, negative on error); nothing is
+ *     thrown across the ABI and a failed argument check enqueues no work.
+ *     Device-side failures (a bounded wait that ran out) set a flag in the
+ *     workspace that moe_get_device_status reads.
+ *   - Inputs must be finite; NaN or Inf in x or the weights gives unspecified
+ *     routing.
+ *   - Limits: 1 <= K <= E <= 256, 1 <= T <= 2^24.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16; /* bfloat16 bit pattern */
+
+/* Problem statement of one layer call ([P2] section 3.1 names T, K, E and the
+ * capacity factor; [P2] section 2 names d_model; the FFN width is d_ff).
+ *   T                 tokens in the batch, exactly (no padding tokens: [P2]
+ *                     section 4.3 warns that padded tokens get routed too)
+ *   d_model, d_ff     hidden and expert FFN widths
+ *   E, K              experts and experts per token
+ *   capacity_factor   <= 0: no per-expert limit.  Otherwise each expert keeps
+ *                     at most C = ceil(capacity_factor * T * K / E) assignments
+ *                     (the ceiling of the exact value of the double), the
+ *                     earliest tokens first ([P2] section 3.1). */
+typedef struct moe_dims {
+    int64_t T;
+    int32_t d_model;
+    int32_t d_ff;
+    int32_t E;
+    int32_t K;
+    double capacity_factor;
+} moe_dims;
+
+enum {
+    MOE_OK = 0,
+    MOE_EINVAL = -1,       /* bad argument: NULL where required, size out of range */
+    MOE_EUNSUPPORTED = -2, /* valid but not supported by this build (alignment, widths) */
+    MOE_ECUDA = -3,        /* a CUDA runtime call failed (launch error, no device) */
+    MOE_EWORKSPACE = -4,   /* workspace too small */
+    MOE_ETIMEOUT = -5,     /* a device-side bounded wait ran out (from moe_get_device_status) */
+};
+
+/* Human-readable name of a status code.  Never NULL. */
+MOE_API const char* moe_status_str(int status);
+
+/* Library ABI version (major * 100 + minor). */
+MOE_API int moe_version(void);
+
+/* Capacity C of [P2] section 3.1 for these dims: -1 when there is no limit,
+ * else ceil(capacity_factor * T * K / E) >= 1.  Returns < -1 on bad dims. */
+MOE_API int64_t moe_capacity(const moe_dims* dims);
+
+/* Bytes of device workspace that moe_layer_forward and the step entry points
+ * need for these dims.  *bytes receives the size.  Host only. */
+MOE_API int moe_workspace_size(const moe_dims* dims, size_t* bytes);
+
+/* Zero the workspace's device status flag (enqueued on `stream`). */
+MOE_API int moe_reset_device_status(void* ws, void* stream);
+
+/* Read the workspace's device status flag: synchronises `stream`, then
+ * *status = MOE_OK, or MOE_ETIMEOUT with *detail naming the wait that ran
+ * out (a small integer; 0 if none). */
+MOE_API int moe_get_device_status(const void* ws, void* stream, int* status, int* detail);
+
+/* One-time re-layout of the expert weights for the tensor-core GEMMs.
+ *   W1, W3  [E, d_model, d_ff]   (x . W1 is the gate, x . W3 the up projection)
+ *   W2      [E, d_ff, d_model]   (down projection)
+ *   W13p    [E, 2*d_ff, d_model] out: rows 32b..32b+15 are W1[:, 16b..16b+15]^T,
+ *                                rows 32b+16..32b+31 are W3[:, 16b..16b+15]^T
+ *   W2p     [E, d_model, d_ff]   out: W2^T per expert
+ * The expert FFN is the SwiGLU form y = (silu(x W1) * (x W3)) W2 ([P2]
+ * section 2: each expert is an FFN).  This is a load-time step, outside the
+ * per-batch path; the caller may free W1/W3/W2 afterwards. */
+MOE_API int moe_pack_weights(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3,
+                     const moe_bf16* W2, moe_bf16* W13p, moe_bf16* W2p, void* stream);
+
+/* Step 1+2: router logits, top-K and renormalisation ([P2] sections 1.2, 2
+ * and 2.1; [P3] sections 1 and 1.2).
+ *   x          [T, d_model] bf16 tokens
+ *   Wr         [d_model, E] bf16 router weight
+ *   bias       [E] fp32 or NULL: added (in fp32) to the logits before
+ *              selection; the weights use the biased logits too
+ *   logits     [T, E] fp32 out (unbiased logits) or NULL
+ *   topk_idx   [T, K] int32 out: selected experts, descending biased logit,
+ *              equal values ranked by lower expert index
+ *   topk_w     [T, K] fp32 out: softmax over the K selected (biased) logits
+ *   prob_mean  [E] fp32 out or NULL: P_i = mean over tokens of the full
+ *              softmax of the unbiased logits ([P2] section 1.2)
+ *   ws         workspace of at least ws_bytes = moe_workspace_size bytes */
+MOE_API int moe_route(const moe_dims* dims, const moe_bf16* x, const moe_bf16* Wr, const float* bias,
+              float* logits, int32_t* topk_idx, float* topk_w, float* prob_mean,
+              void* ws, size_t ws_bytes, void* stream);
+
+/* Step 2 alone, from given fp32 logits [T, E] (same outputs and rules as
+ * moe_route).  Lets the selection be checked bit for bit on logits both
+ * sides share.  prob_mean may be NULL. */
+MOE_API int moe_route_from_logits(const moe_dims* dims, const float* logits, const float* bias,
+                          int32_t* topk_idx, float* topk_w, float* prob_mean,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Step 3: dispatch ([P2] section 2.1: group by expert via sort and cumsum;
+ * section 3.1: capacity drop).
+ *   topk_idx  [T, K] int32 in
+ *   x         [T, d_model] bf16 in, or NULL to skip the row gather
+ *   counts    [E] int32 out: selections per expert before drops
+ *   kept      [E] int32 out: min(counts, C)
+ *   offsets   [E+1] int32 out: exclusive cumsum of kept (offsets[E] = N_kept)
+ *   inv       [T, K] int32 out: row of (t, k) in x_perm, or -1 if dropped
+ *   src       [T*K] int32 out: token of each row (rows >= N_kept untouched)
+ *   x_perm    [T*K, d_model] bf16 out (rows >= N_kept untouched), or NULL
+ *   n_dropped [1] int32 out or NULL
+ * The rank of (t, k) within its expert is the number of tokens t' < t that
+ * chose the same expert; rows are expert-major, token-ascending. */
+MOE_API int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x,
+                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
+                moe_bf16* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 4: grouped SwiGLU expert FFN on the rows of each expert ([P2]
+ * section 2 step 3; section 2.2: experts only see their own tokens).
+ *   x_perm   [T*K, d_model] bf16 in (rows 0..offsets[E]-1 are used)
+ *   offsets  [E+1] int32 in (device; read by the kernels, never by the host)
+ *   W13p, W2p packed weights from moe_pack_weights
+ *   h        [T*K, d_ff] bf16 out: silu(X W1) * (X W3) rounded to bf16
+ *   y_perm   [T*K, d_model] fp32 out: h W2, fp32 accumulation */
+MOE_API int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets,
+                   const moe_bf16* W13p, const moe_bf16* W2p, moe_bf16* h, float* y_perm,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* Step 5: combine ([P2] section 2 step 4 and section 2.3: weighted sum back
+ * in token order; section 2.2: unselected experts add nothing).
+ *   y[t] = sum_{k=0..K-1, inv[t,k] >= 0} topk_w[t,k] * y_perm[inv[t,k]]
+ * summed in k order in fp32; a dropped slot adds nothing and the remaining
+ * weights are not renormalised.  y [T, d_model] fp32 out. */
+MOE_API int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* inv,
+                const float* topk_w, float* y, void* stream);
+
+/* Load statistics ([P2] section 1.2): f_i = counts_i / (T K),
+ * P_i = prob_mean_i, aux = E * sum_i f_i P_i.  Any output may be NULL. */
+MOE_API int moe_load_stats(const moe_dims* dims, const int32_t* counts, const float* prob_mean,
+                   float* f, float* aux, void* stream);
+
+/* Aux-free bias update ([P3] section 1.2): for each expert, b -= alpha if
+ * counts*E > T*K (above the target load T*K/E), b += alpha if below,
+ * unchanged if equal.  One fp32 add per expert; bias [E] fp32 in/out. */
+MOE_API int moe_bias_update(const moe_dims* dims, const int32_t* counts, float alpha, float* bias,
+                    void* stream);
+
+/* Optional outputs of moe_layer_forward: device pointers, each may be NULL
+ * (the value then stays in the workspace). */
+typedef struct moe_layer_outputs {
+    int32_t* topk_idx;  /* [T, K] */
+    float* topk_w;      /* [T, K] */
+    float* logits;      /* [T, E] unbiased */
+    int32_t* counts;    /* [E] before drops */
+    int32_t* kept;      /* [E] */
+    int32_t* offsets;   /* [E+1] */
+    int32_t* inv;       /* [T, K] */
+    int32_t* n_dropped; /* [1] */
+    float* f;           /* [E] */
+    float* P;           /* [E] */
+    float* aux;         /* [1] */
+    /* Caller-created CUDA events (cudaEvent_t), or NULL.  When set, the
+     * layer records, on `stream`: [0] before routing, [1] after routing,
+     * [2] after dispatch, [3] after the gate/up GEMM, [4] after the down
+     * GEMM, [5] after combine and statistics.  For per-stage timing. */
+    void* const* stage_events; /* [MOE_NUM_STAGE_EVENTS] */
+} moe_layer_outputs;
+
+#define MOE_NUM_STAGE_EVENTS 6
+
+/* Number of kernel launches one moe_layer_forward call enqueues for these
+ * dims and options (stats = P_i / f_i / aux requested, bias_update = bias
+ * non-NULL and alpha != 0).  Host only; < 0 on bad dims. */
+MOE_API int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update);
+
+/* The whole layer: route -> permute -> expert FFN -> combine (-> stats, bias
+ * update), all enqueued on `stream` with no host synchronisation.
+ *   x [T, d_model] bf16, Wr [d_model, E] bf16, W13p/W2p from moe_pack_weights
+ *   bias  [E] fp32 or NULL; if non-NULL and alpha != 0 it is updated in place
+ *         after routing (so the routing of this call uses the old value)
+ *   y     [T, d_model] fp32 out
+ *   out   optional extra outputs (NULL = none)
+ * [P1] section 2 lists the same sequence: score, select, dispatch, expert
+ * FFN, gather back. */
+MOE_API int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* Wr, float* bias,
+                      float alpha, const moe_bf16* W13p, const moe_bf16* W2p, float* y,
+                      const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

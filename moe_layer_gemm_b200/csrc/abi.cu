@@ -1,0 +1,441 @@
+// C ABI of the MoE layer library: argument checks, the workspace layout and
+// the order of kernel launches.  All compute is in the other .cu files.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/moe_b200.h"
+#include "internal.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kVersion = 100;
+constexpr int64_t kMaxT = int64_t(1) << 24;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const moe_dims* d) {
+    if (!d) return MOE_EINVAL;
+    if (d->T < 1 || d->T > kMaxT) return MOE_EINVAL;
+    if (d->E < 1 || d->E > 256) return MOE_EINVAL;
+    if (d->K < 1 || d->K > d->E || d->K > 16) return MOE_EINVAL;
+    if (d->d_model < 16 || d->d_ff < 16) return MOE_EINVAL;
+    if (d->d_model > (1 << 16) || d->d_ff > (1 << 17)) return MOE_EINVAL;
+    if (d->d_model % 16 != 0 || d->d_ff % 16 != 0) return MOE_EUNSUPPORTED;
+    if (std::isnan(d->capacity_factor)) return MOE_EINVAL;
+    return MOE_OK;
+}
+
+// C = ceil(cf * T * K / E) on the exact binary value of cf; -1 = no limit.
+int64_t capacity_of(const moe_dims* d) {
+    const double cf = d->capacity_factor;
+    if (!(cf > 0.0)) return -1;
+    if (std::isinf(cf)) return INT64_MAX / 2;
+    int ex = 0;
+    const double m = std::frexp(cf, &ex);                    // cf = m * 2^ex, m in [0.5, 1)
+    const __int128 mant = static_cast<__int128>(std::ldexp(m, 53));  // exact 53-bit integer
+    const int p = ex - 53;                                    // cf = mant * 2^p
+    __int128 num = mant * static_cast<__int128>(d->T) * d->K;
+    __int128 den = d->E;
+    if (p >= 0) {
+        if (p > 40) return INT64_MAX / 2;
+        num <<= p;
+    } else {
+        if (-p > 100) return 1;  // value < 2^-15: ceil is 1
+        den <<= -p;
+    }
+    __int128 c = (num + den - 1) / den;
+    if (c > INT64_MAX / 2) return INT64_MAX / 2;
+    return static_cast<int64_t>(c);
+}
+
+struct Layout {
+    size_t status, idx, w, logits, counts, kept, offsets, ndrop, prob_part, prob_mean, f, aux, block_hist, inv,
+        src, xperm, h, yperm, wrt, total;
+    int route_nb, perm_nb, nsplit, E_pad, swap;
+    bool fused_router;
+};
+
+// Weight rows of one group on the MMA M side pay off when groups are small.
+int choose_swap(const moe_dims* d) {
+    const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
+    return (avg <= 96 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
+}
+
+// Split of the down projection's reduction that keeps the last wave full.
+int choose_nsplit(const moe_dims* d, int swap) {
+    if (!swap) return 1;
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    const int64_t rows = d->T * d->K;
+    const int64_t chunk = 128;
+    const int64_t tiles = std::min<int64_t>((rows + chunk - 1) / chunk + d->E, d->E * ((d->T + chunk - 1) / chunk)) *
+                          (d->d_model / 128);
+    const int kblocks = (d->d_ff + 63) / 64;
+    int best = 1;
+    double best_eff = 0.0;
+    for (int ks = 1; ks <= 8 && ks <= kblocks; ++ks) {
+        const int64_t units = tiles * ks;
+        const int64_t rounds = (units + sms - 1) / sms;
+        double eff = static_cast<double>(units) / static_cast<double>(rounds * sms);
+        if (units < sms) eff *= 0.999;  // fewer units than SMs: never fills the machine
+        if (eff > best_eff + 0.02) {
+            best_eff = eff;
+            best = ks;
+        }
+    }
+    return best;
+}
+
+Layout layout_of(const moe_dims* d) {
+    Layout L{};
+    const int64_t T = d->T, E = d->E, K = d->K, D = d->d_model, F = d->d_ff;
+    const int64_t A = T * K;
+    L.route_nb = route_blocks(T);
+    L.perm_nb = permute_blocks(T);
+    L.fused_router = route_fused_supported(d->d_model, d->E) != 0;
+    L.E_pad = static_cast<int>(((E + 31) / 32) * 32);
+    L.swap = choose_swap(d);
+    L.nsplit = choose_nsplit(d, L.swap);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align256(o + bytes);
+        return at;
+    };
+    L.status = take(64);
+    L.idx = take(A * 4);
+    L.w = take(A * 4);
+    L.logits = take(T * E * 4);
+    L.counts = take(E * 4);
+    L.kept = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.ndrop = take(4);
+    L.prob_part = take(static_cast<size_t>(L.route_nb) * E * 4);
+    L.prob_mean = take(E * 4);
+    L.f = take(E * 4);
+    L.aux = take(4);
+    L.block_hist = take(static_cast<size_t>(L.perm_nb) * E * 4);
+    L.inv = take(A * 4);
+    L.src = take(A * 4);
+    L.xperm = take(A * D * 2);
+    L.h = take(A * F * 2);
+    L.yperm = take(static_cast<size_t>(L.nsplit) * A * D * 4);
+    L.wrt = take(static_cast<size_t>(L.E_pad) * D * 2);
+    L.total = o;
+    return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int map_launch(int r) {
+    if (r == 0) return MOE_OK;
+    if (r == -2) return MOE_EUNSUPPORTED;
+    return MOE_ECUDA;
+}
+
+int check_ws(const moe_dims* d, void* ws, size_t ws_bytes) {
+    if (!ws || !aligned16(ws)) return MOE_EINVAL;
+    if (ws_bytes < layout_of(d).total) return MOE_EWORKSPACE;
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)               \
+    do {                            \
+        int _s = (expr);            \
+        if (_s != MOE_OK) return _s; \
+    } while (0)
+
+int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, const float* bias, float* logits,
+             int32_t* idx, float* w, float* prob_mean, void* ws, cudaStream_t st) {
+    float* part = prob_mean ? at<float>(ws, L.prob_part) : nullptr;
+    if (L.fused_router) {
+        MOE_TRY(map_launch(launch_route_fused(x, Wr, bias, d->T, d->d_model, d->E, d->K, logits, idx, w, part,
+                                              L.route_nb, st)));
+    } else {
+        float* lg = logits ? logits : at<float>(ws, L.logits);
+        bf16* wrt = at<bf16>(ws, L.wrt);
+        MOE_TRY(map_launch(launch_transpose_router(Wr, d->d_model, d->E, L.E_pad, wrt, st)));
+        GemmLaunch g{};
+        g.tok = x;
+        g.tok_rows = d->T;
+        g.w = wrt;
+        g.G = 1;
+        g.N = L.E_pad;
+        g.N_store = d->E;
+        g.Kdim = d->d_model;
+        g.group_off = nullptr;
+        g.dense_rows = d->T;
+        g.max_group_rows = d->T;
+        g.swap = 0;
+        g.ksplit = 1;
+        g.epi = EPI_F32;
+        g.out = lg;
+        g.ldo = d->E;
+        g.split_stride = 0;
+        g.status = at<int>(ws, L.status);
+        MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
+        MOE_TRY(map_launch(launch_topk_from_logits(lg, bias, d->T, d->E, d->K, idx, w, part, L.route_nb, st)));
+    }
+    if (prob_mean) MOE_TRY(map_launch(launch_prob_finalize(part, L.route_nb, d->E, d->T, prob_mean, st)));
+    return MOE_OK;
+}
+
+template <typename Mid>
+int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
+           const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st, Mid between) {
+    const int64_t A = d->T * d->K;
+    int64_t maxrows = d->T;
+    const int64_t C = capacity_of(d);
+    if (C >= 0 && C < maxrows) maxrows = C;
+    GemmLaunch g{};
+    g.tok = xperm;
+    g.tok_rows = A;
+    g.w = W13p;
+    g.G = d->E;
+    g.N = 2 * d->d_ff;
+    g.N_store = 2 * d->d_ff;
+    g.Kdim = d->d_model;
+    g.group_off = offsets;
+    g.dense_rows = 0;
+    g.max_group_rows = maxrows;
+    g.swap = L.swap;
+    g.ksplit = 1;
+    g.epi = EPI_SWIGLU_BF16;
+    g.out = h;
+    g.ldo = d->d_ff;
+    g.split_stride = 0;
+    g.status = at<int>(ws, L.status);
+    MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
+    between();
+    GemmLaunch g2 = g;
+    g2.tok = h;
+    g2.w = W2p;
+    g2.N = d->d_model;
+    g2.N_store = d->d_model;
+    g2.Kdim = d->d_ff;
+    g2.ksplit = nsplit;
+    g2.epi = EPI_F32;
+    g2.out = yout;
+    g2.ldo = d->d_model;
+    g2.split_stride = A * d->d_model;
+    MOE_TRY(map_launch(launch_grouped_gemm(g2, st)));
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(int s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_EINVAL: return "MOE_EINVAL: invalid argument";
+        case MOE_EUNSUPPORTED: return "MOE_EUNSUPPORTED: unsupported shape or alignment";
+        case MOE_ECUDA: return "MOE_ECUDA: CUDA runtime error";
+        case MOE_EWORKSPACE: return "MOE_EWORKSPACE: workspace too small";
+        case MOE_ETIMEOUT: return "MOE_ETIMEOUT: a device-side wait ran out";
+        default: return "unknown status";
+    }
+}
+
+int moe_version(void) { return kVersion; }
+
+int64_t moe_capacity(const moe_dims* dims) {
+    if (check_dims(dims) != MOE_OK) return -2;
+    return capacity_of(dims);
+}
+
+int moe_workspace_size(const moe_dims* dims, size_t* bytes) {
+    MOE_TRY(check_dims(dims));
+    if (!bytes) return MOE_EINVAL;
+    *bytes = layout_of(dims).total;
+    return MOE_OK;
+}
+
+int moe_reset_device_status(void* ws, void* stream) {
+    if (!ws) return MOE_EINVAL;
+    return cudaMemsetAsync(ws, 0, 64, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+int moe_get_device_status(const void* ws, void* stream, int* status, int* detail) {
+    if (!ws || !status) return MOE_EINVAL;
+    int host = 0;
+    if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream)) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MOE_ECUDA;
+    *status = host == 0 ? MOE_OK : MOE_ETIMEOUT;
+    if (detail) *detail = host;
+    return MOE_OK;
+}
+
+int moe_pack_weights(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                     moe_bf16* W13p, moe_bf16* W2p, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!W1 || !W3 || !W2 || !W13p || !W2p) return MOE_EINVAL;
+    if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(W13p) || !aligned16(W2p))
+        return MOE_EUNSUPPORTED;
+    return map_launch(launch_pack(reinterpret_cast<const bf16*>(W1), reinterpret_cast<const bf16*>(W3),
+                                  reinterpret_cast<const bf16*>(W2), dims->E, dims->d_model, dims->d_ff,
+                                  reinterpret_cast<bf16*>(W13p), reinterpret_cast<bf16*>(W2p),
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route(const moe_dims* dims, const moe_bf16* x, const moe_bf16* Wr, const float* bias, float* logits,
+              int32_t* topk_idx, float* topk_w, float* prob_mean, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!x || !Wr || !topk_idx || !topk_w) return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(Wr)) return MOE_EUNSUPPORTED;
+    MOE_TRY(check_ws(dims, ws, ws_bytes));
+    const Layout L = layout_of(dims);
+    return do_route(dims, L, reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(Wr), bias, logits,
+                    topk_idx, topk_w, prob_mean, ws, static_cast<cudaStream_t>(stream));
+}
+
+int moe_route_from_logits(const moe_dims* dims, const float* logits, const float* bias, int32_t* topk_idx,
+                          float* topk_w, float* prob_mean, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!logits || !topk_idx || !topk_w) return MOE_EINVAL;
+    MOE_TRY(check_ws(dims, ws, ws_bytes));
+    const Layout L = layout_of(dims);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* part = prob_mean ? at<float>(ws, L.prob_part) : nullptr;
+    MOE_TRY(map_launch(launch_topk_from_logits(logits, bias, dims->T, dims->E, dims->K, topk_idx, topk_w, part,
+                                               L.route_nb, st)));
+    if (prob_mean) MOE_TRY(map_launch(launch_prob_finalize(part, L.route_nb, dims->E, dims->T, prob_mean, st)));
+    return MOE_OK;
+}
+
+int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x, int32_t* counts, int32_t* kept,
+                int32_t* offsets, int32_t* inv, int32_t* src, moe_bf16* x_perm, int32_t* n_dropped, void* ws,
+                size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!topk_idx || !counts || !kept || !offsets || !inv || !src) return MOE_EINVAL;
+    if ((x == nullptr) != (x_perm == nullptr)) return MOE_EINVAL;
+    if (x && (!aligned16(x) || !aligned16(x_perm))) return MOE_EUNSUPPORTED;
+    MOE_TRY(check_ws(dims, ws, ws_bytes));
+    const Layout L = layout_of(dims);
+    return map_launch(launch_permute(topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model, dims->E,
+                                     dims->K, capacity_of(dims), at<int32_t>(ws, L.block_hist), counts, kept,
+                                     offsets, inv, src, reinterpret_cast<bf16*>(x_perm), n_dropped,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets, const moe_bf16* W13p,
+                   const moe_bf16* W2p, moe_bf16* h, float* y_perm, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!x_perm || !offsets || !W13p || !W2p || !h || !y_perm) return MOE_EINVAL;
+    if (!aligned16(x_perm) || !aligned16(W13p) || !aligned16(W2p) || !aligned16(h) || !aligned16(y_perm))
+        return MOE_EUNSUPPORTED;
+    MOE_TRY(check_ws(dims, ws, ws_bytes));
+    const Layout L = layout_of(dims);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* yout = L.nsplit > 1 ? at<float>(ws, L.yperm) : y_perm;
+    MOE_TRY(do_ffn(dims, L, reinterpret_cast<const bf16*>(x_perm), offsets, reinterpret_cast<const bf16*>(W13p),
+                   reinterpret_cast<const bf16*>(W2p), reinterpret_cast<bf16*>(h), yout, L.nsplit, ws, st,
+                   []() {}));
+    if (L.nsplit > 1)
+        MOE_TRY(map_launch(launch_reduce_splits(yout, L.nsplit, dims->T * dims->K * dims->d_model, offsets, dims->E,
+                                                dims->d_model, y_perm, st)));
+    return MOE_OK;
+}
+
+int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* inv, const float* topk_w, float* y,
+                void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!y_perm || !inv || !topk_w || !y) return MOE_EINVAL;
+    if (!aligned16(y_perm) || !aligned16(y)) return MOE_EUNSUPPORTED;
+    return map_launch(launch_combine(y_perm, 1, 0, inv, topk_w, dims->T, dims->d_model, dims->K, y,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int moe_load_stats(const moe_dims* dims, const int32_t* counts, const float* prob_mean, float* f, float* aux,
+                   void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!counts) return MOE_EINVAL;
+    if (aux && !prob_mean) return MOE_EINVAL;
+    return map_launch(launch_stats(counts, prob_mean, dims->T, dims->E, dims->K, f, aux, nullptr,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int moe_bias_update(const moe_dims* dims, const int32_t* counts, float alpha, float* bias, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!counts || !bias) return MOE_EINVAL;
+    if (!std::isfinite(alpha)) return MOE_EINVAL;
+    return map_launch(launch_bias_update(counts, dims->T, dims->E, dims->K, alpha, bias,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* Wr, float* bias, float alpha,
+                      const moe_bf16* W13p, const moe_bf16* W2p, float* y, const moe_layer_outputs* out,
+                      void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!x || !Wr || !W13p || !W2p || !y) return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(Wr) || !aligned16(W13p) || !aligned16(W2p) || !aligned16(y))
+        return MOE_EUNSUPPORTED;
+    if (!std::isfinite(alpha)) return MOE_EINVAL;
+    MOE_TRY(check_ws(dims, ws, ws_bytes));
+    const Layout L = layout_of(dims);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    moe_layer_outputs o{};
+    if (out) o = *out;
+    int32_t* idx = o.topk_idx ? o.topk_idx : at<int32_t>(ws, L.idx);
+    float* w = o.topk_w ? o.topk_w : at<float>(ws, L.w);
+    int32_t* counts = o.counts ? o.counts : at<int32_t>(ws, L.counts);
+    int32_t* kept = o.kept ? o.kept : at<int32_t>(ws, L.kept);
+    int32_t* offsets = o.offsets ? o.offsets : at<int32_t>(ws, L.offsets);
+    int32_t* inv = o.inv ? o.inv : at<int32_t>(ws, L.inv);
+    int32_t* ndrop = o.n_dropped ? o.n_dropped : at<int32_t>(ws, L.ndrop);
+    const bool want_stats = o.P || o.aux || o.f;
+    float* P = o.P ? o.P : at<float>(ws, L.prob_mean);
+    const bf16* xb = reinterpret_cast<const bf16*>(x);
+
+    auto mark = [&](int i) {
+        if (o.stage_events && o.stage_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(o.stage_events[i]), st);
+    };
+    mark(0);
+    MOE_TRY(do_route(dims, L, xb, reinterpret_cast<const bf16*>(Wr), bias, o.logits, idx, w,
+                     want_stats ? P : nullptr, ws, st));
+    mark(1);
+    MOE_TRY(map_launch(launch_permute(idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
+                                      at<int32_t>(ws, L.block_hist), counts, kept, offsets, inv,
+                                      at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop, st)));
+    mark(2);
+    float* yp = at<float>(ws, L.yperm);
+    MOE_TRY(do_ffn(dims, L, at<bf16>(ws, L.xperm), offsets, reinterpret_cast<const bf16*>(W13p),
+                   reinterpret_cast<const bf16*>(W2p), at<bf16>(ws, L.h), yp, L.nsplit, ws, st,
+                   [&]() { mark(3); }));
+    mark(4);
+    MOE_TRY(map_launch(launch_combine(yp, L.nsplit, dims->T * dims->K * dims->d_model, inv, w, dims->T,
+                                      dims->d_model, dims->K, y, st)));
+    if (want_stats || o.f)
+        MOE_TRY(map_launch(launch_stats(counts, want_stats ? P : nullptr, dims->T, dims->E, dims->K, o.f, o.aux,
+                                        nullptr, st)));
+    if (bias && alpha != 0.0f)
+        MOE_TRY(map_launch(launch_bias_update(counts, dims->T, dims->E, dims->K, alpha, bias, st)));
+    mark(5);
+    return MOE_OK;
+}
+
+int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update) {
+    if (check_dims(dims) != MOE_OK) return -1;
+    const Layout L = layout_of(dims);
+    int n = L.fused_router ? 1 : 3;  // fused router, or transpose + logits GEMM + top-K
+    if (stats) n += 1;               // P_i finalize
+    n += 4;                          // histogram, scan, rank, gather
+    n += 2;                          // gate/up GEMM, down GEMM
+    n += 1;                          // combine
+    if (stats) n += 1;               // f_i and aux
+    if (bias_update) n += 1;
+    return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+// Combine, load statistics and the aux-free bias update.
+//
+// Combine: "MoE computation notes" (cf-1.com/news/5905749), section 2 step 4
+// and section 2.3: the output is the weighted sum of the K experts' outputs,
+// put back in token order; section 2.2: unselected experts add nothing.  A
+// deterministic gather: one CTA per token reads its K rows (skipping
+// dropped slots) and sums them in slot order in fp32; no atomics.  When the
+// expert GEMM split its reduction, the partial slices are summed here first,
+// in slice order.
+//
+// Statistics: same notes, section 1.2: aux = N * sum_i f_i * P_i.
+// Bias: "MoE inference engineering in practice"
+// (ybb.press/quantum-computing/18594), section 1.2: overloaded experts get
+// bias -= alpha, underloaded bias += alpha.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaxK = 16;
+
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, const int32_t* __restrict__ inv,
+               const float* __restrict__ w, int64_t T, int d, int K, float* __restrict__ y) {
+    const int nvec = d / 4;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        int32_t rows[kMaxK];
+        float ws[kMaxK];
+        for (int k = 0; k < K; ++k) {
+            rows[k] = inv[t * K + k];
+            ws[k] = w[t * K + k];
+        }
+        for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 0; k < K; ++k) {
+                if (rows[k] < 0) continue;
+                const float* base = yp + static_cast<int64_t>(rows[k]) * d;
+                float4 v = reinterpret_cast<const float4*>(base)[c];
+                for (int s = 1; s < nsplit; ++s) {
+                    const float4 u = reinterpret_cast<const float4*>(base + s * split_stride)[c];
+                    v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+                }
+                acc.x = fmaf(ws[k], v.x, acc.x);
+                acc.y = fmaf(ws[k], v.y, acc.y);
+                acc.z = fmaf(ws[k], v.z, acc.z);
+                acc.w = fmaf(ws[k], v.w, acc.w);
+            }
+            reinterpret_cast<float4*>(y + t * d)[c] = acc;
+        }
+    }
+}
+
+// y_perm[r] = sum over slices s of part[s][r], rows r < offsets[E].
+__global__ void __launch_bounds__(256)
+reduce_splits_kernel(const float* __restrict__ part, int nsplit, int64_t split_stride,
+                     const int32_t* __restrict__ offsets, int E, int d, float* __restrict__ out) {
+    const int64_t n = static_cast<int64_t>(offsets[E]) * (d / 4);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float4 v = reinterpret_cast<const float4*>(part)[i];
+        for (int s = 1; s < nsplit; ++s) {
+            const float4 u = reinterpret_cast<const float4*>(part + s * split_stride)[i];
+            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
+        reinterpret_cast<float4*>(out)[i] = v;
+    }
+}
+
+// One block: f_i = counts_i / (T K); aux = E * sum_i f_i P_i (fixed-order tree).
+__global__ void __launch_bounds__(256)
+stats_kernel(const int32_t* __restrict__ counts, const float* __restrict__ P, int64_t T, int E, int K,
+             float* __restrict__ f, float* __restrict__ aux) {
+    __shared__ float red[256];
+    const float inv = 1.0f / static_cast<float>(T * K);
+    float part = 0.f;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const float fe = static_cast<float>(counts[e]) * inv;
+        if (f) f[e] = fe;
+        if (P) part += fe * P[e];
+    }
+    red[threadIdx.x] = part;
+    __syncthreads();
+    for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+        if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
+}
+
+__global__ void bias_update_kernel(const int32_t* __restrict__ counts, int64_t TK, int E, float alpha,
+                                   float* __restrict__ bias) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    const int64_t lhs = static_cast<int64_t>(counts[e]) * E;
+    float b = bias[e];
+    if (lhs > TK) b = __fsub_rn(b, alpha);
+    else if (lhs < TK) b = __fadd_rn(b, alpha);
+    bias[e] = b;
+}
+
+// W13p[e][32b + j][k] = (j < 16 ? W1 : W3)[e][k][16b + (j & 15)];  W2p[e][n][k] = W2[e][k][n].
+// Both are [rows][cols] <- transpose of a [cols][rows]-shaped source, by
+// 32 x 32 tiles through shared memory.
+__global__ void pack_w13_kernel(const __nv_bfloat16* __restrict__ W1, const __nv_bfloat16* __restrict__ W3,
+                                int d, int f, __nv_bfloat16* __restrict__ W13p) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int e = blockIdx.z;
+    const int k0 = blockIdx.x * 32;  // d index
+    const int r0 = blockIdx.y * 32;  // packed row index (2f rows), one 32-row block = 16 gate + 16 up
+    const int b = r0 / 32;
+    const __nv_bfloat16* s1 = W1 + static_cast<int64_t>(e) * d * f;
+    const __nv_bfloat16* s3 = W3 + static_cast<int64_t>(e) * d * f;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int k = k0 + i;
+        const int j = threadIdx.x;
+        const int col = 16 * b + (j & 15);
+        __nv_bfloat16 v = __float2bfloat16_rn(0.f);
+        if (k < d) v = (j < 16 ? s1 : s3)[static_cast<int64_t>(k) * f + col];
+        tile[i][j] = v;
+    }
+    __syncthreads();
+    __nv_bfloat16* dst = W13p + static_cast<int64_t>(e) * 2 * f * d;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, k = k0 + threadIdx.x;
+        if (k < d) dst[static_cast<int64_t>(r) * d + k] = tile[threadIdx.x][i];
+    }
+}
+
+__global__ void pack_w2_kernel(const __nv_bfloat16* __restrict__ W2, int d, int f, __nv_bfloat16* __restrict__ W2p) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int e = blockIdx.z;
+    const int k0 = blockIdx.x * 32;  // f index (reduction of the down projection)
+    const int n0 = blockIdx.y * 32;  // d index (output rows of W2p)
+    const __nv_bfloat16* s = W2 + static_cast<int64_t>(e) * f * d;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int k = k0 + i, n = n0 + threadIdx.x;
+        tile[i][threadIdx.x] = (k < f && n < d) ? s[static_cast<int64_t>(k) * d + n] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    __nv_bfloat16* dst = W2p + static_cast<int64_t>(e) * d * f;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int n = n0 + i, k = k0 + threadIdx.x;
+        if (n < d && k < f) dst[static_cast<int64_t>(n) * f + k] = tile[threadIdx.x][i];
+    }
+}
+
+}  // namespace
+
+int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv, const float* w,
+                   int64_t T, int d, int K, float* y, cudaStream_t st) {
+    if (K > kMaxK || d % 4 != 0) return -2;
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    int64_t grid = T < static_cast<int64_t>(sms) * 16 ? T : static_cast<int64_t>(sms) * 16;
+    int threads = d / 4 >= 256 ? 256 : ((d / 4 + 31) / 32) * 32;
+    combine_kernel<<<static_cast<int>(grid < 1 ? 1 : grid), threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w,
+                                                                             T, d, K, y);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int launch_reduce_splits(const float* part, int nsplit, int64_t split_stride, const int32_t* offsets, int E, int d,
+                         float* y_perm, cudaStream_t st) {
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    reduce_splits_kernel<<<sms * 4, 256, 0, st>>>(part, nsplit, split_stride, offsets, E, d, y_perm);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E, int K, float* f, float* aux,
+                 const float*, cudaStream_t st) {
+    stats_kernel<<<1, 256, 0, st>>>(counts, prob_mean, T, E, K, f, aux);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias, cudaStream_t st) {
+    bias_update_kernel<<<(E + 255) / 256, 256, 0, st>>>(counts, T * K, E, alpha, bias);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int launch_pack(const bf16* W1, const bf16* W3, const bf16* W2, int E, int d, int f, bf16* W13p, bf16* W2p,
+                cudaStream_t st) {
+    dim3 block(32, 8);
+    dim3 g13((d + 31) / 32, (2 * f) / 32, E);
+    pack_w13_kernel<<<g13, block, 0, st>>>(W1, W3, d, f, W13p);
+    dim3 g2((f + 31) / 32, (d + 31) / 32, E);
+    pack_w2_kernel<<<g2, block, 0, st>>>(W2, d, f, W2p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+}  // namespace moe

@@ -1,0 +1,326 @@
+// Router: logits = x . W_r (+ bias), top-K selection and renormalisation.
+//
+// "MoE computation notes" (cf-1.com/news/5905749), section 1.2: the router
+// is one linear map from the hidden state to one score per expert;
+// section 2 steps 2-3 and section 2.1: keep the K best experts and weight
+// them by a softmax over the K kept scores.  "MoE inference engineering in
+// practice" (ybb.press/quantum-computing/18594), section 1: top-k on the
+// logits then softmax; section 1.2: route on gate(x) + bias.
+//
+// Small E (<= 32) with W_r fitting in shared memory: one warp per token.
+// Lanes stream the token's row with 16-byte loads, each lane keeps E partial
+// dot products, a butterfly reduction leaves all E logits in every lane, and
+// the top-K and the softmax over the kept logits run in registers.  Nothing
+// but the K indices and weights (and optionally the logits) is written.
+//
+// Large E: the logits come from the tensor-core GEMM (gemm.cu) and a
+// warp-per-token kernel selects from them (lane j owns experts j, j+32, ..).
+//
+// Ties: equal fp32 values rank the lower expert index first (-0.0 == +0.0).
+// The per-token full softmax of the unbiased logits is summed per block in a
+// fixed order for P_i; blocks' partial sums are added in block order later,
+// so the statistics are deterministic.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cfloat>
+
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteWarps = 8;
+
+// Warp-wide top-K over values v[j] of expert (lane + 32 j), j < J.
+// Returns, in lane r < K, the r-th selected (value, expert); other lanes get
+// (-inf, -1).  `valid[j]` marks real experts.
+template <int J>
+__device__ __forceinline__ void warp_topk(const float (&v)[J], const bool (&valid)[J], int K, int lane,
+                                          float& out_v, int& out_e) {
+    bool taken[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) taken[j] = !valid[j];
+    out_v = -FLT_MAX;
+    out_e = -1;
+    for (int r = 0; r < K; ++r) {
+        float bv = -FLT_MAX;
+        int be = 0x7fffffff;
+        bool have = false;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int e = lane + 32 * j;
+            if (!taken[j] && (!have || v[j] > bv)) {  // ascending j: ties keep the lower index
+                bv = v[j];
+                be = e;
+                have = true;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const bool ohave = __shfl_xor_sync(0xffffffffu, static_cast<int>(have), o) != 0;
+            if (ohave && (!have || ov > bv || (ov == bv && oe < be))) {
+                bv = ov;
+                be = oe;
+                have = true;
+            }
+        }
+        // every lane now holds the same winner
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            if (lane + 32 * j == be) taken[j] = true;
+        if (lane == r) {
+            out_v = bv;
+            out_e = be;
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+// Selection, weights and probability accumulation for one token whose
+// unbiased logits are l[j] (expert lane + 32 j).
+template <int J>
+__device__ __forceinline__ void finish_token(const float (&l)[J], const bool (&valid)[J], const float* bias,
+                                             int64_t t, int K, int lane, int32_t* idx, float* w,
+                                             float (&psum)[J], bool want_prob) {
+    if (want_prob) {
+        float m = -FLT_MAX;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            if (valid[j]) m = fmaxf(m, l[j]);
+        m = warp_max(m);
+        float p[J];
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            p[j] = valid[j] ? expf(l[j] - m) : 0.f;
+            s += p[j];
+        }
+        s = warp_sum(s);
+        const float inv = 1.0f / s;
+#pragma unroll
+        for (int j = 0; j < J; ++j) psum[j] += p[j] * inv;
+    }
+    float lb[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) lb[j] = (bias != nullptr && valid[j]) ? l[j] + bias[lane + 32 * j] : l[j];
+    float sv;
+    int se;
+    warp_topk<J>(lb, valid, K, lane, sv, se);
+    const float vmax = __shfl_sync(0xffffffffu, sv, 0);
+    const float ex = (lane < K) ? expf(sv - vmax) : 0.f;
+    const float den = warp_sum(ex);
+    if (lane < K) {
+        idx[t * K + lane] = se;
+        w[t * K + lane] = ex / den;
+    }
+}
+
+template <int J>
+__device__ __forceinline__ void write_prob_partials(const float (&psum)[J], int E, float* prob_part) {
+    __shared__ float sp[kRouteWarps][J * 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < J; ++j) sp[warp][lane + 32 * j] = psum[j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float s = 0.f;
+        for (int wi = 0; wi < kRouteWarps; ++wi) s += sp[wi][e];
+        prob_part[static_cast<int64_t>(blockIdx.x) * E + e] = s;
+    }
+}
+
+// Fused router for E <= 32.  W_r is staged in shared memory as [d][8*EV]
+// bf16 rows (zero-padded), EV = 16-byte vectors per row.
+template <int EV>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr,
+                   const float* __restrict__ bias, int64_t T, int d, int E, int K,
+                   float* __restrict__ logits, int32_t* __restrict__ idx, float* __restrict__ w,
+                   float* __restrict__ prob_part) {
+    constexpr int EP = EV * 8;  // padded experts per row
+    extern __shared__ uint4 swr_raw[];
+    __nv_bfloat16* swr = reinterpret_cast<__nv_bfloat16*>(swr_raw);
+    for (int i = threadIdx.x; i < d * EP; i += blockDim.x) {
+        const int r = i / EP, e = i - r * EP;
+        swr[i] = e < E ? Wr[static_cast<int64_t>(r) * E + e] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kRouteWarps;
+    float psum[1] = {0.f};
+    const bool want_prob = prob_part != nullptr;
+    const int nvec = d / 8;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps + warp; t < T; t += nwarps) {
+        float acc[EP];
+#pragma unroll
+        for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+        for (int c = lane; c < nvec; c += 32) {
+            const uint4 xv = __ldg(xr + c);
+            const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
+            float xf[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f2 = __bfloat1622float2(xp[i]);
+                xf[2 * i] = f2.x;
+                xf[2 * i + 1] = f2.y;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4* wrow = reinterpret_cast<const uint4*>(swr + static_cast<int64_t>(c * 8 + i) * EP);
+#pragma unroll
+                for (int vv = 0; vv < EV; ++vv) {
+                    const uint4 wv = wrow[vv];
+                    const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float2 w2 = __bfloat1622float2(wp[h]);
+                        acc[vv * 8 + 2 * h] = fmaf(xf[i], w2.x, acc[vv * 8 + 2 * h]);
+                        acc[vv * 8 + 2 * h + 1] = fmaf(xf[i], w2.y, acc[vv * 8 + 2 * h + 1]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EP; ++e) acc[e] = warp_sum(acc[e]);
+        float l[1] = {-FLT_MAX};
+#pragma unroll
+        for (int e = 0; e < EP; ++e)
+            if (e == lane) l[0] = acc[e];
+        bool valid[1] = {lane < E};
+        if (logits != nullptr && valid[0]) logits[t * E + lane] = l[0];
+        finish_token<1>(l, valid, bias, t, K, lane, idx, w, psum, want_prob);
+    }
+    if (want_prob) write_prob_partials<1>(psum, E, prob_part);
+}
+
+template <int J>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+topk_from_logits_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int64_t T, int E,
+                        int K, int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ prob_part) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kRouteWarps;
+    float psum[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) psum[j] = 0.f;
+    const bool want_prob = prob_part != nullptr;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps + warp; t < T; t += nwarps) {
+        float l[J];
+        bool valid[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int e = lane + 32 * j;
+            valid[j] = e < E;
+            l[j] = valid[j] ? logits[t * E + e] : -FLT_MAX;
+        }
+        finish_token<J>(l, valid, bias, t, K, lane, idx, w, psum, want_prob);
+    }
+    if (want_prob) write_prob_partials<J>(psum, E, prob_part);
+}
+
+__global__ void prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float invT,
+                                     float* __restrict__ out) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+        float s = 0.f;
+        for (int b = 0; b < nblocks; ++b) s += part[static_cast<int64_t>(b) * E + e];
+        out[e] = s * invT;
+    }
+}
+
+// WrT[e][k] = Wr[k][e] for e < E, 0 for E <= e < E_pad.
+__global__ void transpose_router_kernel(const __nv_bfloat16* __restrict__ Wr, int d, int E, int E_pad,
+                                        __nv_bfloat16* __restrict__ WrT) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int k0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int k = k0 + i, e = e0 + threadIdx.x;
+        tile[i][threadIdx.x] = (k < d && e < E) ? Wr[static_cast<int64_t>(k) * E + e] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int e = e0 + i, k = k0 + threadIdx.x;
+        if (e < E_pad && k < d) WrT[static_cast<int64_t>(e) * d + k] = tile[threadIdx.x][i];
+    }
+}
+
+}  // namespace
+
+int route_blocks(int64_t T) {
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    int64_t need = (T + kRouteWarps - 1) / kRouteWarps;
+    int64_t cap = static_cast<int64_t>(sms) * 4;
+    return static_cast<int>(need < cap ? (need < 1 ? 1 : need) : cap);
+}
+
+int route_fused_supported(int d, int E) {
+    if (E > 32 || d % 8 != 0) return 0;
+    const int EP = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
+    return static_cast<size_t>(d) * EP * 2 <= 96 * 1024 ? 1 : 0;
+}
+
+int launch_route_fused(const bf16* x, const bf16* Wr, const float* bias, int64_t T, int d, int E, int K,
+                       float* logits, int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st) {
+    const int EV = E <= 8 ? 1 : (E <= 16 ? 2 : 4);
+    const size_t smem = static_cast<size_t>(d) * EV * 8 * 2;
+    cudaError_t err;
+    switch (EV) {
+        case 1:
+            cudaFuncSetAttribute(route_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+            route_fused_kernel<1><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+            break;
+        case 2:
+            cudaFuncSetAttribute(route_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+            route_fused_kernel<2><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+            break;
+        default:
+            cudaFuncSetAttribute(route_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+            route_fused_kernel<4><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+            break;
+    }
+    err = cudaGetLastError();
+    return err == cudaSuccess ? 0 : -3;
+}
+
+int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, int E, int K, int32_t* idx,
+                            float* w, float* prob_part, int nblocks, cudaStream_t st) {
+    const int th = kRouteWarps * 32;
+    if (E <= 32)
+        topk_from_logits_kernel<1><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+    else if (E <= 64)
+        topk_from_logits_kernel<2><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+    else if (E <= 128)
+        topk_from_logits_kernel<4><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+    else if (E <= 256)
+        topk_from_logits_kernel<8><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+    else
+        return -2;
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, float* prob_mean, cudaStream_t st) {
+    prob_finalize_kernel<<<(E + 255) / 256, 256, 0, st>>>(prob_part, nblocks, E, 1.0f / static_cast<float>(T),
+                                                         prob_mean);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int launch_transpose_router(const bf16* Wr, int d, int E, int E_pad, bf16* WrT, cudaStream_t st) {
+    dim3 grid((d + 31) / 32, (E_pad + 31) / 32), block(32, 8);
+    transpose_router_kernel<<<grid, block, 0, st>>>(Wr, d, E, E_pad, WrT);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+}  // namespace moe

@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI: no GPU needed, no kernel launched."""
+import ctypes
+import math
+import os
+import re
+from fractions import Fraction
+
+import pytest
+
+from moe_layer_gemm_b200 import abi, build
+from oracle import moe_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.load()
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_every_header_function_is_exported(lib):
+    names = _header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(abi.EXPORTED) == names
+
+
+def test_status_strings_and_version(lib):
+    assert abi.moe_version() >= 100
+    for s in (0, -1, -2, -3, -4, -5):
+        assert abi.moe_status_str(s).startswith("MOE_")
+    assert abi.moe_status_str(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("T,K,E,cf", [
+    (8192, 4, 60, 1.0), (64, 2, 8, 1.25), (30, 2, 3, 0.8), (30, 2, 3, 0.75), (1, 1, 1, 1e-30),
+    (16384, 2, 8, 1.1), (4096, 8, 256, 0.3), (777, 3, 7, 2.0 / 3.0), (100, 2, 8, 0.0), (100, 2, 8, -1.0),
+    (5, 1, 2, 1e6)])
+def test_capacity_matches_oracle(lib, T, K, E, cf):
+    d = abi.Dims(T, 128, 256, E, K, cf)
+    want = O.capacity(T, K, E, cf)
+    assert abi.moe_capacity(d) == (-1 if want is None else want)
+
+
+def test_dims_validation(lib):
+    good = abi.Dims(64, 128, 256, 8, 2)
+    assert abi.moe_workspace_size(good) > 0
+    bad = [abi.Dims(0, 128, 256, 8, 2), abi.Dims(64, 128, 256, 8, 9), abi.Dims(64, 128, 256, 0, 1),
+           abi.Dims(64, 128, 256, 300, 2), abi.Dims(64, 8, 256, 8, 2), abi.Dims(1 << 25, 128, 256, 8, 2)]
+    for d in bad:
+        with pytest.raises(abi.MoEError) as e:
+            abi.moe_workspace_size(d)
+        assert e.value.status == abi.MOE_EINVAL
+    with pytest.raises(abi.MoEError) as e:
+        abi.moe_workspace_size(abi.Dims(64, 136, 256, 8, 2))  # d_model not a multiple of 16
+    assert e.value.status == abi.MOE_EUNSUPPORTED
+    assert abi.moe_capacity(abi.Dims(0, 128, 256, 8, 2)) < -1
+
+
+def test_null_arguments_are_rejected_before_any_launch(lib):
+    d = abi.Dims(64, 128, 256, 8, 2).c()
+    ws_bytes = abi.moe_workspace_size(d)
+    nul = None
+    assert lib.moe_route(ctypes.byref(d), nul, nul, nul, nul, nul, nul, nul, nul, ws_bytes, nul) == abi.MOE_EINVAL
+    assert lib.moe_permute(ctypes.byref(d), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul, 0, nul) == abi.MOE_EINVAL
+    assert lib.moe_combine(ctypes.byref(d), nul, nul, nul, nul, nul) == abi.MOE_EINVAL
+    assert lib.moe_layer_forward(ctypes.byref(d), nul, nul, nul, 0.0, nul, nul, nul, nul, nul, 0, nul) == abi.MOE_EINVAL
+    assert lib.moe_bias_update(ctypes.byref(d), nul, 0.001, nul, nul) == abi.MOE_EINVAL
+    assert lib.moe_pack_weights(None, nul, nul, nul, nul, nul, nul) == abi.MOE_EINVAL
+
+
+def test_workspace_too_small_and_misaligned(lib):
+    d = abi.Dims(64, 128, 256, 8, 2).c()
+    n = abi.moe_workspace_size(d)
+    fake = ctypes.c_void_p(0x10000)   # never dereferenced: the size check fails first
+    st = lib.moe_route_from_logits(ctypes.byref(d), fake, None, fake, fake, None, fake, n - 1, None)
+    assert st == abi.MOE_EWORKSPACE
+    st = lib.moe_route_from_logits(ctypes.byref(d), fake, None, fake, fake, None, ctypes.c_void_p(0x10008), n, None)
+    assert st == abi.MOE_EINVAL
+
+
+def test_workspace_grows_with_problem(lib):
+    small = abi.moe_workspace_size(abi.Dims(64, 128, 256, 8, 2))
+    big = abi.moe_workspace_size(abi.Dims(16384, 4096, 14336, 8, 2))
+    assert big > small
+    # at least x_perm + h + y_perm for the big case
+    A = 16384 * 2
+    assert big >= A * 4096 * 2 + A * 14336 * 2 + A * 4096 * 4

@@ -1,0 +1,76 @@
+"""Expert FFN parity: the grouped tcgen05 GEMMs against the fp64 oracle FFN.
+
+Shapes cover both tile orientations (weight rows on the MMA M side for small
+groups, token rows for large ones), empty groups, groups smaller than one
+tile, ragged tails, split reductions and the packed-weight layout.
+"""
+import numpy as np
+import pytest
+import torch
+
+from moe_layer_gemm_b200 import abi, synth
+from oracle import moe_oracle as O
+from tests.gpu_util import Y_MAX_ABS, Y_MIRROR_MAX_ABS, Y_MIRROR_REL_L2, Y_REL_L2, assert_close_y, dev, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
+    dv = dev()
+    wts = None if skew == 0 else torch.tensor([(r + 1.0) ** -skew for r in range(E)])
+    idx = synth.distinct_choices(T, E, K, seed=seed, weights=wts).to(dv)
+    x = synth.normal_bf16((T, d), seed, synth.STREAM_X, 1.0, dv)
+    W1 = synth.normal_bf16((E, d, f), seed, synth.STREAM_W1, w_std, dv)
+    W3 = synth.normal_bf16((E, d, f), seed, synth.STREAM_W3, w_std, dv)
+    W2 = synth.normal_bf16((E, f, d), seed, synth.STREAM_W2, w_std, dv)
+    dims = abi.Dims(T, d, f, E, K)
+    ws = abi.alloc_workspace(dims)
+    W13p, W2p = abi.pack_weights(dims, W1, W3, W2)
+    i32 = dict(dtype=torch.int32, device=dv)
+    A = T * K
+    counts, kept, offsets = torch.empty(E, **i32), torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    inv, src = torch.empty(T, K, **i32), torch.empty(A, **i32)
+    xp = torch.zeros(A, d, dtype=torch.bfloat16, device=dv)
+    abi.moe_permute(dims, idx, x, counts, kept, offsets, inv, src, xp, None, ws)
+    h = torch.zeros(A, f, dtype=torch.bfloat16, device=dv)
+    yp = torch.zeros(A, d, dtype=torch.float32, device=dv)
+    abi.moe_expert_ffn(dims, xp, offsets, W13p, W2p, h, yp, ws)
+    torch.cuda.synchronize()
+    st, detail = abi.moe_get_device_status(ws)
+    assert st == abi.MOE_OK, f"device wait ran out (code {detail})"
+    # oracle: its own dispatch of the same idx, then the FFN per expert
+    o = O.dispatch(idx.cpu().numpy(), E, None)
+    x64 = f64(x)
+    W1h, W3h, W2h = f64(W1), f64(W3), f64(W2)
+    off, srco = o["offsets"], o["src"]
+    Y = np.zeros((A, d))
+    Yr = np.zeros((A, d))
+    H = np.zeros((A, f))
+    for e in range(E):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if r1 == r0:
+            continue
+        Xe = x64[srco[r0:r1]]
+        g, u = Xe @ W1h[e], Xe @ W3h[e]
+        H[r0:r1] = O.silu(g) * u
+        Y[r0:r1] = O.swiglu_ffn(Xe, W1h[e], W3h[e], W2h[e])
+        Yr[r0:r1] = O.swiglu_ffn(Xe, W1h[e], W3h[e], W2h[e], h_round=O.bf16_round)
+    return dict(h=f64(h), yp=f64(yp), H=H, Y=Y, Yr=Yr, n=int(off[-1]), offsets=off)
+
+
+@pytest.mark.parametrize("T,d,f,E,K,skew", [
+    (64, 128, 256, 8, 2, 0.0),        # small groups: weight-major tiles
+    (256, 512, 512, 8, 2, 0.0),       # decode-like, split reduction
+    (300, 256, 192, 16, 4, 1.0),      # ragged, some groups tiny
+    (2000, 256, 320, 4, 2, 0.0),      # large groups: token-major tiles, ragged m tail
+    (1500, 384, 704, 12, 3, 1.5),     # skewed: empty groups possible
+    (130, 128, 128, 1, 1, 0.0),       # single expert = dense FFN
+])
+def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
+    r = _run(T, d, f, E, K, skew)
+    n = r["n"]
+    # H: bf16 rounding of an fp32 value close to the fp64 one
+    Hg, H = r["h"][:n], r["H"][:n]
+    assert np.all(np.abs(Hg - H) <= np.abs(H) * 2.0 ** -8 + 1e-4)
+    assert_close_y(r["yp"][:n], r["Y"][:n], Y_MAX_ABS, Y_REL_L2, "y_perm")
+    assert_close_y(r["yp"][:n], r["Yr"][:n], Y_MIRROR_MAX_ABS, Y_MIRROR_REL_L2, "y_perm (H rounded)")

@@ -1,0 +1,87 @@
+"""Router parity: top-K, renormalisation, P_i (bit-exact selection on shared logits)."""
+import numpy as np
+import pytest
+import torch
+
+from moe_layer_gemm_b200 import abi, synth
+from oracle import moe_oracle as O
+from tests.gpu_util import (P_TOL, W_TOL, ambiguous_tokens, check_routing_validity, dev, f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _bias(E, seed, scale=0.5):
+    return (synth.normal_f32(E, seed, synth.STREAM_MISC) * scale).to(torch.float32)
+
+
+@pytest.mark.parametrize("T,E,K,use_bias,tie", [
+    (1000, 8, 2, False, 0.3), (777, 60, 4, True, 0.3), (513, 256, 8, True, 0.3), (64, 1, 1, False, 0.0),
+    (100, 16, 16, False, 0.5), (300, 33, 5, True, 0.2), (1, 8, 2, False, 0.0), (4097, 128, 6, True, 0.1)])
+def test_route_from_logits_bitexact(T, E, K, use_bias, tie):
+    d = dev()
+    logits = synth.logits_f32(T, E, seed=T + E, tie_frac=tie, device=d)
+    bias = _bias(E, T).to(d) if use_bias else None
+    dims = abi.Dims(T, 128, 256, E, K)
+    ws = abi.alloc_workspace(dims)
+    idx = torch.empty(T, K, dtype=torch.int32, device=d)
+    w = torch.empty(T, K, dtype=torch.float32, device=d)
+    P = torch.empty(E, dtype=torch.float32, device=d)
+    abi.moe_route_from_logits(dims, logits, bias, idx, w, P, ws)
+    torch.cuda.synchronize()
+    l_host = logits.cpu().numpy()
+    b_host = None if bias is None else bias.cpu().numpy()
+    idx_o, w_o, _ = O.route_from_logits_f32(l_host, K, b_host)
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert np.max(np.abs(f64(w) - w_o)) <= W_TOL
+    P_o = O.softmax_rows(l_host.astype(np.float64)).mean(axis=0)
+    assert np.max(np.abs(f64(P) - P_o)) <= P_TOL
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 64), ("mixtral_decode", 256), ("mixtral_prefill", 3000),
+                                    ("qwen_capacity", 1000), ("deepseek_bias", 700)])
+def test_route_fused_vs_oracle(name, T):
+    d = dev()
+    wl = synth.get_workload(name)
+    x = synth.make_x(wl, device=d)[:T].contiguous()
+    Wr = synth.make_router(wl, device=d)
+    E, K = wl.E, wl.K
+    bias = _bias(E, 7, 0.05).to(d) if wl.use_bias else None
+    dims = abi.Dims(T, wl.d_model, wl.d_ff, E, K, wl.capacity_factor)
+    ws = abi.alloc_workspace(dims)
+    logits = torch.empty(T, E, dtype=torch.float32, device=d)
+    idx = torch.empty(T, K, dtype=torch.int32, device=d)
+    w = torch.empty(T, K, dtype=torch.float32, device=d)
+    P = torch.empty(E, dtype=torch.float32, device=d)
+    abi.moe_route(dims, x, Wr, bias, logits, idx, w, P, ws)
+    torch.cuda.synchronize()
+    x64, Wr64 = f64(x), f64(Wr)
+    l64 = O.router_logits(x64, Wr64)
+    # fp32 accumulation bound; x2 covers tensor-core accumulation (non-RNE adds)
+    bound = 2.0 * O.dot_error_bound(x64, Wr64) + np.abs(l64) * 2.0 ** -23
+    lg = f64(logits)
+    assert np.all(np.abs(lg - l64) <= bound), float(np.max(np.abs(lg - l64) - bound))
+    b32 = None if bias is None else bias.cpu().numpy()
+    idx_o, w_o, _ = O.route_from_logits_f32(l64.astype(np.float32), K, b32)
+    amb = ambiguous_tokens(l64, bound, K, b32)
+    ig = idx.cpu().numpy()
+    # exact where the worst-case bound leaves one answer; valid everywhere;
+    # and in practice (errors far below the worst case) nearly always equal
+    assert np.array_equal(ig[~amb], idx_o[~amb])
+    assert np.mean(np.all(ig == idx_o, axis=1)) >= 0.995
+    check_routing_validity(ig, l64, bound, K, b32)
+    # the library's choice is the exact top-K of its own (biased) fp32 logits
+    lb = logits.cpu().numpy() if b32 is None else (logits.cpu().numpy() + b32[None, :]).astype(np.float32)
+    for t in range(T):
+        sel = ig[t].tolist()
+        vals = [lb[t, e] for e in sel]
+        assert all(vals[j] > vals[j + 1] or (vals[j] == vals[j + 1] and sel[j] < sel[j + 1]) for j in range(K - 1))
+        rest = [e for e in range(E) if e not in sel]
+        if rest:
+            m = max(lb[t, e] for e in rest)
+            assert vals[-1] >= m
+            if vals[-1] == m:
+                assert sel[-1] < min(e for e in rest if lb[t, e] == m)
+    wt = np.max(2 * bound, axis=1, keepdims=True) + W_TOL
+    assert np.all(np.abs(f64(w)[~amb] - w_o[~amb]) <= wt[~amb])
+    P_o = O.softmax_rows(l64).mean(axis=0)
+    assert np.max(np.abs(f64(P) - P_o)) <= P_TOL + 2 * float(bound.max())
