@@ -5,7 +5,7 @@ import torch
 
 from moe_layer_gemm_b200 import abi, synth
 from oracle import moe_oracle as O
-from tests.gpu_util import (Y_MAX_ABS, Y_MIRROR_MAX_ABS, Y_MIRROR_REL_L2, LayerInputs, ambiguous_tokens,
+from tests.gpu_util import (Y_MAX_ABS, Y_MIRROR_MAX_ABS, Y_MIRROR_REL_L2, Y_REL_L2, LayerInputs, ambiguous_tokens,
                             assert_close_y, check_routing_validity, dev, f64, oracle_layer,
                             uncertain_tokens)
 
