@@ -101,15 +101,27 @@ MOE_API int moe_reset_device_status(void* ws, void* stream);
  * out (a small integer; 0 if none). */
 MOE_API int moe_get_device_status(const void* ws, void* stream, int* status, int* detail);
 
+/* Bytes of the packed expert weights moe_pack_weights writes for these dims:
+ * *w13_bytes for the gate/up weights, *w2_bytes for the down weights.  Host
+ * only. */
+MOE_API int moe_packed_weight_bytes(const moe_dims* dims, size_t* w13_bytes, size_t* w2_bytes);
+
 /* One-time re-layout of the expert weights for the tensor-core GEMMs.
  *   W1, W3  [E, d_model, d_ff]   (x . W1 is the gate, x . W3 the up projection)
  *   W2      [E, d_ff, d_model]   (down projection)
- *   W13p    [E, 2*d_ff, d_model] out: rows 32b..32b+15 are W1[:, 16b..16b+15]^T,
- *                                rows 32b+16..32b+31 are W3[:, 16b..16b+15]^T
- *   W2p     [E, d_model, d_ff]   out: W2^T per expert
+ *   W13p    out, moe_packed_weight_bytes(..)->w13_bytes bytes: per expert the
+ *           K-major gate/up matrix [2*d_ff rows, d_model] whose rows
+ *           32b..32b+15 are W1[:, 16b..16b+15]^T and rows 32b+16..32b+31 are
+ *           W3[:, 16b..16b+15]^T, stored as 128-row x 64-column tiles (16 KB,
+ *           row-block-major, then column-block) with the 128-byte swizzle of
+ *           the tensor-core operand layout inside each tile; padding is zero
+ *   W2p     out, w2_bytes bytes: per expert W2^T [d_model rows, d_ff] in the
+ *           same tiled form
  * The expert FFN is the SwiGLU form y = (silu(x W1) * (x W3)) W2 ([P2]
- * section 2: each expert is an FFN).  This is a load-time step, outside the
- * per-batch path; the caller may free W1/W3/W2 afterwards. */
+ * section 2: each expert is an FFN).  A weight tile is one contiguous 16 KB
+ * block, so the GEMMs stream weights with plain bulk copies.  This is a
+ * load-time step, outside the per-batch path; the caller may free W1/W3/W2
+ * afterwards. */
 MOE_API int moe_pack_weights(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3,
                      const moe_bf16* W2, moe_bf16* W13p, moe_bf16* W2p, void* stream);
 
@@ -200,8 +212,9 @@ typedef struct moe_layer_outputs {
     float* aux;         /* [1] */
     /* Caller-created CUDA events (cudaEvent_t), or NULL.  When set, the
      * layer records, on `stream`: [0] before routing, [1] after routing,
-     * [2] after dispatch, [3] after the gate/up GEMM, [4] after the down
-     * GEMM, [5] after combine and statistics.  For per-stage timing. */
+     * [2] after dispatch, [3] after the expert GEMMs (gate/up and down run
+     * in one launch), [4] after combine, [5] after statistics and the bias
+     * update.  For per-stage timing. */
     void* const* stage_events; /* [MOE_NUM_STAGE_EVENTS] */
 } moe_layer_outputs;
 

@@ -30,7 +30,7 @@ EXPORTED = [
     "moe_status_str", "moe_version", "moe_capacity", "moe_workspace_size", "moe_reset_device_status",
     "moe_get_device_status", "moe_pack_weights", "moe_route", "moe_route_from_logits", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
-    "moe_layer_launch_count",
+    "moe_layer_launch_count", "moe_packed_weight_bytes",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -82,6 +82,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_bias_update": (I, [dims_p, P, F, P, P]),
         "moe_layer_forward": (I, [dims_p, P, P, P, F, P, P, P, ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
         "moe_layer_launch_count": (I, [dims_p, I, I]),
+        "moe_packed_weight_bytes": (I, [dims_p, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -263,15 +264,18 @@ def moe_layer_launch_count(dims, stats: bool, bias_update: bool) -> int:
 
 # ---------------------------------------------------------------- helpers
 
-def packed_weight_shapes(dims):
-    d = _dims(dims)
-    return (d.E, 2 * d.d_ff, d.d_model), (d.E, d.d_model, d.d_ff)
+def moe_packed_weight_bytes(dims):
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check("moe_packed_weight_bytes",
+           load().moe_packed_weight_bytes(ctypes.byref(_dims(dims)), ctypes.byref(a), ctypes.byref(b)))
+    return int(a.value), int(b.value)
 
 
 def pack_weights(dims, W1, W3, W2, stream=None):
-    """Allocate and fill the packed expert weights (W13p, W2p)."""
-    s13, s2 = packed_weight_shapes(dims)
-    W13p = torch.empty(s13, dtype=BF16, device=W1.device)
-    W2p = torch.empty(s2, dtype=BF16, device=W1.device)
+    """Allocate and fill the packed expert weights (W13p, W2p): flat bf16
+    buffers in the library's tiled layout."""
+    n13, n2 = moe_packed_weight_bytes(dims)
+    W13p = torch.empty(n13 // 2, dtype=BF16, device=W1.device)
+    W2p = torch.empty(n2 // 2, dtype=BF16, device=W1.device)
     moe_pack_weights(dims, W1, W3, W2, W13p, W2p, stream)
     return W13p, W2p

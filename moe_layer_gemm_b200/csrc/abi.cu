@@ -55,40 +55,36 @@ int64_t capacity_of(const moe_dims* d) {
 }
 
 struct Layout {
-    size_t status, idx, w, logits, counts, kept, offsets, ndrop, prob_part, prob_mean, f, aux, block_hist, inv,
-        src, xperm, h, yperm, wrt, total;
+    size_t status, sched_ffn, sched_router, idx, w, logits, counts, kept, offsets, ndrop, prob_part, prob_mean, f,
+        aux, block_hist, inv, src, xperm, h, yperm, wrt, total;
     int route_nb, perm_nb, nsplit, E_pad, swap;
     bool fused_router;
 };
 
-// Weight rows of one group on the MMA M side pay off when groups are small.
+// Groups of at most this many token rows put the weight rows on the MMA M
+// side (weight-major tiles): small groups then waste no tensor-core rows on
+// padding and the weight stream dominates.
+constexpr int kSwapMaxRows = 128;
+
+// Weight-major tiles are enabled when groups of decode size are expected:
+// a mean group of at most 256 rows (skewed routing then also leaves many
+// small groups).
 int choose_swap(const moe_dims* d) {
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
-    return (avg <= 96 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
+    return (avg <= 256 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
 }
 
-// Split of the down projection's reduction that keeps the last wave full.
+// Reduction split of weight-major down-projection tiles: about as many
+// weight bytes per tile as a gate/up tile (128 x d_model), so the dynamic
+// scheduler's last tiles are short.
 int choose_nsplit(const moe_dims* d, int swap) {
     if (!swap) return 1;
-    const int sms = num_sms() > 0 ? num_sms() : 148;
-    const int64_t rows = d->T * d->K;
-    const int64_t chunk = 128;
-    const int64_t tiles = std::min<int64_t>((rows + chunk - 1) / chunk + d->E, d->E * ((d->T + chunk - 1) / chunk)) *
-                          (d->d_model / 128);
-    const int kblocks = (d->d_ff + 63) / 64;
-    int best = 1;
-    double best_eff = 0.0;
-    for (int ks = 1; ks <= 8 && ks <= kblocks; ++ks) {
-        const int64_t units = tiles * ks;
-        const int64_t rounds = (units + sms - 1) / sms;
-        double eff = static_cast<double>(units) / static_cast<double>(rounds * sms);
-        if (units < sms) eff *= 0.999;  // fewer units than SMs: never fills the machine
-        if (eff > best_eff + 0.02) {
-            best_eff = eff;
-            best = ks;
-        }
-    }
-    return best;
+    const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
+    if (avg > kSwapMaxRows) return 1;
+    int ks = static_cast<int>((d->d_ff + d->d_model - 1) / d->d_model);
+    if (ks < 1) ks = 1;
+    if (ks > 8) ks = 8;
+    return ks;
 }
 
 Layout layout_of(const moe_dims* d) {
@@ -108,6 +104,8 @@ Layout layout_of(const moe_dims* d) {
         return at;
     };
     L.status = take(64);
+    L.sched_ffn = take(gemm_sched_bytes(d->E));
+    L.sched_router = take(gemm_sched_bytes(1));
     L.idx = take(A * 4);
     L.w = take(A * 4);
     L.logits = take(T * E * 4);
@@ -125,7 +123,7 @@ Layout layout_of(const moe_dims* d) {
     L.xperm = take(A * D * 2);
     L.h = take(A * F * 2);
     L.yperm = take(static_cast<size_t>(L.nsplit) * A * D * 4);
-    L.wrt = take(static_cast<size_t>(L.E_pad) * D * 2);
+    L.wrt = take(static_cast<size_t>((L.E_pad + 127) / 128) * 128 * ((D + 63) / 64) * 64 * 2);
     L.total = o;
     return L;
 }
@@ -154,7 +152,7 @@ int check_ws(const moe_dims* d, void* ws, size_t ws_bytes) {
     } while (0)
 
 int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, const float* bias, float* logits,
-             int32_t* idx, float* w, float* prob_mean, void* ws, cudaStream_t st) {
+             int32_t* idx, float* w, float* prob_mean, void* ws, cudaStream_t st, bool finalize = true) {
     float* part = prob_mean ? at<float>(ws, L.prob_part) : nullptr;
     if (L.fused_router) {
         MOE_TRY(map_launch(launch_route_fused(x, Wr, bias, d->T, d->d_model, d->E, d->K, logits, idx, w, part,
@@ -164,70 +162,77 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
         bf16* wrt = at<bf16>(ws, L.wrt);
         MOE_TRY(map_launch(launch_transpose_router(Wr, d->d_model, d->E, L.E_pad, wrt, st)));
         GemmLaunch g{};
-        g.tok = x;
-        g.tok_rows = d->T;
-        g.w = wrt;
         g.G = 1;
-        g.N = L.E_pad;
-        g.N_store = d->E;
-        g.Kdim = d->d_model;
         g.group_off = nullptr;
         g.dense_rows = d->T;
         g.max_group_rows = d->T;
-        g.swap = 0;
-        g.ksplit = 1;
-        g.epi = EPI_F32;
-        g.out = lg;
-        g.ldo = d->E;
-        g.split_stride = 0;
+        g.swap_max_rows = 0;
+        g.nphase = 1;
+        g.ph[0].tok = x;
+        g.ph[0].tok_rows = d->T;
+        g.ph[0].w = wrt;
+        g.ph[0].N = L.E_pad;
+        g.ph[0].N_store = d->E;
+        g.ph[0].Kdim = d->d_model;
+        g.ph[0].ksplit = 1;
+        g.ph[0].epi = EPI_F32;
+        g.ph[0].out = lg;
+        g.ph[0].ldo = d->E;
+        g.ph[0].split_stride = 0;
         g.status = at<int>(ws, L.status);
+        g.sched = at<int>(ws, L.sched_router);
+        if (cudaMemsetAsync(g.sched, 0, gemm_sched_bytes(1), st) != cudaSuccess) return MOE_ECUDA;
         MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
         MOE_TRY(map_launch(launch_topk_from_logits(lg, bias, d->T, d->E, d->K, idx, w, part, L.route_nb, st)));
     }
-    if (prob_mean) MOE_TRY(map_launch(launch_prob_finalize(part, L.route_nb, d->E, d->T, prob_mean, st)));
+    if (prob_mean && finalize)
+        MOE_TRY(map_launch(launch_prob_finalize(part, L.route_nb, d->E, d->T, prob_mean, st)));
     return MOE_OK;
 }
 
-template <typename Mid>
+// Both expert GEMMs in one launch.  The scheduler words at L.sched_ffn must
+// be zero when it starts (the dispatch kernels clear them; the standalone
+// entry point clears them with a memset).
 int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
-           const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st, Mid between) {
+           const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st) {
     const int64_t A = d->T * d->K;
     int64_t maxrows = d->T;
     const int64_t C = capacity_of(d);
     if (C >= 0 && C < maxrows) maxrows = C;
     GemmLaunch g{};
-    g.tok = xperm;
-    g.tok_rows = A;
-    g.w = W13p;
     g.G = d->E;
-    g.N = 2 * d->d_ff;
-    g.N_store = 2 * d->d_ff;
-    g.Kdim = d->d_model;
     g.group_off = offsets;
     g.dense_rows = 0;
     g.max_group_rows = maxrows;
-    g.swap = L.swap;
-    g.ksplit = 1;
-    g.epi = EPI_SWIGLU_BF16;
-    g.out = h;
-    g.ldo = d->d_ff;
-    g.split_stride = 0;
+    g.swap_max_rows = L.swap ? kSwapMaxRows : 0;
+    g.nphase = 2;
+    GemmPhase& p0 = g.ph[0];
+    p0.tok = xperm;
+    p0.tok_rows = A;
+    p0.w = W13p;
+    p0.N = 2 * d->d_ff;
+    p0.N_store = 2 * d->d_ff;
+    p0.Kdim = d->d_model;
+    p0.ksplit = 1;
+    p0.epi = EPI_SWIGLU_BF16;
+    p0.out = h;
+    p0.ldo = d->d_ff;
+    p0.split_stride = 0;
+    GemmPhase& p1 = g.ph[1];
+    p1.tok = h;
+    p1.tok_rows = A;
+    p1.w = W2p;
+    p1.N = d->d_model;
+    p1.N_store = d->d_model;
+    p1.Kdim = d->d_ff;
+    p1.ksplit = nsplit;
+    p1.epi = EPI_F32;
+    p1.out = yout;
+    p1.ldo = d->d_model;
+    p1.split_stride = A * d->d_model;
     g.status = at<int>(ws, L.status);
-    MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
-    between();
-    GemmLaunch g2 = g;
-    g2.tok = h;
-    g2.w = W2p;
-    g2.N = d->d_model;
-    g2.N_store = d->d_model;
-    g2.Kdim = d->d_ff;
-    g2.ksplit = nsplit;
-    g2.epi = EPI_F32;
-    g2.out = yout;
-    g2.ldo = d->d_model;
-    g2.split_stride = A * d->d_model;
-    MOE_TRY(map_launch(launch_grouped_gemm(g2, st)));
-    return MOE_OK;
+    g.sched = at<int>(ws, L.sched_ffn);
+    return map_launch(launch_grouped_gemm(g, st));
 }
 
 }  // namespace
@@ -274,6 +279,14 @@ int moe_get_device_status(const void* ws, void* stream, int* status, int* detail
         return MOE_ECUDA;
     *status = host == 0 ? MOE_OK : MOE_ETIMEOUT;
     if (detail) *detail = host;
+    return MOE_OK;
+}
+
+int moe_packed_weight_bytes(const moe_dims* dims, size_t* w13_bytes, size_t* w2_bytes) {
+    MOE_TRY(check_dims(dims));
+    if (!w13_bytes || !w2_bytes) return MOE_EINVAL;
+    *w13_bytes = packed_w13_bytes(dims->E, dims->d_model, dims->d_ff);
+    *w2_bytes = packed_w2_bytes(dims->E, dims->d_model, dims->d_ff);
     return MOE_OK;
 }
 
@@ -326,6 +339,7 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x
     return map_launch(launch_permute(topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model, dims->E,
                                      dims->K, capacity_of(dims), at<int32_t>(ws, L.block_hist), counts, kept,
                                      offsets, inv, src, reinterpret_cast<bf16*>(x_perm), n_dropped,
+                                     at<int32_t>(ws, L.sched_ffn), static_cast<int>(gemm_sched_bytes(dims->E) / 4),
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -339,9 +353,9 @@ int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* 
     const Layout L = layout_of(dims);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* yout = L.nsplit > 1 ? at<float>(ws, L.yperm) : y_perm;
+    if (cudaMemsetAsync(at<int>(ws, L.sched_ffn), 0, gemm_sched_bytes(dims->E), st) != cudaSuccess) return MOE_ECUDA;
     MOE_TRY(do_ffn(dims, L, reinterpret_cast<const bf16*>(x_perm), offsets, reinterpret_cast<const bf16*>(W13p),
-                   reinterpret_cast<const bf16*>(W2p), reinterpret_cast<bf16*>(h), yout, L.nsplit, ws, st,
-                   []() {}));
+                   reinterpret_cast<const bf16*>(W2p), reinterpret_cast<bf16*>(h), yout, L.nsplit, ws, st));
     if (L.nsplit > 1)
         MOE_TRY(map_launch(launch_reduce_splits(yout, L.nsplit, dims->T * dims->K * dims->d_model, offsets, dims->E,
                                                 dims->d_model, y_perm, st)));
@@ -403,22 +417,24 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
     };
     mark(0);
     MOE_TRY(do_route(dims, L, xb, reinterpret_cast<const bf16*>(Wr), bias, o.logits, idx, w,
-                     want_stats ? P : nullptr, ws, st));
+                     want_stats ? P : nullptr, ws, st, /*finalize=*/false));
     mark(1);
     MOE_TRY(map_launch(launch_permute(idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
                                       at<int32_t>(ws, L.block_hist), counts, kept, offsets, inv,
-                                      at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop, st)));
+                                      at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop,
+                                      at<int32_t>(ws, L.sched_ffn), static_cast<int>(gemm_sched_bytes(dims->E) / 4),
+                                      st)));
     mark(2);
     float* yp = at<float>(ws, L.yperm);
     MOE_TRY(do_ffn(dims, L, at<bf16>(ws, L.xperm), offsets, reinterpret_cast<const bf16*>(W13p),
-                   reinterpret_cast<const bf16*>(W2p), at<bf16>(ws, L.h), yp, L.nsplit, ws, st,
-                   [&]() { mark(3); }));
-    mark(4);
+                   reinterpret_cast<const bf16*>(W2p), at<bf16>(ws, L.h), yp, L.nsplit, ws, st));
+    mark(3);
     MOE_TRY(map_launch(launch_combine(yp, L.nsplit, dims->T * dims->K * dims->d_model, inv, w, dims->T,
                                       dims->d_model, dims->K, y, st)));
-    if (want_stats || o.f)
-        MOE_TRY(map_launch(launch_stats(counts, want_stats ? P : nullptr, dims->T, dims->E, dims->K, o.f, o.aux,
-                                        nullptr, st)));
+    mark(4);
+    if (want_stats)
+        MOE_TRY(map_launch(launch_finalize_stats(at<float>(ws, L.prob_part), L.route_nb, counts, dims->T, dims->E,
+                                                 dims->K, P, o.f, o.aux, st)));
     if (bias && alpha != 0.0f)
         MOE_TRY(map_launch(launch_bias_update(counts, dims->T, dims->E, dims->K, alpha, bias, st)));
     mark(5);
@@ -429,11 +445,10 @@ int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update) {
     if (check_dims(dims) != MOE_OK) return -1;
     const Layout L = layout_of(dims);
     int n = L.fused_router ? 1 : 3;  // fused router, or transpose + logits GEMM + top-K
-    if (stats) n += 1;               // P_i finalize
-    n += 4;                          // histogram, scan, rank, gather
-    n += 2;                          // gate/up GEMM, down GEMM
+    n += launch_count(dims->T) + 1;  // dispatch kernels + row gather
+    n += 1;                          // both expert GEMMs in one persistent launch
     n += 1;                          // combine
-    if (stats) n += 1;               // f_i and aux
+    if (stats) n += 1;               // P_i, f_i and aux
     if (bias_update) n += 1;
     return n;
 }

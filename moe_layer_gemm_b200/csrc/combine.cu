@@ -15,12 +15,15 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 
 namespace {
 
 constexpr int kMaxK = 16;
+
+constexpr int kMaxSplit = 8;
 
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, const int32_t* __restrict__ inv,
@@ -37,12 +40,15 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int k = 0; k < K; ++k) {
                 if (rows[k] < 0) continue;
-                const float* base = yp + static_cast<int64_t>(rows[k]) * d;
-                float4 v = reinterpret_cast<const float4*>(base)[c];
-                for (int s = 1; s < nsplit; ++s) {
-                    const float4 u = reinterpret_cast<const float4*>(base + s * split_stride)[c];
-                    v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-                }
+                const float4* base = reinterpret_cast<const float4*>(yp + static_cast<int64_t>(rows[k]) * d) + c;
+                float4 part[kMaxSplit];
+#pragma unroll
+                for (int s = 0; s < kMaxSplit; ++s)   // all slices in flight, then summed in slice order
+                    if (s < nsplit) part[s] = __ldg(base + s * (split_stride / 4));
+                float4 v = part[0];
+#pragma unroll
+                for (int s = 1; s < kMaxSplit; ++s)
+                    if (s < nsplit) { v.x += part[s].x; v.y += part[s].y; v.z += part[s].z; v.w += part[s].w; }
                 acc.x = fmaf(ws[k], v.x, acc.x);
                 acc.y = fmaf(ws[k], v.y, acc.y);
                 acc.z = fmaf(ws[k], v.z, acc.z);
@@ -90,6 +96,33 @@ stats_kernel(const int32_t* __restrict__ counts, const float* __restrict__ P, in
     if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
 }
 
+// One block: P_i = (sum over router blocks of the per-block sums) / T, in
+// block order; then f_i and aux as in stats_kernel.
+__global__ void __launch_bounds__(256)
+finalize_stats_kernel(const float* __restrict__ part, int nblocks, const int32_t* __restrict__ counts, int64_t T,
+                      int E, int K, float* __restrict__ P, float* __restrict__ f, float* __restrict__ aux) {
+    __shared__ float red[256];
+    const float invT = 1.0f / static_cast<float>(T);
+    const float invA = 1.0f / static_cast<float>(T * K);
+    float acc = 0.f;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float s = 0.f;
+        for (int b = 0; b < nblocks; ++b) s += part[static_cast<int64_t>(b) * E + e];
+        const float pe = s * invT;
+        const float fe = static_cast<float>(counts[e]) * invA;
+        P[e] = pe;
+        if (f) f[e] = fe;
+        acc += fe * pe;
+    }
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+        if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
+}
+
 __global__ void bias_update_kernel(const int32_t* __restrict__ counts, int64_t TK, int E, float alpha,
                                    float* __restrict__ bias) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -122,10 +155,11 @@ __global__ void pack_w13_kernel(const __nv_bfloat16* __restrict__ W1, const __nv
         tile[i][j] = v;
     }
     __syncthreads();
-    __nv_bfloat16* dst = W13p + static_cast<int64_t>(e) * 2 * f * d;
+    const int64_t kb = (d + 63) / 64;
+    __nv_bfloat16* dst = W13p + static_cast<int64_t>(e) * ((2 * f + 127) / 128) * kb * 8192;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int r = r0 + i, k = k0 + threadIdx.x;
-        if (k < d) dst[static_cast<int64_t>(r) * d + k] = tile[threadIdx.x][i];
+        if (k < d) dst[tiled_offset(r, k, kb)] = tile[threadIdx.x][i];
     }
 }
 
@@ -140,10 +174,11 @@ __global__ void pack_w2_kernel(const __nv_bfloat16* __restrict__ W2, int d, int 
         tile[i][threadIdx.x] = (k < f && n < d) ? s[static_cast<int64_t>(k) * d + n] : __float2bfloat16_rn(0.f);
     }
     __syncthreads();
-    __nv_bfloat16* dst = W2p + static_cast<int64_t>(e) * d * f;
+    const int64_t kb = (f + 63) / 64;
+    __nv_bfloat16* dst = W2p + static_cast<int64_t>(e) * ((d + 127) / 128) * kb * 8192;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int n = n0 + i, k = k0 + threadIdx.x;
-        if (n < d && k < f) dst[static_cast<int64_t>(n) * f + k] = tile[threadIdx.x][i];
+        if (n < d && k < f) dst[tiled_offset(n, k, kb)] = tile[threadIdx.x][i];
     }
 }
 
@@ -151,7 +186,7 @@ __global__ void pack_w2_kernel(const __nv_bfloat16* __restrict__ W2, int d, int 
 
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv, const float* w,
                    int64_t T, int d, int K, float* y, cudaStream_t st) {
-    if (K > kMaxK || d % 4 != 0) return -2;
+    if (K > kMaxK || d % 4 != 0 || nsplit > kMaxSplit) return -2;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     int64_t grid = T < static_cast<int64_t>(sms) * 16 ? T : static_cast<int64_t>(sms) * 16;
     int threads = d / 4 >= 256 ? 256 : ((d / 4 + 31) / 32) * 32;
@@ -173,13 +208,29 @@ int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
+int launch_finalize_stats(const float* prob_part, int nblocks, const int32_t* counts, int64_t T, int E, int K,
+                          float* P, float* f, float* aux, cudaStream_t st) {
+    finalize_stats_kernel<<<1, 256, 0, st>>>(prob_part, nblocks, counts, T, E, K, P, f, aux);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
 int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias, cudaStream_t st) {
     bias_update_kernel<<<(E + 255) / 256, 256, 0, st>>>(counts, T * K, E, alpha, bias);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
+size_t packed_w13_bytes(int E, int d, int f) {
+    return static_cast<size_t>(E) * ((2 * f + 127) / 128) * ((d + 63) / 64) * 16384;
+}
+size_t packed_w2_bytes(int E, int d, int f) {
+    return static_cast<size_t>(E) * ((d + 127) / 128) * ((f + 63) / 64) * 16384;
+}
+
 int launch_pack(const bf16* W1, const bf16* W3, const bf16* W2, int E, int d, int f, bf16* W13p, bf16* W2p,
                 cudaStream_t st) {
+    // padding of partial tiles stays zero
+    if (cudaMemsetAsync(W13p, 0, packed_w13_bytes(E, d, f), st) != cudaSuccess) return -3;
+    if (cudaMemsetAsync(W2p, 0, packed_w2_bytes(E, d, f), st) != cudaSuccess) return -3;
     dim3 block(32, 8);
     dim3 g13((d + 31) / 32, (2 * f) / 32, E);
     pack_w13_kernel<<<g13, block, 0, st>>>(W1, W3, d, f, W13p);

@@ -2,31 +2,37 @@
 // TMA, for the expert FFN of an MoE layer: each expert g multiplies its own
 // contiguous group of token rows by its own weight matrix ("MoE computation
 // notes", cf-1.com/news/5905749, section 2.1: permute tokens so each expert
-// gets one contiguous batch and run one matrix product per group).
+// gets one contiguous batch and run one matrix product per group; section
+// 2.2: experts never see tokens that did not choose them).
 //
-// One persistent CTA per SM walks a device-built list of output tiles, so
-// the ragged group sizes never travel to the host.  Roles per CTA (192
-// threads):
-//   warp 0        TMA producer (one elected thread), multi-stage smem ring
+// One persistent CTA per SM.  Up to two phases run in one launch: the
+// gate/up projection with its SwiGLU epilogue (phase 0) and the down
+// projection (phase 1).  Tiles are handed out by a global atomic counter in
+// phase order, and a phase-1 tile of expert g waits (bounded) until every
+// phase-0 tile of g has stored its H rows, so the down projection of early
+// experts overlaps the gate/up projection of late ones and there is one
+// tail instead of two.  Roles per CTA (192 threads):
+//   warp 0        scheduler + producer (one elected thread): claims tiles,
+//                 broadcasts them through a shared-memory ring and fills a
+//                 multi-stage operand ring: token rows by TMA tile loads,
+//                 weight tiles by contiguous 16 KB bulk copies of the
+//                 pre-tiled, pre-swizzled packed weights
 //   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2..5    epilogue: TMEM -> registers -> SwiGLU / fp32 -> global
-// The accumulator is double-buffered in TMEM (2 x 256 fp32 columns), so the
-// epilogue of tile i overlaps the main loop of tile i+1.
+// The accumulator is double-buffered in TMEM (2 x 256 fp32 columns).
 //
-// Two tile orientations:
-//   token-major (swap = 0):  D[128 tokens x BN weight rows]; used when groups
-//                            hold many tokens (prefill).
-//   weight-major (swap = 1): D[128 weight rows x n tokens] (n <= 128, a
-//                            multiple of 32); used when groups are small
-//                            (decode), so no tensor-core rows are wasted on
-//                            padding and the weight stream dominates.  The
-//                            reduction can be split (deterministic partial
-//                            slices, summed later in a fixed order).
+// Tile orientation is chosen per group:
+//   token-major:  D[128 tokens x BN weight rows]   (groups with many tokens)
+//   weight-major: D[128 weight rows x n tokens], n <= 128 a multiple of 32
+//                 (small groups: no tensor-core rows spent on padding; the
+//                 weight stream dominates).  In phase 1 the reduction of a
+//                 weight-major tile can be split into slices written to
+//                 separate partial buffers and summed later in slice order.
 // No TMA multicast is used anywhere.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
-#include <cstdio>
+#include <cstring>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -35,85 +41,111 @@ namespace moe {
 
 namespace {
 
-constexpr int kBK = 64;                 // reduction elements per stage (one 128 B swizzle row)
+constexpr int kBK = 64;                        // reduction elements per stage (one 128 B swizzle row)
 constexpr int kThreads = 192;
 constexpr uint32_t kTileABytes = 128u * 128u;  // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxGroups = 1024;
+constexpr int kMaxGroups = 256;
+constexpr int kRing = 8;                       // scheduled tiles buffered between roles
+
+struct PhaseArgs {
+    const bf16* w;  // tiled weights (tiled_offset), groups w_group_elems apart
+    int64_t w_group_elems;
+    int N;        // weight rows per group
+    int N_store;  // output columns written (router: E of E_pad)
+    int k_blocks;
+    int ksplit;   // weight-major tiles only
+    int kb_per_split;
+    int epi;
+    int BN;       // token-major: weight rows per tile
+    void* out;
+    int64_t ldo;
+    int64_t split_stride;
+};
 
 struct DevArgs {
     const int32_t* group_off;
     int G;
     int64_t dense_rows;
-    int N;
-    int N_store;
-    int k_blocks;
-    int ksplit;
-    int kb_per_split;
-    int swap;
-    int BN;  // token-major: weight rows per tile; weight-major: max tokens per tile
-    int epi;
-    int stages;
-    uint32_t stage_b_bytes;
-    void* out;
-    int64_t ldo;
-    int64_t split_stride;
+    int swap_max_rows;  // groups with rows <= this use weight-major tiles
+    int BNs;            // weight-major: max tokens per tile (multiple of 32, <= 128)
+    int nphase;
+    int dep;            // phase-1 tiles of g wait for all phase-0 tiles of g
+    PhaseArgs ph[2];
+    int stages;                 // operand ring depth; a stage holds one weight and one token slot
+    uint32_t wslot, xslot;      // bytes per weight / token slot
     int* status;
+    int* sched;         // [0] tile counter, [1..G] phase-0 tiles done per group (x4 warps)
+};
+
+struct Maps {
+    CUtensorMap tokA[2];  // token rows, box 128 (token-major A)
+    CUtensorMap tokB[2];  // token rows, box 32  (weight-major B)
 };
 
 struct Tile {
+    int phase;
     int g;
-    int64_t row0;  // first token row of the tile
-    int rows;      // valid token rows (<= 128 or <= BN)
+    int swap;
+    int64_t row0;  // first token row
+    int rows;      // valid token rows
     int n0;        // first weight row within the group
-    int kb0, kb1;  // reduction blocks [kb0, kb1)
+    int kb0, kb1;
     int split;
 };
 
-__device__ __forceinline__ int64_t grp_off(const int64_t* off, int g) { return off[g]; }
-
-__device__ __forceinline__ int tiles_of_group(const DevArgs& a, int64_t rows) {
-    if (rows <= 0) return 0;
-    if (!a.swap) {
-        int64_t mt = (rows + 127) / 128;
-        return static_cast<int>(mt * (a.N / a.BN));
-    }
-    int64_t nch = (rows + a.BN - 1) / a.BN;
-    return static_cast<int>(nch * (a.N / 128) * a.ksplit);
+__device__ __forceinline__ bool group_swaps(const DevArgs& a, int p, int64_t rows) {
+    return rows <= a.swap_max_rows && a.ph[p].N % 128 == 0;
 }
 
-__device__ __forceinline__ Tile decode_tile(const DevArgs& a, int tile, const int* tstart,
-                                            const int64_t* off) {
-    int lo = 0, hi = a.G;  // tstart[lo] <= tile < tstart[hi]
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (tstart[mid] <= tile) lo = mid; else hi = mid;
-    }
+__device__ __forceinline__ int tiles_of(const DevArgs& a, int p, int64_t rows) {
+    if (rows <= 0) return 0;
+    const PhaseArgs& ph = a.ph[p];
+    if (!group_swaps(a, p, rows)) return static_cast<int>(((rows + 127) / 128) * (ph.N / ph.BN));
+    return static_cast<int>(((rows + a.BNs - 1) / a.BNs) * (ph.N / 128) * ph.ksplit);
+}
+
+// tstart[p*(G+1) + g]: first tile of group g in phase p (global numbering).
+__device__ __forceinline__ Tile decode_tile(const DevArgs& a, int tile, const int* tstart, const int64_t* off) {
     Tile t;
+    const int G = a.G;
+    int p = 0;
+    if (a.nphase > 1 && tile >= tstart[G]) p = 1;
+    const int* ts = tstart + p * (G + 1);
+    int lo = 0, hi = G;  // ts[lo] <= tile < ts[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ts[mid] <= tile) lo = mid; else hi = mid;
+    }
+    const PhaseArgs& ph = a.ph[p];
+    t.phase = p;
     t.g = lo;
-    int local = tile - tstart[lo];
-    int64_t base = off[lo];
-    int64_t rows_g = off[lo + 1] - base;
-    if (!a.swap) {
-        int mt = static_cast<int>((rows_g + 127) / 128);
-        int n = local / mt, m = local - n * mt;
-        t.row0 = base + static_cast<int64_t>(m) * 128;
-        t.rows = static_cast<int>(rows_g - static_cast<int64_t>(m) * 128 < 128 ? rows_g - static_cast<int64_t>(m) * 128 : 128);
-        t.n0 = n * a.BN;
+    const int local = tile - ts[lo];
+    const int64_t base = off[lo];
+    const int64_t rows_g = off[lo + 1] - base;
+    t.swap = group_swaps(a, p, rows_g) ? 1 : 0;
+    if (!t.swap) {
+        const int mt = static_cast<int>((rows_g + 127) / 128);
+        const int n = local / mt, m = local - n * mt;  // m fastest: weight tile reused from L2
+        const int64_t r0 = static_cast<int64_t>(m) * 128;
+        t.row0 = base + r0;
+        t.rows = static_cast<int>(rows_g - r0 < 128 ? rows_g - r0 : 128);
+        t.n0 = n * ph.BN;
         t.kb0 = 0;
-        t.kb1 = a.k_blocks;
+        t.kb1 = ph.k_blocks;
         t.split = 0;
     } else {
-        int nch = static_cast<int>((rows_g + a.BN - 1) / a.BN);
-        int s = local % a.ksplit;
-        int rest = local / a.ksplit;
-        int c = rest % nch;
-        int w = rest / nch;
-        t.row0 = base + static_cast<int64_t>(c) * a.BN;
-        t.rows = static_cast<int>(rows_g - static_cast<int64_t>(c) * a.BN < a.BN ? rows_g - static_cast<int64_t>(c) * a.BN : a.BN);
+        const int nch = static_cast<int>((rows_g + a.BNs - 1) / a.BNs);
+        const int s = local % ph.ksplit;
+        const int rest = local / ph.ksplit;
+        const int c = rest % nch;
+        const int w = rest / nch;
+        const int64_t r0 = static_cast<int64_t>(c) * a.BNs;
+        t.row0 = base + r0;
+        t.rows = static_cast<int>(rows_g - r0 < a.BNs ? rows_g - r0 : a.BNs);
         t.n0 = w * 128;
-        t.kb0 = s * a.kb_per_split;
-        t.kb1 = min(a.k_blocks, t.kb0 + a.kb_per_split);
+        t.kb0 = s * ph.kb_per_split;
+        t.kb1 = min(ph.k_blocks, t.kb0 + ph.kb_per_split);
         t.split = s;
     }
     return t;
@@ -126,137 +158,219 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&p);
 }
 
+// Rows n .. n+rows-1 (rows <= 128, n a multiple of 8, within one 128-row
+// block) of k-block kb of group g's tiled weights: one contiguous range.
+__device__ __forceinline__ const bf16* weight_rows(const PhaseArgs& pa, int g, int n, int kb) {
+    return pa.w + static_cast<int64_t>(g) * pa.w_group_elems + tiled_offset(n, static_cast<int64_t>(kb) * 64, pa.k_blocks);
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok,
-                    const __grid_constant__ CUtensorMap tm_w, const DevArgs a) {
+grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int S = a.stages;
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + static_cast<size_t>(S) * kTileABytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + static_cast<size_t>(S) * a.stage_b_bytes);
+    uint8_t* sW = smem;                                               // [S][wslot]
+    uint8_t* sX = smem + static_cast<size_t>(S) * a.wslot;            // [S][xslot]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sX + static_cast<size_t>(S) * a.xslot);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* rfull = tempty + 2;
+    uint64_t* rempty = rfull + kRing;
+    uint64_t* drain = rempty + kRing;
+    int* ring = reinterpret_cast<int*>(drain + 1);                   // [kRing]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + kRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int64_t* off = reinterpret_cast<int64_t*>(tmem_slot + 4);  // [G+1]
-    int* tstart = reinterpret_cast<int*>(off + a.G + 1);        // [G+1]
+    int64_t* off = reinterpret_cast<int64_t*>(tmem_slot + 2);        // [G+1]
+    int* tstart = reinterpret_cast<int*>(off + a.G + 1);             // [2][G+1]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int G = a.G;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 4);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], 5);  // MMA thread + 4 epilogue warps
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_tok);
-        tma_prefetch_desc(&tm_w);
+        for (int p = 0; p < a.nphase; ++p) {
+            tma_prefetch_desc(&maps.tokA[p]);
+            tma_prefetch_desc(&maps.tokB[p]);
+        }
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
-    for (int g = threadIdx.x; g <= a.G; g += blockDim.x)
+    for (int g = threadIdx.x; g <= G; g += blockDim.x)
         off[g] = a.group_off ? static_cast<int64_t>(a.group_off[g]) : (g == 0 ? 0 : a.dense_rows);
     __syncthreads();
     if (warp == 0) {
-        // tile prefix over groups: each lane scans a contiguous span
-        const int span = (a.G + 31) / 32;
-        const int g0 = min(a.G, lane * span), g1 = min(a.G, g0 + span);
-        int sum = 0;
-        for (int g = g0; g < g1; ++g) sum += tiles_of_group(a, off[g + 1] - off[g]);
-        int incl = sum;
+        // tile prefix over (phase, group): each lane scans a contiguous span of groups
+        const int span = (G + 31) / 32;
+        const int g0 = min(G, lane * span), g1 = min(G, g0 + span);
+        int carry = 0;
+        for (int p = 0; p < a.nphase; ++p) {
+            int sum = 0;
+            for (int g = g0; g < g1; ++g) sum += tiles_of(a, p, off[g + 1] - off[g]);
+            int incl = sum;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int run = carry + incl - sum;
+            int* ts = tstart + p * (G + 1);
+            for (int g = g0; g < g1; ++g) {
+                ts[g] = run;
+                run += tiles_of(a, p, off[g + 1] - off[g]);
+            }
+            const int tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (lane == 0) ts[G] = carry + tot;
+            carry += tot;
         }
-        int run = incl - sum;
-        for (int g = g0; g < g1; ++g) {
-            tstart[g] = run;
-            run += tiles_of_group(a, off[g + 1] - off[g]);
-        }
-        if (lane == 31) tstart[a.G] = incl;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = tstart[a.G];
+    const int total = tstart[(a.nphase - 1) * (G + 1) + G];
 
     if (warp == 0) {
         if (lane == 0) {
-            // ------------------------------------------------ TMA producer
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_t = policy_evict_last();
-            uint32_t s = 0, ph = 0;
+            // ------------------------------------------- scheduler + producer
+            const uint64_t pol_first = policy_evict_first();
+            const uint64_t pol_last = policy_evict_last();
+            const uint64_t pol_norm = policy_evict_normal();
+            uint32_t s = 0, ph = 0, r = 0, rph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            bool sent_end = false;
+            // claims run one tile ahead so the atomic's round trip overlaps
+            // the loads of the current tile
+            int next = atomicAdd(&a.sched[0], 1);
+            while (ok) {
+                const int tile = next < total ? next : -1;
+                if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
+                if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                ring[r] = tile;
+                mbar_arrive(&rfull[r]);
+                if (++r == kRing) { r = 0; rph ^= 1u; }
+                if (tile < 0) {
+                    sent_end = true;
+                    break;
+                }
                 const Tile t = decode_tile(a, tile, tstart, off);
-                const int nb = a.swap ? (t.rows + 31) / 32 : 0;
-                const uint32_t bytes = a.swap ? kTileABytes + static_cast<uint32_t>(nb) * 4096u
-                                              : kTileABytes + static_cast<uint32_t>(a.BN) * 128u;
-                const int wrow = t.g * a.N + t.n0;
+                const PhaseArgs& pa = a.ph[t.phase];
+                if (t.phase == 1 && a.dep) {
+                    // all phase-0 tiles of this group must have stored their rows
+                    const int need = 4 * (tstart[t.g + 1] - tstart[t.g]);
+                    uint32_t i = 0;
+                    while (ld_acquire(&a.sched[1 + t.g]) < need) {
+                        if (++i > kWaitLimit || *abort_flag) {
+                            atomicCAS(a.status, 0, DEV_TIMEOUT_DEPENDENCY);
+                            *abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                        if (i > 64) __nanosleep(128);
+                    }
+                    fence_proxy_async_global();
+                    if (!ok) break;
+                }
+                const int nb = t.swap ? (t.rows + 31) / 32 : 0;
+                const uint32_t wbytes = t.swap ? 16384u : static_cast<uint32_t>(pa.BN) * 128u;
+                const uint32_t xbytes = t.swap ? static_cast<uint32_t>(nb) * 4096u : kTileABytes;
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], bytes);
-                    uint8_t* dA = sA + static_cast<size_t>(s) * kTileABytes;
-                    uint8_t* dB = sB + static_cast<size_t>(s) * a.stage_b_bytes;
+                    mbar_arrive_expect_tx(&full[s], wbytes + xbytes);
+                    uint8_t* dW = sW + static_cast<size_t>(s) * a.wslot;
+                    uint8_t* dX = sX + static_cast<size_t>(s) * a.xslot;
                     const int kx = kb * kBK;
-                    if (!a.swap) {
-                        tma_load_2d(&tm_tok, dA, &full[s], kx, static_cast<int32_t>(t.row0), pol_t);
-                        tma_load_2d(&tm_w, dB, &full[s], kx, wrow, pol_w);
-                    } else {
-                        tma_load_2d(&tm_w, dA, &full[s], kx, wrow, pol_w);
+                    if (t.swap) {
+                        // weights (M side): one contiguous 16 KB tile, streamed once
+                        bulk_load(dW, weight_rows(pa, t.g, t.n0, kb), 16384u, &full[s], pol_first);
                         for (int j = 0; j < nb; ++j)
-                            tma_load_2d(&tm_tok, dB + j * 4096, &full[s], kx,
-                                        static_cast<int32_t>(t.row0 + 32 * j), pol_t);
+                            tma_load_2d(&maps.tokB[t.phase], dX + j * 4096, &full[s], kx,
+                                        static_cast<int32_t>(t.row0 + 32 * j), pol_last);
+                    } else {
+                        // tokens (M side): 128 rows; weights: BN rows, reused by the
+                        // group's other row tiles from L2
+                        tma_load_2d(&maps.tokA[t.phase], dX, &full[s], kx, static_cast<int32_t>(t.row0), pol_norm);
+                        if (pa.BN >= 128) {
+                            for (int j = 0; j < pa.BN / 128; ++j)
+                                bulk_load(dW + j * 16384, weight_rows(pa, t.g, t.n0 + 128 * j, kb), 16384u, &full[s],
+                                          pol_norm);
+                        } else {
+                            bulk_load(dW, weight_rows(pa, t.g, t.n0, kb), wbytes, &full[s], pol_norm);
+                        }
                     }
                     issued_mask |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
             }
-            // Drain: every issued load has landed before the CTA may exit.
+            if (!sent_end) {
+                // a failed wait: hand the consumers the end marker (bounded)
+                for (uint32_t i = 0; i < kWaitLimit; ++i)
+                    if (mbar_try_wait(&rempty[r], rph ^ 1u)) break;
+                ring[r] = -1;
+                mbar_arrive(&rfull[r]);
+            }
+            // Drain: every issued copy has landed before the CTA may exit.
             for (int i = 0; i < S; ++i)
-                if (issued_mask & (1u << i)) {
-                    uint32_t p = (issued_ph >> i) & 1u;
+                if (issued_mask & (1u << i))
                     for (uint32_t it = 0; it < kWaitLimit; ++it)
-                        if (mbar_try_wait(&full[i], p)) break;
-                }
+                        if (mbar_try_wait(&full[i], (issued_ph >> i) & 1u)) break;
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
-            uint32_t s = 0, ph = 0;
+            uint32_t s = 0, ph = 0, r = 0, rph = 0;
             int it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+            while (ok) {
+                if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) break;
+                const int tile = ring[r];
+                mbar_arrive(&rempty[r]);
+                if (++r == kRing) { r = 0; rph ^= 1u; }
+                if (tile < 0) break;
                 const Tile t = decode_tile(a, tile, tstart, off);
                 const int buf = it & 1;
                 const uint32_t use = static_cast<uint32_t>(it >> 1);
-                if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+                ++it;
+                if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
-                const uint32_t n_mma = a.swap ? static_cast<uint32_t>((t.rows + 31) / 32) * 32u
-                                              : static_cast<uint32_t>(a.BN);
+                const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 31) / 32) * 32u
+                                              : static_cast<uint32_t>(a.ph[t.phase].BN);
                 const uint32_t idesc = umma_idesc_bf16(128, n_mma);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
@@ -264,13 +378,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok,
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(sA + static_cast<size_t>(s) * kTileABytes);
-                    const uint32_t b_base = smem_u32(sB + static_cast<size_t>(s) * a.stage_b_bytes);
+                    const uint32_t w_base = smem_u32(sW + static_cast<size_t>(s) * a.wslot);
+                    const uint32_t x_base = smem_u32(sX + static_cast<size_t>(s) * a.xslot);
+                    const uint32_t a_base = t.swap ? w_base : x_base;  // M side: weights or tokens
+                    const uint32_t b_base = t.swap ? x_base : w_base;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                    for (int kk = 0; kk < kBK / 16; ++kk)
                         umma_bf16(d_tmem, umma_desc_sw128(a_base + kk * 32), umma_desc_sw128(b_base + kk * 32),
                                   idesc, (kb > t.kb0 || kk > 0) ? 1u : 0u);
-                    }
                     umma_commit(&empty[s]);
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
@@ -284,38 +399,47 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok,
     } else {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        uint32_t r = 0, rph = 0;
         int it = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+        for (;;) {
+            if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            const int tile = ring[r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[r]);
+            if (++r == kRing) { r = 0; rph ^= 1u; }
+            if (tile < 0) break;
             const Tile t = decode_tile(a, tile, tstart, off);
+            const PhaseArgs& pa = a.ph[t.phase];
             const int buf = it & 1;
             const uint32_t use = static_cast<uint32_t>(it >> 1);
+            ++it;
             if (!mbar_wait(&tfull[buf], use & 1u, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf) * 256u +
                                    (static_cast<uint32_t>(q * 32) << 16);
             float v[32];
-            if (!a.swap) {
-                const int r = q * 32 + lane;
-                const bool valid = r < t.rows;
-                const int64_t grow = t.row0 + r;
-                const int nchunks = a.BN / 32;
+            if (!t.swap) {
+                const int rr = q * 32 + lane;
+                const bool valid = rr < t.rows;
+                const int64_t grow = t.row0 + rr;
+                const int nchunks = pa.BN / 32;
                 for (int c = 0; c < nchunks; ++c) {
                     tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
                     if (!valid) continue;
-                    if (a.epi == EPI_SWIGLU_BF16) {
+                    if (pa.epi == EPI_SWIGLU_BF16) {
                         uint32_t pk[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             pk[i] = pack_bf16x2(silu_f(v[2 * i]) * v[16 + 2 * i],
                                                 silu_f(v[2 * i + 1]) * v[16 + 2 * i + 1]);
-                        bf16* H = static_cast<bf16*>(a.out) + grow * a.ldo + (t.n0 / 2 + c * 16);
-                        uint4* dst = reinterpret_cast<uint4*>(H);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(pa.out) + grow * pa.ldo +
+                                                              (t.n0 / 2 + c * 16));
                         dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     } else {
                         const int col0 = t.n0 + c * 32;
-                        float* Y = static_cast<float*>(a.out) + grow * a.ldo + col0;
-                        if (col0 + 32 <= a.N_store && (a.ldo & 3) == 0) {  // float4 rows need 16 B alignment
+                        float* Y = static_cast<float*>(pa.out) + grow * pa.ldo + col0;
+                        if (col0 + 32 <= pa.N_store && (pa.ldo & 3) == 0) {  // float4 rows need 16 B alignment
                             float4* dst = reinterpret_cast<float4*>(Y);
 #pragma unroll
                             for (int i = 0; i < 8; ++i)
@@ -323,7 +447,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok,
                         } else {
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
-                                if (col0 + i < a.N_store) Y[i] = v[i];
+                                if (col0 + i < pa.N_store) Y[i] = v[i];
                         }
                     }
                 }
@@ -331,30 +455,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok,
                 const int nb = (t.rows + 31) / 32;
                 for (int c = 0; c < nb; ++c) {
                     tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
-                    if (a.epi == EPI_SWIGLU_BF16) {
+                    if (pa.epi == EPI_SWIGLU_BF16) {
                         const int f = t.n0 / 2 + q * 16 + (lane & 15);
-                        bf16* H = static_cast<bf16*>(a.out);
+                        bf16* H = static_cast<bf16*>(pa.out);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const float u = __shfl_xor_sync(0xffffffffu, v[j], 16);
                             const int tok = c * 32 + j;
                             if (lane < 16 && tok < t.rows)
-                                H[(t.row0 + tok) * a.ldo + f] = __float2bfloat16_rn(silu_f(v[j]) * u);
+                                H[(t.row0 + tok) * pa.ldo + f] = __float2bfloat16_rn(silu_f(v[j]) * u);
                         }
                     } else {
-                        float* Y = static_cast<float*>(a.out) + static_cast<int64_t>(t.split) * a.split_stride;
+                        float* Y = static_cast<float*>(pa.out) + static_cast<int64_t>(t.split) * pa.split_stride;
                         const int col = t.n0 + q * 32 + lane;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int tok = c * 32 + j;
-                            if (tok < t.rows && col < a.N_store) Y[(t.row0 + tok) * a.ldo + col] = v[j];
+                            if (tok < t.rows && col < pa.N_store) Y[(t.row0 + tok) * pa.ldo + col] = v[j];
                         }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (lane == 0) {
+                mbar_arrive(&tempty[buf]);
+                if (t.phase == 0 && a.dep) {
+                    // publish this warp's rows of H to the phase-1 tiles of group g
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(&a.sched[1 + t.g], 1);
+                }
+            }
         }
     }
 
@@ -386,7 +518,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
     cuuint64_t strides[1] = {cols * 2};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
     cuuint32_t es[2] = {1, 1};
@@ -402,85 +534,115 @@ int num_sms() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
     static int cached[64] = {0};
-    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    if (dev < 64) cached[dev] = n;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
     return n;
 }
 
+size_t gemm_sched_bytes(int G) { return static_cast<size_t>(G + 1) * sizeof(int); }
+
 // Returns 0 on success, -2 for an unsupported shape, -3 for a CUDA failure.
+// L.sched must point at gemm_sched_bytes(G) bytes that are zero when the
+// kernel starts.
 int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
-    if (L.G < 1 || L.G > kMaxGroups || L.Kdim < 16 || L.Kdim % 8 != 0 || L.N < 16) return -2;
+    if (L.G < 1 || L.G > kMaxGroups || L.nphase < 1 || L.nphase > 2 || !L.sched) return -2;
     DevArgs a{};
     a.group_off = L.group_off;
     a.G = L.G;
     a.dense_rows = L.dense_rows;
-    a.N = L.N;
-    a.N_store = L.N_store;
-    a.k_blocks = (L.Kdim + kBK - 1) / kBK;
-    a.swap = L.swap;
-    a.epi = L.epi;
-    a.out = L.out;
-    a.ldo = L.ldo;
-    a.split_stride = L.split_stride;
+    a.nphase = L.nphase;
+    a.dep = (L.nphase == 2) ? 1 : 0;
     a.status = L.status;
-    if (!L.swap) {
+    a.sched = L.sched;
+    const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
+    a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
+    {
+        const int64_t lim = mx < a.swap_max_rows ? mx : a.swap_max_rows;
+        a.BNs = static_cast<int>(lim >= 128 ? 128 : ((lim + 31) / 32) * 32);
+        if (a.BNs < 32) a.BNs = 32;
+    }
+    bool any_swap_possible = false;
+    uint32_t wslot = 0, xslot = kTileABytes;
+    for (int p = 0; p < L.nphase; ++p) {
+        const GemmPhase& g = L.ph[p];
+        if (g.Kdim < 16 || g.Kdim % 8 != 0 || g.N < 32) return -2;
+        PhaseArgs& ph = a.ph[p];
+        ph.w = g.w;
+        ph.w_group_elems = static_cast<int64_t>((g.N + 127) / 128) * ((g.Kdim + kBK - 1) / kBK) * 8192;
+        if ((reinterpret_cast<uintptr_t>(g.w) & 15u) != 0) return -2;
+        ph.N = g.N;
+        ph.N_store = g.N_store;
+        ph.k_blocks = (g.Kdim + kBK - 1) / kBK;
+        ph.epi = g.epi;
+        ph.out = g.out;
+        ph.ldo = g.ldo;
+        ph.split_stride = g.split_stride;
+        // Token-major tiles take the widest BN that divides N; when
+        // weight-major tiles are enabled (small groups expected) BN is capped
+        // at 128 so every weight slot is one 16 KB tile and the weight ring
+        // can be deep.
+        const int bn_cap = a.swap_max_rows > 0 ? 128 : 256;
         int bn = 0;
         for (int c : {256, 128, 64, 32})
-            if (L.N % c == 0) { bn = c; break; }
+            if (c <= bn_cap && g.N % c == 0) { bn = c; break; }
         if (bn == 0) return -2;
-        a.BN = bn;
-        a.ksplit = 1;
-        a.kb_per_split = a.k_blocks;
-    } else {
-        if (L.N % 128 != 0) return -2;
-        int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
-        a.BN = static_cast<int>(mx >= 128 ? 128 : ((mx + 31) / 32) * 32);
-        int ks = L.ksplit < 1 ? 1 : L.ksplit;
-        if (ks > a.k_blocks) ks = a.k_blocks;
-        a.kb_per_split = (a.k_blocks + ks - 1) / ks;
-        a.ksplit = (a.k_blocks + a.kb_per_split - 1) / a.kb_per_split;
+        if (g.epi == EPI_SWIGLU_BF16 && g.N % 32 != 0) return -2;
+        ph.BN = bn;
+        int ks = g.ksplit < 1 ? 1 : g.ksplit;
+        if (ks > ph.k_blocks) ks = ph.k_blocks;
+        ph.kb_per_split = (ph.k_blocks + ks - 1) / ks;
+        ph.ksplit = (ph.k_blocks + ph.kb_per_split - 1) / ph.kb_per_split;
+        wslot = wslot > static_cast<uint32_t>(bn) * 128u ? wslot : static_cast<uint32_t>(bn) * 128u;
+        if (g.N % 128 == 0 && a.swap_max_rows > 0) any_swap_possible = true;
     }
-    if (L.epi == EPI_SWIGLU_BF16 && (L.N % 32 != 0)) return -2;
-    a.stage_b_bytes = static_cast<uint32_t>(a.BN) * 128u;
-    const uint32_t stage = kTileABytes + a.stage_b_bytes;
-    const size_t fixed = 1024 + (2 * 8 + 5) * 8 + 16 + static_cast<size_t>(L.G + 1) * 12 + 64;
+    if (any_swap_possible) {
+        if (wslot < kTileABytes) wslot = kTileABytes;
+        const uint32_t xs = static_cast<uint32_t>(a.BNs) * 128u;
+        if (xs > xslot) xslot = xs;
+    }
+    a.wslot = wslot;
+    a.xslot = xslot;
+    const size_t fixed = 1024 + static_cast<size_t>(2 * 16 + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
+                         static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + 64;
     const size_t budget = 227 * 1024 - fixed;
-    int stages = static_cast<int>(budget / stage);
-    if (stages > 8) stages = 8;
+    int stages = static_cast<int>(budget / (wslot + xslot));
+    if (stages > 16) stages = 16;
     if (stages < 2) return -2;
     a.stages = stages;
-    const size_t smem = fixed + static_cast<size_t>(stages) * stage;
+    const size_t smem = fixed + static_cast<size_t>(stages) * (wslot + xslot);
 
-    CUtensorMap tm_tok, tm_w;
-    const uint64_t tok_rows = static_cast<uint64_t>(L.tok_rows < 1 ? 1 : L.tok_rows);
-    if (!make_map(&tm_tok, L.tok, tok_rows, static_cast<uint64_t>(L.Kdim),
-                  L.swap ? 32u : 128u))
-        return -3;
-    if (!make_map(&tm_w, L.w, static_cast<uint64_t>(L.G) * L.N, static_cast<uint64_t>(L.Kdim),
-                  L.swap ? 128u : static_cast<uint32_t>(a.BN)))
-        return -3;
+    Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    for (int p = 0; p < L.nphase; ++p) {
+        const GemmPhase& g = L.ph[p];
+        const uint64_t tok_rows = static_cast<uint64_t>(g.tok_rows < 1 ? 1 : g.tok_rows);
+        if (!make_map(&maps.tokA[p], g.tok, tok_rows, g.Kdim, 128u)) return -3;
+        if (!make_map(&maps.tokB[p], g.tok, tok_rows, g.Kdim, 32u)) return -3;
+    }
 
     static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024) != cudaSuccess)
+        if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess)
             return -3;
         attr_set = true;
     }
-    int sms = num_sms();
+    const int sms = num_sms();
     if (sms <= 0) return -3;
     // Upper bound on the tile count, to avoid idle CTAs on tiny problems.
-    int64_t rows_total = L.group_off ? L.tok_rows : L.dense_rows;
-    int64_t bound;
-    if (!L.swap) {
-        bound = ((rows_total + 127) / 128 + L.G) * (L.N / a.BN);
-    } else {
-        bound = ((rows_total + a.BN - 1) / a.BN + L.G) * (L.N / 128) * a.ksplit;
+    int64_t bound = 0;
+    for (int p = 0; p < L.nphase; ++p) {
+        const GemmPhase& g = L.ph[p];
+        const int64_t rows_total = L.group_off ? g.tok_rows : L.dense_rows;
+        const int64_t tm = ((rows_total + 127) / 128 + L.G) * (g.N / a.ph[p].BN);
+        const int64_t sw =
+            (g.N % 128 == 0) ? ((rows_total + a.BNs - 1) / a.BNs + L.G) * (g.N / 128) * a.ph[p].ksplit : 0;
+        bound += tm > sw ? tm : sw;
     }
-    int grid = static_cast<int>(bound < sms ? (bound < 1 ? 1 : bound) : sms);
-    grouped_gemm_kernel<<<grid, kThreads, smem, st>>>(tm_tok, tm_w, a);
+    const int grid = static_cast<int>(bound < sms ? (bound < 1 ? 1 : bound) : sms);
+    grouped_gemm_kernel<<<grid, kThreads, smem, st>>>(maps, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

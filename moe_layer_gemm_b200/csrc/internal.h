@@ -15,32 +15,37 @@ enum GemmEpilogue : int {
     EPI_F32 = 1,          // D stored as fp32
 };
 
-struct GemmLaunch {
-    // Token-side matrix [tok_rows, Kdim] bf16, K contiguous.
-    const bf16* tok;
+// One matrix product over all groups: out[rows of g] = tok[rows of g] . w[g]^T.
+struct GemmPhase {
+    const bf16* tok;      // [tok_rows, Kdim] bf16, K contiguous
     int64_t tok_rows;
-    // Weight matrix [G * N, Kdim] bf16, K contiguous (group g owns rows g*N ..).
-    const bf16* w;
-    int G;
-    int N;             // weight rows per group
-    int N_store;       // output columns actually written (<= N)
+    const bf16* w;        // per group a K-major [N, Kdim] matrix in 128 x 64 swizzled tiles
+                          // (tiled_offset), groups ceil(N/128) * ceil(Kdim/64) tiles apart
+    int N;                // weight rows per group
+    int N_store;          // output columns actually written (<= N)
     int Kdim;
-    // Groups: rows group_off[g] .. group_off[g+1]-1 of `tok` (device array), or
-    // a single group of dense_rows rows when group_off == nullptr.
+    int ksplit;           // reduction split of weight-major tiles (partial slices)
+    int epi;
+    void* out;
+    int64_t ldo;          // output row stride (elements)
+    int64_t split_stride; // elements between partial slices
+};
+
+struct GemmLaunch {
+    int G;
+    // Groups: rows group_off[g] .. group_off[g+1]-1 of the token matrices
+    // (device array), or a single group of dense_rows rows when NULL.
     const int32_t* group_off;
     int64_t dense_rows;
     int64_t max_group_rows;  // host-known upper bound on any group's rows
-    // Layout choice: 0 = token rows on the MMA M side (prefill-sized groups),
-    // 1 = weight rows on the M side and tokens on N (decode-sized groups).
-    int swap;
-    int ksplit;        // split of the reduction (swap == 1 only)
-    int epi;
-    void* out;
-    int64_t ldo;           // output row stride (elements)
-    int64_t split_stride;  // elements between split-K partial slices
-    int* status;           // device status word
+    int swap_max_rows;       // groups with at most this many rows use weight-major tiles
+    int nphase;              // 1, or 2: phase 1 of group g starts after phase 0 of g
+    GemmPhase ph[2];
+    int* status;             // device status word
+    int* sched;              // gemm_sched_bytes(G) bytes, zero at launch
 };
 
+size_t gemm_sched_bytes(int G);
 int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st);
 int num_sms();
 
@@ -52,6 +57,7 @@ int route_fused_supported(int d, int E);
 int route_blocks(int64_t T);
 int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, int E, int K,
                             int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st);
+// WrT: the router weight as a K-major [E_pad, d] matrix in 128 x 64 swizzled tiles.
 int launch_transpose_router(const bf16* Wr, int d, int E, int E_pad, bf16* WrT, cudaStream_t st);
 int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, float* prob_mean,
                          cudaStream_t st);
@@ -60,7 +66,8 @@ int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, 
 int permute_blocks(int64_t T);
 int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                    int32_t* block_hist, int32_t* counts, int32_t* kept, int32_t* offsets,
-                   int32_t* inv, int32_t* src, bf16* x_perm, int32_t* n_dropped, cudaStream_t st);
+                   int32_t* inv, int32_t* src, bf16* x_perm, int32_t* n_dropped, int32_t* zero_out,
+                   int zero_count, cudaStream_t st);
 
 // ------------------------------------------------------------ combine / stats
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv,
@@ -69,11 +76,16 @@ int launch_reduce_splits(const float* part, int nsplit, int64_t split_stride, co
                          int E, int d, float* y_perm, cudaStream_t st);
 int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E, int K,
                  float* f, float* aux, const float* alpha_bias_unused, cudaStream_t st);
+int launch_finalize_stats(const float* prob_part, int nblocks, const int32_t* counts, int64_t T, int E, int K,
+                          float* P, float* f, float* aux, cudaStream_t st);
+int launch_count(int64_t T);  // kernels launch_permute enqueues before the row gather
 int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias,
                        cudaStream_t st);
 
 // ------------------------------------------------------------ packing
 int launch_pack(const bf16* W1, const bf16* W3, const bf16* W2, int E, int d, int f, bf16* W13p,
                 bf16* W2p, cudaStream_t st);
+size_t packed_w13_bytes(int E, int d, int f);
+size_t packed_w2_bytes(int E, int d, int f);
 
 }  // namespace moe

@@ -6,16 +6,17 @@
 // offsets; section 3.1: an expert keeps at most C = CF * T * K / E
 // assignments and the overflow is dropped.
 //
-// Four launches, no atomics in any ordering decision:
-//   1. hist:   block b counts its tokens' selections per expert
-//   2. scan:   per expert, exclusive scan over blocks (rank base of block b),
-//              totals = counts, kept = min(counts, C), offsets = exclusive
-//              cumsum of kept, n_dropped
-//   3. rank:   each (t, k) gets rank = (# earlier tokens choosing the same
-//              expert): block base + earlier warps of the block + earlier
-//              lanes of the warp.  Kept iff rank < C; row = offsets[e] + rank
-//   4. gather: one warp per token reads x[t] once with 16-byte loads and
-//              writes it to each of its kept rows
+// The rank of (t, k) on expert e is the number of earlier tokens that chose
+// e.  It is assembled from three exact integer counts, never from the order
+// in which atomics happen to land:
+//   base of the block (earlier blocks)  + earlier warps of the block
+//   + earlier lanes of the warp (one __match_any_sync per slot).
+// Kept iff rank < C; row = offsets[e] + rank.
+//
+// Batches of at most kSmallT tokens take one fused single-CTA kernel
+// (count, scan, rank); larger ones take hist -> scan -> rank over many CTAs.
+// A gather kernel then copies each token row once per kept slot with
+// 16-byte loads, all of a lane's loads issued before its stores.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -26,7 +27,37 @@ namespace moe {
 namespace {
 
 constexpr int kTokPerBlock = 256;  // one token per thread in hist/rank
-constexpr int kMaxE = 1024;
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 16;
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallT = 1024;
+
+// Per-warp table used to count, for each of this lane's experts, the earlier
+// lanes of the warp that chose the same expert in any slot.
+struct WarpTable {
+    unsigned* mask;  // [E]
+    int* tag;        // [E]
+};
+
+__device__ __forceinline__ void warp_prefix(const int (&my)[kMaxK], int K, int lane, WarpTable tab, int gen,
+                                            int (&pre)[kMaxK]) {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) pre[k] = 0;
+    for (int k2 = 0; k2 < K; ++k2) {
+        const int v = my[k2];
+        const unsigned m = __match_any_sync(0xffffffffu, v);
+        if (v >= 0) {  // lanes with the same v write the same mask
+            tab.mask[v] = m;
+            tab.tag[v] = gen + k2;
+        }
+        __syncwarp();
+        for (int k = 0; k < K; ++k) {
+            const int e = my[k];
+            if (e >= 0 && tab.tag[e] == gen + k2) pre[k] += __popc(tab.mask[e] & lt);
+        }
+        __syncwarp();
+    }
+}
 
 __global__ void __launch_bounds__(kTokPerBlock)
 hist_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int32_t* __restrict__ block_hist) {
@@ -44,7 +75,9 @@ hist_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int32_t* _
 // block's rank base.
 __global__ void __launch_bounds__(1024)
 scan_kernel(int32_t* __restrict__ block_hist, int nblocks, int E, int64_t C, int32_t* __restrict__ counts,
-            int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped) {
+            int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
+            int32_t* __restrict__ zero_out, int zero_count) {
+    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_out[i] = 0;  // next kernel's scheduler words
     __shared__ int32_t sk[kMaxE];
     __shared__ int32_t sdrop[kMaxE];
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -62,15 +95,27 @@ scan_kernel(int32_t* __restrict__ block_hist, int nblocks, int E, int64_t C, int
         sdrop[e] = run - kp;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {  // E <= 1024: a serial exclusive scan is a few microseconds at most
-        int32_t run = 0, dr = 0;
-        for (int e = 0; e < E; ++e) {
-            offsets[e] = run;
-            run += sk[e];
-            dr += sdrop[e];
+    if (threadIdx.x < 32) {  // warp-level exclusive scan over E <= 256 (8 per lane)
+        const int lane = threadIdx.x;
+        const int per = (E + 31) / 32;
+        int s = 0, dsum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) { s += sk[e]; dsum += sdrop[e]; }
         }
-        offsets[E] = run;
-        if (n_dropped) *n_dropped = dr;
+        int incl = s;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - s;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) { offsets[e] = run; run += sk[e]; }
+        }
+        for (int o = 16; o >= 1; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+        if (lane == 31) offsets[E] = incl;
+        if (lane == 0 && n_dropped) *n_dropped = dsum;
     }
 }
 
@@ -79,28 +124,30 @@ rank_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int64_t C,
             const int32_t* __restrict__ block_base, const int32_t* __restrict__ offsets,
             int32_t* __restrict__ inv, int32_t* __restrict__ src) {
     constexpr int W = kTokPerBlock / 32;
-    constexpr int kMaxK = 16;
-    __shared__ int32_t wh[W][kMaxE / 4];  // per-warp histograms for E <= 256
-    __shared__ int32_t ids[W][32][kMaxK];
+    __shared__ int32_t wh[W][kMaxE];
+    __shared__ unsigned tmask[W][kMaxE];
+    __shared__ int tag[W][kMaxE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kTokPerBlock + threadIdx.x;
     const bool live = t < T;
-    for (int i = threadIdx.x; i < W * E; i += blockDim.x) wh[i / E][i % E] = 0;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) {
+        wh[i / E][i % E] = 0;
+        tag[i / E][i % E] = 0;
+    }
     __syncthreads();
     int my[kMaxK];
     for (int k = 0; k < K; ++k) {
         my[k] = live ? idx[t * K + k] : -1;
-        ids[warp][lane][k] = my[k];
         if (live) atomicAdd(&wh[warp][my[k]], 1);
     }
+    int pre[kMaxK];
+    warp_prefix(my, K, lane, WarpTable{tmask[warp], tag[warp]}, 1, pre);
     __syncthreads();
     if (!live) return;
     for (int k = 0; k < K; ++k) {
         const int e = my[k];
-        int32_t r = block_base[static_cast<int64_t>(blockIdx.x) * E + e];
+        int32_t r = block_base[static_cast<int64_t>(blockIdx.x) * E + e] + pre[k];
         for (int w2 = 0; w2 < warp; ++w2) r += wh[w2][e];
-        for (int j = 0; j < lane; ++j)
-            for (int k2 = 0; k2 < K; ++k2) r += (ids[warp][j][k2] == e) ? 1 : 0;
         if (C < 0 || r < C) {
             const int32_t row = offsets[e] + r;
             inv[t * K + k] = row;
@@ -111,14 +158,103 @@ rank_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int64_t C,
     }
 }
 
+// Whole dispatch of a batch of T <= kSmallT tokens in one CTA.
+__global__ void __launch_bounds__(kSmallThreads)
+dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int E, int K, int64_t C,
+                      int32_t* __restrict__ counts, int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
+                      int32_t* __restrict__ inv, int32_t* __restrict__ src, int32_t* __restrict__ n_dropped,
+                      int32_t* __restrict__ zero_out, int zero_count) {
+    constexpr int W = kSmallThreads / 32;
+    for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_out[i] = 0;  // next kernel's scheduler words
+    extern __shared__ int32_t sm[];
+    int32_t* wh = sm;                                              // [W][E]
+    unsigned* tmask = reinterpret_cast<unsigned*>(wh + W * E);     // [W][E]
+    int* tag = reinterpret_cast<int*>(tmask + W * E);              // [W][E]
+    int32_t* soff = tag + W * E;                                   // [E+1]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = threadIdx.x;
+    const bool live = t < T;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) {
+        wh[i] = 0;
+        tag[i] = 0;
+    }
+    __syncthreads();
+    int my[kMaxK];
+    for (int k = 0; k < K; ++k) {
+        my[k] = live ? idx[t * K + k] : -1;
+        if (live) atomicAdd(&wh[warp * E + my[k]], 1);
+    }
+    int pre[kMaxK];
+    warp_prefix(my, K, lane, WarpTable{tmask + warp * E, tag + warp * E}, 1, pre);
+    __syncthreads();
+    if (warp == 0) {
+        // totals, capacity, exclusive scan of kept counts, drops
+        const int per = (E + 31) / 32;
+        int s = 0, dsum = 0;
+        int kp_local[8];
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            int kp = 0;
+            if (e < E) {
+                int c = 0;
+                for (int w2 = 0; w2 < W; ++w2) c += wh[w2 * E + e];
+                kp = (C >= 0 && c > C) ? static_cast<int>(C) : c;
+                counts[e] = c;
+                kept[e] = kp;
+                dsum += c - kp;
+            }
+            kp_local[i] = kp;
+            s += kp;
+        }
+        int incl = s;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - s;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                soff[e] = run;
+                offsets[e] = run;
+            }
+            run += kp_local[i];
+        }
+        for (int o = 16; o >= 1; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+        if (lane == 31) offsets[E] = incl;
+        if (lane == 0 && n_dropped) *n_dropped = dsum;
+    }
+    __syncthreads();
+    if (!live) return;
+    for (int k = 0; k < K; ++k) {
+        const int e = my[k];
+        int r = pre[k];
+        for (int w2 = 0; w2 < warp; ++w2) r += wh[w2 * E + e];
+        if (C < 0 || r < C) {
+            const int row = soff[e] + r;
+            inv[t * K + k] = row;
+            src[row] = t;
+        } else {
+            inv[t * K + k] = -1;
+        }
+    }
+}
+
+constexpr int kGatherBatch = 8;
+
 __global__ void __launch_bounds__(256)
 gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ inv, int64_t T, int d, int K,
-              __nv_bfloat16* __restrict__ x_perm) {
+              int parts, __nv_bfloat16* __restrict__ x_perm) {
+    // `parts` warps share one token row, each copying a contiguous slice
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
     const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     const int nvec = d / 8;
-    for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp; t < T; t += nw) {
-        int32_t rows[16];
+    const int slice = (nvec + parts - 1) / parts;
+    for (int64_t job = gw; job < T * parts; job += nw) {
+        const int64_t t = job / parts;
+        const int p = static_cast<int>(job - t * parts);
+        int32_t rows[kMaxK];
         int nr = 0;
         for (int k = 0; k < K; ++k) {
             const int32_t r = inv[t * K + k];
@@ -126,10 +262,22 @@ gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ i
         }
         if (nr == 0) continue;
         const uint4* s = reinterpret_cast<const uint4*>(x + t * d);
-        for (int c = lane; c < nvec; c += 32) {
-            const uint4 v = __ldg(s + c);
-            for (int i = 0; i < nr; ++i)
-                reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(rows[i]) * d)[c] = v;
+        const int c_end = min(nvec, (p + 1) * slice);
+        for (int c0 = p * slice + lane; c0 < c_end; c0 += 32 * kGatherBatch) {
+            uint4 v[kGatherBatch];
+#pragma unroll
+            for (int b = 0; b < kGatherBatch; ++b) {
+                const int c = c0 + 32 * b;
+                if (c < c_end) v[b] = __ldg(s + c);
+            }
+            for (int i = 0; i < nr; ++i) {
+                uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(rows[i]) * d);
+#pragma unroll
+                for (int b = 0; b < kGatherBatch; ++b) {
+                    const int c = c0 + 32 * b;
+                    if (c < c_end) dst[c] = v[b];
+                }
+            }
         }
     }
 }
@@ -140,19 +288,40 @@ int permute_blocks(int64_t T) { return static_cast<int>((T + kTokPerBlock - 1) /
 
 int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                    int32_t* block_hist, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv,
-                   int32_t* src, bf16* x_perm, int32_t* n_dropped, cudaStream_t st) {
-    if (E > 256 || K > 16) return -2;
-    const int nb = permute_blocks(T);
-    hist_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, block_hist);
-    scan_kernel<<<1, 1024, 0, st>>>(block_hist, nb, E, C, counts, kept, offsets, n_dropped);
-    rank_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, C, block_hist, offsets, inv, src);
+                   int32_t* src, bf16* x_perm, int32_t* n_dropped, int32_t* zero_out, int zero_count,
+                   cudaStream_t st) {
+    if (E > kMaxE || K > kMaxK) return -2;
+    if (T <= kSmallT) {
+        const size_t smem = static_cast<size_t>(3 * (kSmallThreads / 32) * E + E + 1) * 4;
+        static bool attr = false;
+        if (!attr) {
+            if (cudaFuncSetAttribute(dispatch_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1) * 4) != cudaSuccess)
+                return -3;
+            attr = true;
+        }
+        dispatch_small_kernel<<<1, kSmallThreads, smem, st>>>(idx, static_cast<int>(T), E, K, C, counts, kept,
+                                                              offsets, inv, src, n_dropped, zero_out, zero_count);
+    } else {
+        const int nb = permute_blocks(T);
+        hist_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, block_hist);
+        scan_kernel<<<1, 1024, 0, st>>>(block_hist, nb, E, C, counts, kept, offsets, n_dropped, zero_out,
+                                        zero_count);
+        rank_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, C, block_hist, offsets, inv, src);
+    }
     if (x != nullptr && x_perm != nullptr) {
         const int sms = num_sms() > 0 ? num_sms() : 148;
-        int64_t need = (T + 7) / 8;
-        int grid = static_cast<int>(need < sms * 8 ? need : sms * 8);
-        gather_kernel<<<grid, 256, 0, st>>>(x, inv, T, d, K, x_perm);
+        // enough warps to cover the machine a few times over
+        int parts = 1;
+        while (parts < 16 && T * parts < static_cast<int64_t>(sms) * 32 && (d / 8) / (parts * 2) >= 32) parts *= 2;
+        const int64_t jobs = T * parts;
+        const int64_t need = (jobs + 7) / 8;
+        const int grid = static_cast<int>(need < sms * 16 ? need : sms * 16);
+        gather_kernel<<<grid, 256, 0, st>>>(x, inv, T, d, K, parts, x_perm);
     }
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
+
+int launch_count(int64_t T) { return T <= kSmallT ? 1 : 3; }
 
 }  // namespace moe

@@ -17,6 +17,7 @@ enum : int {
     DEV_TIMEOUT_MMA_TEMPTY = 3,
     DEV_TIMEOUT_EPI_TFULL = 4,
     DEV_TIMEOUT_DRAIN = 5,
+    DEV_TIMEOUT_DEPENDENCY = 6,
 };
 
 // About a few seconds of polling on a B200 before a wait gives up.
@@ -49,6 +50,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
                  "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
@@ -89,9 +100,37 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, void* smem_d
         : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` (multiple of 16; both
+// addresses 16-byte aligned), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)),
+          "l"(policy)
+        : "memory");
+}
+
+// Element offset of (row n, column k) of a K-major bf16 matrix stored as
+// 128-row x 64-column tiles (row-block-major, then column-block) with the
+// 128-byte swizzle inside each 16 KB tile: the 16-byte chunk c of row r sits
+// at chunk c ^ (r mod 8), as a 128-byte-swizzled TMA load would place it.
+__host__ __device__ __forceinline__ int64_t tiled_offset(int64_t n, int64_t k, int64_t k_blocks) {
+    const int64_t blk = (n >> 7) * k_blocks + (k >> 6);
+    const int r = static_cast<int>(n & 127), c = static_cast<int>(k & 63);
+    return blk * 8192 + r * 64 + ((((c >> 3) ^ (r & 7)) << 3) | (c & 7));
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 

@@ -25,6 +25,7 @@
 #include <cfloat>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -144,7 +145,11 @@ __device__ __forceinline__ void write_prob_partials(const float (&psum)[J], int 
 }
 
 // Fused router for E <= 32.  W_r is staged in shared memory as [d][8*EV]
-// bf16 rows (zero-padded), EV = 16-byte vectors per row.
+// bf16 rows (zero-padded), EV = 16-byte vectors per row.  Each lane loads
+// all of its 16-byte chunks of the token row before any arithmetic, so a
+// warp keeps up to kXBatch loads in flight instead of one.
+constexpr int kXBatch = 8;
+
 template <int EV>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr,
@@ -153,10 +158,24 @@ route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
                    float* __restrict__ prob_part) {
     constexpr int EP = EV * 8;  // padded experts per row
     extern __shared__ uint4 swr_raw[];
-    __nv_bfloat16* swr = reinterpret_cast<__nv_bfloat16*>(swr_raw);
-    for (int i = threadIdx.x; i < d * EP; i += blockDim.x) {
-        const int r = i / EP, e = i - r * EP;
-        swr[i] = e < E ? Wr[static_cast<int64_t>(r) * E + e] : __float2bfloat16_rn(0.f);
+    // 16-byte slot s of chunk c (8 rows = 8*EV slots) lives at s ^ (c & 7):
+    // the lanes of a quarter-warp read the same row of consecutive chunks,
+    // which would otherwise all fall in the same four banks.
+    if (E == EP) {
+        const uint4* src = reinterpret_cast<const uint4*>(Wr);
+        for (int i = threadIdx.x; i < d * EV; i += blockDim.x) swr_raw[i ^ ((i / (8 * EV)) & 7)] = __ldg(src + i);
+    } else {
+        for (int i = threadIdx.x; i < d * EV; i += blockDim.x) {
+            const int r = i / EV, vv = i - r * EV;
+            uint4 pk;
+            __nv_bfloat16* pe = reinterpret_cast<__nv_bfloat16*>(&pk);
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const int e = vv * 8 + h;
+                pe[h] = e < E ? Wr[static_cast<int64_t>(r) * E + e] : __float2bfloat16_rn(0.f);
+            }
+            swr_raw[i ^ ((i / (8 * EV)) & 7)] = pk;
+        }
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -169,28 +188,36 @@ route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
 #pragma unroll
         for (int e = 0; e < EP; ++e) acc[e] = 0.f;
         const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
-        for (int c = lane; c < nvec; c += 32) {
-            const uint4 xv = __ldg(xr + c);
-            const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
-            float xf[8];
+        for (int c0 = lane; c0 < nvec; c0 += 32 * kXBatch) {
+            uint4 xv[kXBatch];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f2 = __bfloat1622float2(xp[i]);
-                xf[2 * i] = f2.x;
-                xf[2 * i + 1] = f2.y;
+            for (int b = 0; b < kXBatch; ++b) {
+                const int c = c0 + 32 * b;
+                xv[b] = c < nvec ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint4* wrow = reinterpret_cast<const uint4*>(swr + static_cast<int64_t>(c * 8 + i) * EP);
+            for (int b = 0; b < kXBatch; ++b) {
+                const int c = c0 + 32 * b;
+                if (c >= nvec) break;
+                const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv[b]);
 #pragma unroll
-                for (int vv = 0; vv < EV; ++vv) {
-                    const uint4 wv = wrow[vv];
-                    const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&wv);
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    const float2 xf = __bfloat1622float2(xp[i2]);
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float2 w2 = __bfloat1622float2(wp[h]);
-                        acc[vv * 8 + 2 * h] = fmaf(xf[i], w2.x, acc[vv * 8 + 2 * h]);
-                        acc[vv * 8 + 2 * h + 1] = fmaf(xf[i], w2.y, acc[vv * 8 + 2 * h + 1]);
+                    for (int half = 0; half < 2; ++half) {
+                        const float xs = half ? xf.y : xf.x;
+                        const int slot0 = (c * 8 + 2 * i2 + half) * EV;
+#pragma unroll
+                        for (int vv = 0; vv < EV; ++vv) {
+                            const uint4 wv = swr_raw[(slot0 + vv) ^ (c & 7)];
+                            const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const float2 w2 = __bfloat1622float2(wp[h]);
+                                acc[vv * 8 + 2 * h] = fmaf(xs, w2.x, acc[vv * 8 + 2 * h]);
+                                acc[vv * 8 + 2 * h + 1] = fmaf(xs, w2.y, acc[vv * 8 + 2 * h + 1]);
+                            }
+                        }
                     }
                 }
             }
@@ -251,9 +278,10 @@ __global__ void transpose_router_kernel(const __nv_bfloat16* __restrict__ Wr, in
         tile[i][threadIdx.x] = (k < d && e < E) ? Wr[static_cast<int64_t>(k) * E + e] : __float2bfloat16_rn(0.f);
     }
     __syncthreads();
+    const int64_t kb = (d + 63) / 64;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int e = e0 + i, k = k0 + threadIdx.x;
-        if (e < E_pad && k < d) WrT[static_cast<int64_t>(e) * d + k] = tile[threadIdx.x][i];
+        if (e < E_pad && k < kb * 64) WrT[tiled_offset(e, k, kb)] = tile[threadIdx.x][i];  // zero past d and E
     }
 }
 
@@ -272,27 +300,26 @@ int route_fused_supported(int d, int E) {
     return static_cast<size_t>(d) * EP * 2 <= 96 * 1024 ? 1 : 0;
 }
 
+template <int EV>
+int launch_fused_ev(const bf16* x, const bf16* Wr, const float* bias, int64_t T, int d, int E, int K, float* logits,
+                    int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(route_fused_kernel<EV>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+            cudaSuccess)
+            return -3;
+        attr = true;
+    }
+    const size_t smem = static_cast<size_t>(d) * EV * 8 * 2;
+    route_fused_kernel<EV><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
 int launch_route_fused(const bf16* x, const bf16* Wr, const float* bias, int64_t T, int d, int E, int K,
                        float* logits, int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st) {
-    const int EV = E <= 8 ? 1 : (E <= 16 ? 2 : 4);
-    const size_t smem = static_cast<size_t>(d) * EV * 8 * 2;
-    cudaError_t err;
-    switch (EV) {
-        case 1:
-            cudaFuncSetAttribute(route_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-            route_fused_kernel<1><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
-            break;
-        case 2:
-            cudaFuncSetAttribute(route_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-            route_fused_kernel<2><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
-            break;
-        default:
-            cudaFuncSetAttribute(route_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-            route_fused_kernel<4><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
-            break;
-    }
-    err = cudaGetLastError();
-    return err == cudaSuccess ? 0 : -3;
+    if (E <= 8) return launch_fused_ev<1>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
+    if (E <= 16) return launch_fused_ev<2>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
+    return launch_fused_ev<4>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
 }
 
 int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, int E, int K, int32_t* idx,
@@ -318,7 +345,7 @@ int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, 
 }
 
 int launch_transpose_router(const bf16* Wr, int d, int E, int E_pad, bf16* WrT, cudaStream_t st) {
-    dim3 grid((d + 31) / 32, (E_pad + 31) / 32), block(32, 8);
+    dim3 grid(((d + 63) / 64) * 2, (E_pad + 31) / 32), block(32, 8);  // columns up to the tile padding
     transpose_router_kernel<<<grid, block, 0, st>>>(Wr, d, E, E_pad, WrT);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }

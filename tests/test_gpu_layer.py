@@ -108,3 +108,28 @@ def test_layer_bias_update_in_place():
     ref = oracle_layer(inp, bias32=np.zeros(wl.E, np.float32), alpha=1e-3)
     assert np.array_equal(outs["counts"].cpu().numpy(), ref["counts"])
     assert np.array_equal(bias.cpu().numpy().view(np.uint32), ref["bias"].view(np.uint32))
+
+
+@pytest.mark.parametrize("name,ntok", [("mixtral_decode", 24), ("mixtral_prefill", 16), ("qwen_capacity", 24),
+                                       ("deepseek_bias", 10)])
+def test_layer_full_size_sampled(name, ntok):
+    """Each workload at its full size, in the launch configuration bench.py
+    times; the fp64 oracle evaluates a spread of sampled tokens (routing,
+    counts and capacity always over the whole batch)."""
+    inp = LayerInputs(synth.get_workload(name))
+    T = inp.T
+    bias = b32 = None
+    if inp.wl.use_bias:
+        bias = torch.zeros(inp.wl.E, dtype=torch.float32, device=dev())
+        b32 = np.zeros(inp.wl.E, np.float32)
+    y, outs = _forward(inp, bias)
+    tokens = sorted(set(np.linspace(0, T - 1, ntok).astype(int).tolist()))
+    ref = oracle_layer(inp, bias32=b32, tokens=tokens)
+    rows = _check(inp, y, outs, ref, bias32=b32, tokens=tokens)
+    assert len(rows) >= len(tokens) - 2
+    # every token's output is finite and dropped-everything tokens are exactly 0
+    yg = f64(y)
+    assert np.all(np.isfinite(yg))
+    inv = outs["inv"].cpu().numpy()
+    dead = np.all(inv < 0, axis=1)
+    assert np.all(yg[dead] == 0)
