@@ -205,6 +205,7 @@ int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t*
     g.dense_rows = 0;
     g.max_group_rows = maxrows;
     g.swap_max_rows = L.swap ? kSwapMaxRows : 0;
+    g.small_groups = (d->T * d->K) < static_cast<int64_t>(d->E) * 128;
     g.nphase = 2;
     GemmPhase& p0 = g.ph[0];
     p0.tok = xperm;

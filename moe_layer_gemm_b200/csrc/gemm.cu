@@ -262,8 +262,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             // ------------------------------------------- scheduler + producer
             const uint64_t pol_first = policy_evict_first();
             const uint64_t pol_last = policy_evict_last();
-            const uint64_t pol_norm = policy_evict_normal();
-            uint32_t s = 0, ph = 0, r = 0, rph = 0;
+                    uint32_t s = 0, ph = 0, r = 0, rph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool ok = true;
             bool sent_end = false;
@@ -321,15 +320,16 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                             tma_load_2d(&maps.tokB[t.phase], dX + j * 4096, &full[s], kx,
                                         static_cast<int32_t>(t.row0 + 32 * j), pol_last);
                     } else {
-                        // tokens (M side): 128 rows; weights: BN rows, reused by the
-                        // group's other row tiles from L2
-                        tma_load_2d(&maps.tokA[t.phase], dX, &full[s], kx, static_cast<int32_t>(t.row0), pol_norm);
+                        // tokens (M side): 128 rows, kept in L2 for the group's other
+                        // weight tiles; weights: BN rows, marked first to leave L2
+                        // once the group's row tiles (running together) have read them
+                        tma_load_2d(&maps.tokA[t.phase], dX, &full[s], kx, static_cast<int32_t>(t.row0), pol_last);
                         if (pa.BN >= 128) {
                             for (int j = 0; j < pa.BN / 128; ++j)
                                 bulk_load(dW + j * 16384, weight_rows(pa, t.g, t.n0 + 128 * j, kb), 16384u, &full[s],
-                                          pol_norm);
+                                          pol_first);
                         } else {
-                            bulk_load(dW, weight_rows(pa, t.g, t.n0, kb), wbytes, &full[s], pol_norm);
+                            bulk_load(dW, weight_rows(pa, t.g, t.n0, kb), wbytes, &full[s], pol_first);
                         }
                     }
                     issued_mask |= 1u << s;
@@ -579,11 +579,11 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         ph.out = g.out;
         ph.ldo = g.ldo;
         ph.split_stride = g.split_stride;
-        // Token-major tiles take the widest BN that divides N; when
-        // weight-major tiles are enabled (small groups expected) BN is capped
-        // at 128 so every weight slot is one 16 KB tile and the weight ring
-        // can be deep.
-        const int bn_cap = a.swap_max_rows > 0 ? 128 : 256;
+        // Token-major tiles take the widest BN that divides N.  When groups
+        // are expected to be small (mean below 128 rows) BN is capped at 128,
+        // so a weight slot is the same 16 KB a weight-major tile needs and
+        // the operand ring stays deep.
+        const int bn_cap = L.small_groups ? 128 : 256;
         int bn = 0;
         for (int c : {256, 128, 64, 32})
             if (c <= bn_cap && g.N % c == 0) { bn = c; break; }
