@@ -77,6 +77,7 @@ enum {
     MOE_ECUDA = -3,        /* a CUDA runtime call failed (launch error, no device) */
     MOE_EWORKSPACE = -4,   /* workspace too small */
     MOE_ETIMEOUT = -5,     /* a device-side bounded wait ran out (from moe_get_device_status) */
+    MOE_ESCRATCH = -6,     /* batch too large for the static scratch of moe_permute_noalloc */
 };
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -165,6 +166,34 @@ MOE_API int moe_route_from_logits(const moe_dims* dims, const float* logits, con
 MOE_API int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x,
                 int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
                 moe_bf16* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 3 for callers that cannot allocate: the same dispatch as
+ * moe_permute (same arguments, outputs and ordering, bit for bit) with no
+ * workspace argument.  Some callers cannot hand the library device memory:
+ * a plugin or runtime that owns every device buffer and exposes no
+ * allocator to its extensions, or a serving loop where an allocation (or
+ * the device synchronisation an allocator may trigger) is not allowed
+ * between steps.  This entry point allocates nothing and calls no
+ * allocating routine.
+ *
+ * Its scratch (the per-block histogram, ceil(T / 256) * E int32 values) is
+ * a fixed 256 KB array inside the library, held by every GPU that loads the
+ * library until the process exits.  Batches with ceil(T / 256) * E > 65536
+ * are rejected with MOE_ESCRATCH (e.g. T <= 65536 tokens at E = 256).
+ * Batches of at most 1024 tokens need no scratch at all.
+ *
+ * The first call on each device looks up the array's device address (a
+ * one-time host-side set-up, with that device current), so make that first
+ * call before any stream capture.  All calls share the array and it keeps
+ * the last call's contents; every value a call reads is written earlier in
+ * the same call, so no clearing is needed, but calls whose work overlaps on
+ * the same GPU (for example on two streams) race on it: serialise them.
+ *
+ * There is no counterpart of this entry point on the source pages; it
+ * exists for the callers described above. */
+MOE_API int moe_permute_noalloc(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x,
+                                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv,
+                                int32_t* src, moe_bf16* x_perm, int32_t* n_dropped, void* stream);
 
 /* Step 4: grouped SwiGLU expert FFN on the rows of each expert ([P2]
  * section 2 step 3; section 2.2: experts only see their own tokens).

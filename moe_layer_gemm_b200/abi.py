@@ -25,12 +25,13 @@ MOE_EUNSUPPORTED = -2
 MOE_ECUDA = -3
 MOE_EWORKSPACE = -4
 MOE_ETIMEOUT = -5
+MOE_ESCRATCH = -6
 
 EXPORTED = [
     "moe_status_str", "moe_version", "moe_capacity", "moe_workspace_size", "moe_reset_device_status",
     "moe_get_device_status", "moe_pack_weights", "moe_route", "moe_route_from_logits", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
-    "moe_layer_launch_count", "moe_packed_weight_bytes",
+    "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -83,6 +84,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_layer_forward": (I, [dims_p, P, P, P, F, P, P, P, ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
         "moe_layer_launch_count": (I, [dims_p, I, I]),
         "moe_packed_weight_bytes": (I, [dims_p, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
+        "moe_permute_noalloc": (I, [dims_p, P, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -206,6 +208,15 @@ def moe_permute(dims, topk_idx, x, counts, kept, offsets, inv, src, x_perm, n_dr
         _ptr(counts, I32, "counts"), _ptr(kept, I32, "kept"), _ptr(offsets, I32, "offsets"),
         _ptr(inv, I32, "inv"), _ptr(src, I32, "src"), _ptr(x_perm, BF16, "x_perm"),
         _ptr(n_dropped, I32, "n_dropped"), _ptr(ws, None, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_permute_noalloc(dims, topk_idx, x, counts, kept, offsets, inv, src, x_perm, n_dropped, stream=None):
+    """moe_permute without a workspace (scratch held inside the library)."""
+    _check("moe_permute_noalloc", load().moe_permute_noalloc(
+        ctypes.byref(_dims(dims)), _ptr(topk_idx, I32, "topk_idx"), _ptr(x, BF16, "x"),
+        _ptr(counts, I32, "counts"), _ptr(kept, I32, "kept"), _ptr(offsets, I32, "offsets"),
+        _ptr(inv, I32, "inv"), _ptr(src, I32, "src"), _ptr(x_perm, BF16, "x_perm"),
+        _ptr(n_dropped, I32, "n_dropped"), _stream(stream)))
 
 
 def moe_expert_ffn(dims, x_perm, offsets, W13p, W2p, h, y_perm, ws, stream=None):

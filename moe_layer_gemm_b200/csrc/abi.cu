@@ -248,6 +248,7 @@ const char* moe_status_str(int s) {
         case MOE_ECUDA: return "MOE_ECUDA: CUDA runtime error";
         case MOE_EWORKSPACE: return "MOE_EWORKSPACE: workspace too small";
         case MOE_ETIMEOUT: return "MOE_ETIMEOUT: a device-side wait ran out";
+        case MOE_ESCRATCH: return "MOE_ESCRATCH: batch too large for the library's static scratch";
         default: return "unknown status";
     }
 }
@@ -361,6 +362,22 @@ int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* 
         MOE_TRY(map_launch(launch_reduce_splits(yout, L.nsplit, dims->T * dims->K * dims->d_model, offsets, dims->E,
                                                 dims->d_model, y_perm, st)));
     return MOE_OK;
+}
+
+int moe_permute_noalloc(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x, int32_t* counts,
+                        int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src, moe_bf16* x_perm,
+                        int32_t* n_dropped, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!topk_idx || !counts || !kept || !offsets || !inv || !src) return MOE_EINVAL;
+    if ((x == nullptr) != (x_perm == nullptr)) return MOE_EINVAL;
+    if (x && (!aligned16(x) || !aligned16(x_perm))) return MOE_EUNSUPPORTED;
+    if (static_cast<int64_t>(permute_blocks(dims->T)) * dims->E > permute_static_max_hist()) return MOE_ESCRATCH;
+    const int r = launch_permute_static(topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model,
+                                        dims->E, dims->K, capacity_of(dims), counts, kept, offsets, inv, src,
+                                        reinterpret_cast<bf16*>(x_perm), n_dropped,
+                                        static_cast<cudaStream_t>(stream));
+    if (r == -2) return MOE_ESCRATCH;
+    return map_launch(r);
 }
 
 int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* inv, const float* topk_w, float* y,

@@ -80,6 +80,10 @@ int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E
 int launch_finalize_stats(const float* prob_part, int nblocks, const int32_t* counts, int64_t T, int E, int K,
                           float* P, float* f, float* aux, cudaStream_t st);
 int launch_count(int64_t T);  // kernels launch_permute enqueues before the row gather
+int64_t permute_static_max_hist();
+int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
+                          int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
+                          bf16* x_perm, int32_t* n_dropped, cudaStream_t st);
 int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias,
                        cudaStream_t st);
 

@@ -20,6 +20,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "internal.h"
 
 namespace moe {
@@ -323,5 +325,53 @@ int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, i
 }
 
 int launch_count(int64_t T) { return T <= kSmallT ? 1 : 3; }
+
+// ------------------------------------------------------------------------
+// Dispatch without a caller-provided workspace.
+//
+// The only scratch the dispatch kernels need is the per-block histogram /
+// rank-base table (ceil(T/256) x E int32).  Here it lives in a file-scope
+// device array that every GPU loading this library holds until the process
+// exits.  All calls share it: each call writes every element it reads
+// before reading it, so nothing has to be cleared between calls, but two
+// calls whose kernels overlap on the same GPU (different streams) race on
+// it.  Host code cannot use the array's name as a device address; its
+// address is looked up once per device with cudaGetSymbolAddress.
+namespace {
+
+constexpr int64_t kStaticHistInts = int64_t(1) << 16;  // 256 KB
+static __device__ __align__(256) int32_t g_dispatch_scratch[kStaticHistInts];
+
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[64] = {nullptr};
+
+// Device address of g_dispatch_scratch on the current device, looked up on
+// first use; nullptr if the lookup fails.
+int32_t* dispatch_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess) return nullptr;
+        g_scratch_addr[dev] = p;
+    }
+    return static_cast<int32_t*>(g_scratch_addr[dev]);
+}
+
+}  // namespace
+
+int64_t permute_static_max_hist() { return kStaticHistInts; }
+
+// -2: the batch needs more scratch than the static array holds; -3: CUDA failure.
+int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
+                          int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
+                          bf16* x_perm, int32_t* n_dropped, cudaStream_t st) {
+    if (static_cast<int64_t>(permute_blocks(T)) * E > kStaticHistInts) return -2;
+    int32_t* scratch = dispatch_scratch_address();
+    if (scratch == nullptr) return -3;
+    return launch_permute(idx, x, T, d, E, K, C, scratch, counts, kept, offsets, inv, src, x_perm, n_dropped,
+                          nullptr, 0, st);
+}
 
 }  // namespace moe

@@ -93,3 +93,11 @@ def test_workspace_grows_with_problem(lib):
     # at least x_perm + h + y_perm for the big case
     A = 16384 * 2
     assert big >= A * 4096 * 2 + A * 14336 * 2 + A * 4096 * 4
+
+
+def test_noalloc_dispatch_rejects_oversize_on_the_host(lib):
+    d = abi.Dims(70000, 64, 64, 256, 8).c()   # ceil(T/256) * E = 70144 > 65536 scratch entries
+    fake = ctypes.c_void_p(0x10000)            # never dereferenced: the size check fails first
+    st = lib.moe_permute_noalloc(ctypes.byref(d), fake, None, fake, fake, fake, fake, fake, None, None, None)
+    assert st == abi.MOE_ESCRATCH
+    assert abi.moe_status_str(abi.MOE_ESCRATCH).startswith("MOE_ESCRATCH")
