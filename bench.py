@@ -157,6 +157,22 @@ def profile_traffic(workload: str):
         return None
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The maximum of `value` over all ranks (the value itself without a
+    process group).  Multi-GPU timings are reported as the slowest rank."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(T: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own T tokens per step."""
+    return T * world / (ms_per_step * 1e-3)
+
+
 # --------------------------------------------------------------- oracle timing
 
 def time_oracle(wl, x_h, Wr_h, W1_h, W3_h, W2_h, tokens, bias32=None, steps=1):
@@ -312,11 +328,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms_total = start.elapsed_time(end)
-    if pg:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), dev)
     ms_step = ms_total / K
     stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in range(K)])
     stage_ms = stage.mean(axis=0)
@@ -371,11 +383,7 @@ def run_ours(args):
     e1.record(s)
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = e0.elapsed_time(e1) / E2E
-    if pg:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / E2E, dev)
 
     launches = abi.moe_layer_launch_count(dims, True, bias is not None and alpha != 0.0) * K
 
@@ -394,7 +402,7 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
     if rank != 0:
         return 0
-    value = wl.T * world / (ms_step * 1e-3)
+    value = job_tokens_per_s(wl.T, world, ms_step)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -412,7 +420,7 @@ def run_ours(args):
                     "max_over_mean_load": float(counts.max() / (wl.T * wl.K / wl.E)),
                     "count_cv": float(counts.std() / counts.mean()), "n_dropped": int(outs["n_dropped"].item())},
         "cpu_baseline": cpu,
-        "e2e": {"value": wl.T * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(wl.T, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
         "gpu_launches": launches,
         "clocks": clk,
