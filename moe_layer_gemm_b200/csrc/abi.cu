@@ -167,6 +167,7 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
         g.dense_rows = d->T;
         g.max_group_rows = d->T;
         g.swap_max_rows = 0;
+        g.bn_max = 64;  // narrow tiles: more CTAs share the logits GEMM (N = E_pad is small)
         g.nphase = 1;
         g.ph[0].tok = x;
         g.ph[0].tok_rows = d->T;

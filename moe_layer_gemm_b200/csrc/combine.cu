@@ -25,10 +25,14 @@ constexpr int kMaxK = 16;
 
 constexpr int kMaxSplit = 8;
 
+// S >= nsplit slots for partial slices (S == nsplit except the 8-slot
+// fallback, which reads only the nsplit slices that exist).
+template <int S>
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, const int32_t* __restrict__ inv,
                const float* __restrict__ w, int64_t T, int d, int K, float* __restrict__ y) {
     const int nvec = d / 4;
+    const int64_t svec = split_stride / 4;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         int32_t rows[kMaxK];
         float ws[kMaxK];
@@ -38,21 +42,37 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
         }
         for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k < K; ++k) {
-                if (rows[k] < 0) continue;
-                const float4* base = reinterpret_cast<const float4*>(yp + static_cast<int64_t>(rows[k]) * d) + c;
-                float4 part[kMaxSplit];
+            // slots in groups of four: a group's loads are all issued before
+            // its arithmetic; slices are summed in slice order and slots
+            // accumulated in slot order
+            for (int k0 = 0; k0 < K; k0 += 4) {
+                float4 v[4][S];
 #pragma unroll
-                for (int s = 0; s < kMaxSplit; ++s)   // all slices in flight, then summed in slice order
-                    if (s < nsplit) part[s] = __ldg(base + s * (split_stride / 4));
-                float4 v = part[0];
+                for (int j = 0; j < 4; ++j) {
+                    const int k = k0 + j;
+                    const bool live = k < K && rows[k] >= 0;
+                    const float4* base =
+                        reinterpret_cast<const float4*>(yp + static_cast<int64_t>(live ? rows[k] : 0) * d) + c;
 #pragma unroll
-                for (int s = 1; s < kMaxSplit; ++s)
-                    if (s < nsplit) { v.x += part[s].x; v.y += part[s].y; v.z += part[s].z; v.w += part[s].w; }
-                acc.x = fmaf(ws[k], v.x, acc.x);
-                acc.y = fmaf(ws[k], v.y, acc.y);
-                acc.z = fmaf(ws[k], v.z, acc.z);
-                acc.w = fmaf(ws[k], v.w, acc.w);
+                    for (int sl = 0; sl < S; ++sl)
+                        v[j][sl] = (live && sl < nsplit) ? __ldg(base + sl * svec) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = k0 + j;
+                    if (k < K && rows[k] >= 0) {
+                        float4 u = v[j][0];
+#pragma unroll
+                        for (int sl = 1; sl < S; ++sl)
+                            if (sl < nsplit) {
+                                u.x += v[j][sl].x; u.y += v[j][sl].y; u.z += v[j][sl].z; u.w += v[j][sl].w;
+                            }
+                        acc.x = fmaf(ws[k], u.x, acc.x);
+                        acc.y = fmaf(ws[k], u.y, acc.y);
+                        acc.z = fmaf(ws[k], u.z, acc.z);
+                        acc.w = fmaf(ws[k], u.w, acc.w);
+                    }
+                }
             }
             reinterpret_cast<float4*>(y + t * d)[c] = acc;
         }
@@ -96,28 +116,40 @@ stats_kernel(const int32_t* __restrict__ counts, const float* __restrict__ P, in
     if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
 }
 
-// One block: P_i = (sum over router blocks of the per-block sums) / T, in
-// block order; then f_i and aux as in stats_kernel.
-__global__ void __launch_bounds__(256)
+// One block of 1024 threads: P_i = (sum over router blocks of the per-block
+// sums) / T.  Warp w reduces experts w, w+32, ...: lane l adds blocks l,
+// l+32, ... in order, then a fixed butterfly across lanes; f_i and aux as in
+// stats_kernel.  Every sum has a fixed order, so results are reproducible.
+__device__ __forceinline__ float warp_sum_fixed(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__global__ void __launch_bounds__(1024)
 finalize_stats_kernel(const float* __restrict__ part, int nblocks, const int32_t* __restrict__ counts, int64_t T,
                       int E, int K, float* __restrict__ P, float* __restrict__ f, float* __restrict__ aux) {
-    __shared__ float red[256];
+    __shared__ float red[1024];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const float invT = 1.0f / static_cast<float>(T);
     const float invA = 1.0f / static_cast<float>(T * K);
     float acc = 0.f;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    for (int e = warp; e < E; e += nw) {
         float s = 0.f;
-        for (int b = 0; b < nblocks; ++b) s += part[static_cast<int64_t>(b) * E + e];
+        for (int b = lane; b < nblocks; b += 32) s += part[static_cast<int64_t>(b) * E + e];
+        s = warp_sum_fixed(s);
         const float pe = s * invT;
         const float fe = static_cast<float>(counts[e]) * invA;
-        P[e] = pe;
-        if (f) f[e] = fe;
-        acc += fe * pe;
+        if (lane == 0) {
+            if (P) P[e] = pe;
+            if (f) f[e] = fe;
+            acc += fe * pe;
+        }
     }
     red[threadIdx.x] = acc;
     __syncthreads();
-    for (int s = blockDim.x / 2; s > 0; s >>= 1) {
-        if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+        if (threadIdx.x < st) red[threadIdx.x] += red[threadIdx.x + st];
         __syncthreads();
     }
     if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
@@ -186,12 +218,19 @@ __global__ void pack_w2_kernel(const __nv_bfloat16* __restrict__ W2, int d, int 
 
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv, const float* w,
                    int64_t T, int d, int K, float* y, cudaStream_t st) {
-    if (K > kMaxK || d % 4 != 0 || nsplit > kMaxSplit) return -2;
+    if (K > kMaxK || d % 4 != 0 || nsplit < 1 || nsplit > kMaxSplit) return -2;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     int64_t grid = T < static_cast<int64_t>(sms) * 16 ? T : static_cast<int64_t>(sms) * 16;
-    int threads = d / 4 >= 256 ? 256 : ((d / 4 + 31) / 32) * 32;
-    combine_kernel<<<static_cast<int>(grid < 1 ? 1 : grid), threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w,
-                                                                             T, d, K, y);
+    if (grid < 1) grid = 1;
+    const int threads = d / 4 >= 256 ? 256 : ((d / 4 + 31) / 32) * 32;
+    const int g = static_cast<int>(grid);
+    switch (nsplit) {
+        case 1: combine_kernel<1><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
+        case 2: combine_kernel<2><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
+        case 3: combine_kernel<3><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
+        case 4: combine_kernel<4><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
+        default: combine_kernel<8><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
+    }
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
@@ -210,7 +249,7 @@ int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E
 
 int launch_finalize_stats(const float* prob_part, int nblocks, const int32_t* counts, int64_t T, int E, int K,
                           float* P, float* f, float* aux, cudaStream_t st) {
-    finalize_stats_kernel<<<1, 256, 0, st>>>(prob_part, nblocks, counts, T, E, K, P, f, aux);
+    finalize_stats_kernel<<<1, 1024, 0, st>>>(prob_part, nblocks, counts, T, E, K, P, f, aux);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

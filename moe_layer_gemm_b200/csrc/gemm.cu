@@ -583,7 +583,8 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         // are expected to be small (mean below 128 rows) BN is capped at 128,
         // so a weight slot is the same 16 KB a weight-major tile needs and
         // the operand ring stays deep.
-        const int bn_cap = L.small_groups ? 128 : 256;
+        int bn_cap = L.small_groups ? 128 : 256;
+        if (L.bn_max > 0 && L.bn_max < bn_cap) bn_cap = L.bn_max;
         int bn = 0;
         for (int c : {256, 128, 64, 32})
             if (c <= bn_cap && g.N % c == 0) { bn = c; break; }

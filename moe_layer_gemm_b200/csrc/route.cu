@@ -32,6 +32,7 @@ namespace moe {
 namespace {
 
 constexpr int kRouteWarps = 8;
+constexpr int64_t kSplitRouteMaxT = 512;  // batches up to this size take one CTA per token
 
 // Warp-wide top-K over values v[j] of expert (lane + 32 j), j < J.
 // Returns, in lane r < K, the r-th selected (value, expert); other lanes get
@@ -235,6 +236,95 @@ route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
     if (want_prob) write_prob_partials<1>(psum, E, prob_part);
 }
 
+// Small batches (decode): one CTA per token, its hidden dimension split
+// across the 8 warps so the whole machine shares the latency chain.  W_r is
+// read through L1 (each warp touches only its slice of rows).  Per-warp
+// partial logits are summed in warp order in shared memory, then warp 0
+// selects.  prob_part gets one row per CTA (= per token).
+template <int EV>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_split_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr,
+                   const float* __restrict__ bias, int64_t T, int d, int E, int K, float* __restrict__ logits,
+                   int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ prob_part) {
+    constexpr int EP = EV * 8;
+    __shared__ float part[kRouteWarps][EP];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nvec = d / 8;
+    const int per_warp = (nvec + kRouteWarps - 1) / kRouteWarps;
+    const int c_beg = warp * per_warp, c_end = min(nvec, c_beg + per_warp);
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        float acc[EP];
+#pragma unroll
+        for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+        for (int c0 = c_beg + lane; c0 < c_end; c0 += 32 * kXBatch) {
+            uint4 xv[kXBatch];
+#pragma unroll
+            for (int b = 0; b < kXBatch; ++b) {
+                const int c = c0 + 32 * b;
+                xv[b] = c < c_end ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int b = 0; b < kXBatch; ++b) {
+                const int c = c0 + 32 * b;
+                if (c >= c_end) break;
+                const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv[b]);
+#pragma unroll
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    const float2 xf = __bfloat1622float2(xp[i2]);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const float xs = half ? xf.y : xf.x;
+                        const int row = c * 8 + 2 * i2 + half;
+                        if (E == EP) {  // a W_r row is EV whole 16-byte vectors
+                            const uint4* wrow = reinterpret_cast<const uint4*>(Wr + static_cast<int64_t>(row) * EP);
+#pragma unroll
+                            for (int vv = 0; vv < EV; ++vv) {
+                                const uint4 wv = __ldg(wrow + vv);
+                                const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+                                for (int h = 0; h < 4; ++h) {
+                                    const float2 w2 = __bfloat1622float2(wp[h]);
+                                    acc[vv * 8 + 2 * h] = fmaf(xs, w2.x, acc[vv * 8 + 2 * h]);
+                                    acc[vv * 8 + 2 * h + 1] = fmaf(xs, w2.y, acc[vv * 8 + 2 * h + 1]);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < EP; ++e) {
+                                const float wv =
+                                    e < E ? __bfloat162float(__ldg(Wr + static_cast<int64_t>(row) * E + e)) : 0.f;
+                                acc[e] = fmaf(xs, wv, acc[e]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < EP; ++e) acc[e] = warp_sum(acc[e]);
+        if (lane == 0) {
+#pragma unroll
+            for (int e = 0; e < EP; ++e) part[warp][e] = acc[e];
+        }
+        __syncthreads();
+        if (warp == 0) {
+            float l[1] = {-FLT_MAX};
+            if (lane < E) {
+                float sum = 0.f;
+                for (int w2 = 0; w2 < kRouteWarps; ++w2) sum += part[w2][lane];
+                l[0] = sum;
+            }
+            bool valid[1] = {lane < E};
+            if (logits != nullptr && valid[0]) logits[t * E + lane] = l[0];
+            float psum[1] = {0.f};
+            finish_token<1>(l, valid, bias, t, K, lane, idx, w, psum, prob_part != nullptr);
+            if (prob_part != nullptr && lane < E) prob_part[t * E + lane] = psum[0];
+        }
+        __syncthreads();
+    }
+}
+
 template <int J>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 topk_from_logits_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int64_t T, int E,
@@ -259,12 +349,16 @@ topk_from_logits_kernel(const float* __restrict__ logits, const float* __restric
     if (want_prob) write_prob_partials<J>(psum, E, prob_part);
 }
 
-__global__ void prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float invT,
-                                     float* __restrict__ out) {
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+// P_i: warp w reduces experts w, w+32, ...: lane l adds router blocks l,
+// l+32, ... in order, then a fixed butterfly (reproducible).
+__global__ void __launch_bounds__(1024)
+prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float invT, float* __restrict__ out) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int e = warp; e < E; e += nw) {
         float s = 0.f;
-        for (int b = 0; b < nblocks; ++b) s += part[static_cast<int64_t>(b) * E + e];
-        out[e] = s * invT;
+        for (int b = lane; b < nblocks; b += 32) s += part[static_cast<int64_t>(b) * E + e];
+        s = warp_sum(s);
+        if (lane == 0) out[e] = s * invT;
     }
 }
 
@@ -288,6 +382,7 @@ __global__ void transpose_router_kernel(const __nv_bfloat16* __restrict__ Wr, in
 }  // namespace
 
 int route_blocks(int64_t T) {
+    if (T <= kSplitRouteMaxT) return static_cast<int>(T);  // the small-batch router: one CTA per token
     const int sms = num_sms() > 0 ? num_sms() : 148;
     int64_t need = (T + kRouteWarps - 1) / kRouteWarps;
     int64_t cap = static_cast<int64_t>(sms) * 4;
@@ -317,6 +412,17 @@ int launch_fused_ev(const bf16* x, const bf16* Wr, const float* bias, int64_t T,
 
 int launch_route_fused(const bf16* x, const bf16* Wr, const float* bias, int64_t T, int d, int E, int K,
                        float* logits, int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st) {
+    if (T <= kSplitRouteMaxT) {
+        // nblocks == T here (route_blocks): one CTA per token
+        const int th = kRouteWarps * 32;
+        if (E <= 8)
+            route_split_kernel<1><<<static_cast<int>(T), th, 0, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+        else if (E <= 16)
+            route_split_kernel<2><<<static_cast<int>(T), th, 0, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+        else
+            route_split_kernel<4><<<static_cast<int>(T), th, 0, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+        return cudaGetLastError() == cudaSuccess ? 0 : -3;
+    }
     if (E <= 8) return launch_fused_ev<1>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
     if (E <= 16) return launch_fused_ev<2>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
     return launch_fused_ev<4>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
@@ -339,8 +445,7 @@ int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, i
 }
 
 int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, float* prob_mean, cudaStream_t st) {
-    prob_finalize_kernel<<<(E + 255) / 256, 256, 0, st>>>(prob_part, nblocks, E, 1.0f / static_cast<float>(T),
-                                                         prob_mean);
+    prob_finalize_kernel<<<1, 1024, 0, st>>>(prob_part, nblocks, E, 1.0f / static_cast<float>(T), prob_mean);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
