@@ -142,14 +142,14 @@ def profile_traffic(workload: str):
     or None when it is missing or was taken on a different kernel source."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"grouped_gemm_{workload}.txt")
-    src = os.path.join(ROOT, "moe_layer_gemm_b200", "csrc", "gemm.cu")
     try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         vals = {}
         for line in open(path):
-            if ":" in line:
+            if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
+        src = os.path.join(ROOT, "moe_layer_gemm_b200", "csrc", vals.get("source", "gemm.cu"))
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         if vals.get("gemm_cu_sha256_16") != h:
             return None
         return int(float(vals["dram_bytes_per_step"]))

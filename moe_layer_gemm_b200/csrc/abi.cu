@@ -234,6 +234,10 @@ int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t*
     p1.split_stride = A * d->d_model;
     g.status = at<int>(ws, L.status);
     g.sched = at<int>(ws, L.sched_ffn);
+    // CTA-pair tiles are 256 token rows: worth it when groups are large
+    // (ragged 256-row tails of mid-sized groups cost more than they save)
+    const bool large_groups = d->T * d->K >= static_cast<int64_t>(d->E) * 1024;
+    if (large_groups && gemm_2sm_supported(g)) return map_launch(launch_grouped_gemm_2sm(g, st));
     return map_launch(launch_grouped_gemm(g, st));
 }
 

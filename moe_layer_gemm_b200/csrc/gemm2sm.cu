@@ -1,0 +1,534 @@
+// Grouped GEMM for large expert groups on CTA pairs (tcgen05 cta_group::2).
+//
+// Same computation as gemm.cu ("MoE computation notes", cf-1.com/news/5905749,
+// section 2.1: one matrix product per expert group), for launches where every
+// group is large enough for token-major tiles (prefill-sized batches).  Each
+// cluster of two CTAs owns one 256 x 256 output tile at a time:
+//   - CTA r loads token rows m0 + 128 r .. +127 (the M half of A) and weight
+//     rows n0 + 128 r .. +127 (the N half of B) into its own shared memory;
+//   - the leader (rank 0) issues one 256 x 256 x 16 tcgen05.mma per k-step,
+//     which reads A and B halves from both CTAs and accumulates rows
+//     128 r .. of D into CTA r's TMEM;
+//   - each CTA's epilogue drains its own TMEM rows.
+// Per CTA and k-block this moves 32 KB into shared memory for the FLOPs that
+// a single-CTA 128 x 256 tile needed 48 KB for, so the ring is deeper and the
+// weight tile is fetched by half as many CTAs.
+//
+// Pair protocol (barriers live in each CTA; "leader" means rank 0's copy):
+//   full[s]    leader only: the leader registers the pair's bytes, both CTAs'
+//              TMA loads complete on it
+//   empty[s]   both CTAs: the leader's MMA commit arrives on both
+//   tfull[b]   both CTAs: the leader's MMA commit arrives on both
+//   tempty[b]  leader: all 8 epilogue warps of the pair arrive
+//   ring       the leader claims tiles and writes them into both CTAs' rings;
+//              the pair's 10 consumers free a slot on the leader's rempty
+// Every wait is bounded.  No TMA multicast is used.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cstring>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr uint32_t kHalf = 128u * 128u;  // 128 rows x 64 bf16 = 16 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxGroups = 256;
+constexpr int kRing = 8;
+
+struct Phase2 {
+    int N, k_blocks, epi;
+    int64_t nb;  // 128-row weight blocks per group
+    void* out;
+    int64_t ldo;
+};
+
+struct Args2 {
+    const int32_t* group_off;
+    int G;
+    int nphase;
+    int dep;
+    Phase2 ph[2];
+    int stages;
+    int* status;
+    int* sched;
+};
+
+struct Maps2 {
+    CUtensorMap tok[2];  // token rows, box 128, 128-byte swizzle
+    CUtensorMap w[2];    // tiled weights as [rows, 64], box 128, no swizzle (tiles are pre-swizzled)
+};
+
+struct Tile2 {
+    int phase, g;
+    int64_t row0;  // first token row of the pair's 256-row tile
+    int rows;      // valid rows of the 256
+    int n0;        // first weight row (multiple of 256)
+};
+
+// ---- cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void remote_store(uint32_t cluster_addr, int v) {
+    asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// TMA tile load into this CTA's shared memory, completing on the leader's barrier.
+__device__ __forceinline__ void tma_load_pair(const CUtensorMap* map, void* smem_dst, uint32_t leader_bar, int32_t x,
+                                              int32_t y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(leader_bar),
+          "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once all
+// previously issued pair MMAs are complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3))
+                 : "memory");
+}
+
+__device__ __forceinline__ int tiles_of2(const Args2& a, int p, int64_t rows) {
+    if (rows <= 0) return 0;
+    return static_cast<int>(((rows + 255) / 256) * (a.ph[p].N / 256));
+}
+
+__device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* tstart, const int64_t* off) {
+    Tile2 t;
+    const int G = a.G;
+    int p = 0;
+    if (a.nphase > 1 && tile >= tstart[G]) p = 1;
+    const int* ts = tstart + p * (G + 1);
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ts[mid] <= tile) lo = mid; else hi = mid;
+    }
+    t.phase = p;
+    t.g = lo;
+    const int local = tile - ts[lo];
+    const int64_t base = off[lo];
+    const int64_t rows_g = off[lo + 1] - base;
+    const int mt = static_cast<int>((rows_g + 255) / 256);
+    const int n = local / mt, m = local - n * mt;  // m fastest: weight tile reused from L2
+    const int64_t r0 = static_cast<int64_t>(m) * 256;
+    t.row0 = base + r0;
+    t.rows = static_cast<int>(rows_g - r0 < 256 ? rows_g - r0 : 256);
+    t.n0 = n * 256;
+    return t;
+}
+
+__device__ __forceinline__ int ld_acquire2(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float silu2(float g) { return g / (1.0f + expf(-g)); }
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int S = a.stages;
+    uint8_t* sA = smem;                                  // [S][16 KB] token rows (this CTA's M half)
+    uint8_t* sB = smem + static_cast<size_t>(S) * kHalf;  // [S][16 KB] weight rows (this CTA's N half)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + static_cast<size_t>(S) * kHalf);
+    uint64_t* empty = full + S;
+    uint64_t* tfull = empty + S;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* rfull = tempty + 2;
+    uint64_t* rempty = rfull + kRing;
+    uint64_t* drain = rempty + kRing;
+    int* ring = reinterpret_cast<int*>(drain + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + kRing);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int64_t* off = reinterpret_cast<int64_t*>(tmem_slot + 2);
+    int* tstart = reinterpret_cast<int*>(off + a.G + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = a.G;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], 10);  // leader: MMA + 4 epilogue warps; peer: producer + 4 epilogue warps
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0)
+        for (int p = 0; p < a.nphase; ++p) {
+            tma_prefetch_desc(&maps.tok[p]);
+            tma_prefetch_desc(&maps.w[p]);
+        }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
+    __syncthreads();
+    if (warp == 0) {
+        const int span = (G + 31) / 32;
+        const int g0 = min(G, lane * span), g1 = min(G, g0 + span);
+        int carry = 0;
+        for (int p = 0; p < a.nphase; ++p) {
+            int sum = 0;
+            for (int g = g0; g < g1; ++g) sum += tiles_of2(a, p, off[g + 1] - off[g]);
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int run = carry + incl - sum;
+            int* ts = tstart + p * (G + 1);
+            for (int g = g0; g < g1; ++g) {
+                ts[g] = run;
+                run += tiles_of2(a, p, off[g + 1] - off[g]);
+            }
+            const int tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (lane == 0) ts[G] = carry + tot;
+            carry += tot;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tstart[(a.nphase - 1) * (G + 1) + G];
+    const uint32_t leader_rempty0 = mapa_shared(smem_u32(rempty), 0);
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(tempty), 0);
+    const uint32_t leader_full0 = mapa_shared(smem_u32(full), 0);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------- scheduler (leader) + producer (both)
+            const uint64_t pol_first = policy_evict_first();
+            const uint64_t pol_last = policy_evict_last();
+            uint32_t s = 0, ph = 0, r = 0, rph = 0;
+            bool ok = true;
+            bool sent_end = false;
+            int next = leader ? atomicAdd(&a.sched[0], 1) : 0;
+            const uint32_t peer_ring = mapa_shared(smem_u32(ring), 1);
+            const uint32_t peer_rfull = mapa_shared(smem_u32(rfull), 1);
+            while (ok) {
+                int tile;
+                if (leader) {
+                    tile = next < total ? next : -1;
+                    if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
+                    if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    ring[r] = tile;
+                    remote_store(peer_ring + 4u * r, tile);
+                    mbar_arrive(&rfull[r]);
+                    remote_arrive(peer_rfull + 8u * r);
+                } else {
+                    if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tile = ring[r];
+                    remote_arrive(leader_rempty0 + 8u * r);
+                }
+                if (++r == kRing) { r = 0; rph ^= 1u; }
+                if (tile < 0) {
+                    sent_end = true;
+                    break;
+                }
+                const Tile2 t = decode2(a, tile, tstart, off);
+                const Phase2& pa = a.ph[t.phase];
+                if (t.phase == 1 && a.dep) {
+                    const int need = 8 * (tstart[t.g + 1] - tstart[t.g]);
+                    uint32_t i = 0;
+                    while (ld_acquire2(&a.sched[1 + t.g]) < need) {
+                        if (++i > kWaitLimit || *abort_flag) {
+                            atomicCAS(a.status, 0, DEV_TIMEOUT_DEPENDENCY);
+                            *abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                        if (i > 64) __nanosleep(128);
+                    }
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    if (!ok) break;
+                }
+                const int32_t tok_row = static_cast<int32_t>(t.row0 + 128 * rank);
+                const int64_t wblk = static_cast<int64_t>(t.g) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
+                for (int kb = 0; kb < pa.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(&full[s], 4u * kHalf);  // both CTAs' A and B halves
+                    const uint32_t bar = leader_full0 + 8u * s;
+                    tma_load_pair(&maps.tok[t.phase], sA + static_cast<size_t>(s) * kHalf, bar, kb * kBK, tok_row,
+                                  pol_last);
+                    tma_load_pair(&maps.w[t.phase], sB + static_cast<size_t>(s) * kHalf, bar, 0,
+                                  static_cast<int32_t>((wblk * pa.k_blocks + kb) * 128), pol_first);
+                    if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (leader && !sent_end) {
+                // a failed wait: hand every consumer the end marker (bounded)
+                for (uint32_t i = 0; i < kWaitLimit; ++i)
+                    if (mbar_try_wait(&rempty[r], rph ^ 1u)) break;
+                ring[r] = -1;
+                remote_store(peer_ring + 4u * r, -1);
+                mbar_arrive(&rfull[r]);
+                remote_arrive(peer_rfull + 8u * r);
+            }
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            // ------------------------------------------------ pair MMA issuer (leader only)
+            uint32_t s = 0, ph = 0, r = 0, rph = 0;
+            int it = 0;
+            bool ok = true;
+            const uint32_t idesc = umma_idesc_bf16(256, 256);
+            while (ok) {
+                if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) break;
+                const int tile = ring[r];
+                mbar_arrive(&rempty[r]);
+                if (++r == kRing) { r = 0; rph ^= 1u; }
+                if (tile < 0) break;
+                const Tile2 t = decode2(a, tile, tstart, off);
+                const int buf = it & 1;
+                const uint32_t use = static_cast<uint32_t>(it >> 1);
+                ++it;
+                if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
+                const int kbs = a.ph[t.phase].k_blocks;
+                for (int kb = 0; kb < kbs; ++kb) {
+                    if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + static_cast<size_t>(s) * kHalf);
+                    const uint32_t b_base = smem_u32(sB + static_cast<size_t>(s) * kHalf);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_pair(d_tmem, umma_desc_sw128(a_base + kk * 32), umma_desc_sw128(b_base + kk * 32), idesc,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair(&empty[s]);
+                    if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
+                }
+                if (ok) umma_commit_pair(&tfull[buf]);
+            }
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         ::"r"(smem_u32(drain)) : "memory");
+            for (uint32_t i = 0; i < kWaitLimit; ++i)
+                if (mbar_try_wait(drain, 0)) break;
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        uint32_t r = 0, rph = 0;
+        int it = 0;
+        for (;;) {
+            if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            const int tile = ring[r];
+            __syncwarp();
+            if (lane == 0) remote_arrive(leader_rempty0 + 8u * r);
+            if (++r == kRing) { r = 0; rph ^= 1u; }
+            if (tile < 0) break;
+            const Tile2 t = decode2(a, tile, tstart, off);
+            const Phase2& pa = a.ph[t.phase];
+            const int buf = it & 1;
+            const uint32_t use = static_cast<uint32_t>(it >> 1);
+            ++it;
+            if (!mbar_wait(&tfull[buf], use & 1u, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf) * 256u + (static_cast<uint32_t>(q * 32) << 16);
+            const int rr = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the pair's 256
+            const bool valid = rr < t.rows;
+            const int64_t grow = t.row0 + rr;
+            float v[32];
+            for (int c = 0; c < 8; ++c) {
+                tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                if (!valid) continue;
+                if (pa.epi == EPI_SWIGLU_BF16) {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pk[i] = pack2(silu2(v[2 * i]) * v[16 + 2 * i], silu2(v[2 * i + 1]) * v[16 + 2 * i + 1]);
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(pa.out) + grow * pa.ldo +
+                                                          (t.n0 / 2 + c * 16));
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pa.out) + grow * pa.ldo + t.n0 + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                remote_arrive(leader_tempty0 + 8u * buf);
+                if (t.phase == 0 && a.dep) {
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    __threadfence();
+                    atomicAdd(&a.sched[1 + t.g], 1);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer's TMEM and shared memory stay alive until the leader is done
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder2() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, bool swizzle) {
+    auto enc = encoder2();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64u, 128u};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool gemm_2sm_supported(const GemmLaunch& L) {
+    if (L.nphase < 1 || L.nphase > 2 || L.G < 1 || L.G > kMaxGroups || L.group_off == nullptr) return false;
+    if (L.swap_max_rows > 0) return false;
+    for (int p = 0; p < L.nphase; ++p)
+        if (L.ph[p].N % 256 != 0 || L.ph[p].Kdim % 8 != 0 || L.ph[p].Kdim < 16 || L.ph[p].ksplit > 1 ||
+            L.ph[p].N_store != L.ph[p].N || (L.ph[p].ldo & 3) != 0)
+            return false;
+    return true;
+}
+
+int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
+    if (!gemm_2sm_supported(L) || !L.sched) return -2;
+    Args2 a{};
+    a.group_off = L.group_off;
+    a.G = L.G;
+    a.nphase = L.nphase;
+    a.dep = L.nphase == 2 ? 1 : 0;
+    a.status = L.status;
+    a.sched = L.sched;
+    Maps2 maps;
+    std::memset(&maps, 0, sizeof(maps));
+    for (int p = 0; p < L.nphase; ++p) {
+        const GemmPhase& g = L.ph[p];
+        a.ph[p].N = g.N;
+        a.ph[p].k_blocks = (g.Kdim + kBK - 1) / kBK;
+        a.ph[p].epi = g.epi;
+        a.ph[p].nb = g.N / 128;
+        a.ph[p].out = g.out;
+        a.ph[p].ldo = g.ldo;
+        if (!map2(&maps.tok[p], g.tok, static_cast<uint64_t>(g.tok_rows), g.Kdim, true)) return -3;
+        const uint64_t wrows = static_cast<uint64_t>(L.G) * a.ph[p].nb * a.ph[p].k_blocks * 128;
+        if (!map2(&maps.w[p], g.w, wrows, 64, false)) return -3;
+    }
+    const size_t fixed = 1024 + static_cast<size_t>(2 * 16 + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
+                         static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + 64;
+    int stages = static_cast<int>((227 * 1024 - fixed) / (2 * kHalf));
+    if (stages > 16) stages = 16;
+    if (stages < 2) return -2;
+    a.stages = stages;
+    const size_t smem = fixed + static_cast<size_t>(stages) * 2 * kHalf;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess)
+            return -3;
+        attr = true;
+    }
+    const int sms = num_sms();
+    if (sms <= 1) return -3;
+    int clusters = sms / 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = 2;
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_2sm_kernel, maps, a) != cudaSuccess) return -3;
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+}  // namespace moe

@@ -48,6 +48,10 @@ struct GemmLaunch {
 };
 
 size_t gemm_sched_bytes(int G);
+// CTA-pair (cta_group::2) kernel for launches whose groups all take
+// token-major tiles and whose widths are multiples of 256.
+bool gemm_2sm_supported(const GemmLaunch& L);
+int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st);
 int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st);
 int num_sms();
 

@@ -65,6 +65,8 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (2000, 256, 320, 4, 2, 0.0),      # large groups: token-major tiles, ragged m tail
     (1500, 384, 704, 12, 3, 1.5),     # skewed: empty groups possible
     (130, 128, 128, 1, 1, 0.0),       # single expert = dense FFN
+    (2100, 512, 256, 4, 2, 0.0),      # mean group >= 1024 rows, widths x256: CTA-pair tiles, ragged tail
+    (6200, 256, 384, 6, 1, 1.5),      # CTA-pair tiles with skewed groups (the smallest may be tiny)
 ])
 def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
     r = _run(T, d, f, E, K, skew)
