@@ -234,10 +234,13 @@ int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t*
     p1.split_stride = A * d->d_model;
     g.status = at<int>(ws, L.status);
     g.sched = at<int>(ws, L.sched_ffn);
-    // CTA-pair tiles are 256 token rows: worth it when groups are large
-    // (ragged 256-row tails of mid-sized groups cost more than they save)
+    // CTA-pair tiles: token-major pairs are 256 token rows, worth it when
+    // groups are large (ragged 256-row tails of mid-sized groups cost more
+    // than they save); weight-major pairs halve the token traffic of
+    // decode-sized groups.
     const bool large_groups = d->T * d->K >= static_cast<int64_t>(d->E) * 1024;
-    if (large_groups && gemm_2sm_supported(g)) return map_launch(launch_grouped_gemm_2sm(g, st));
+    const bool pair = large_groups || L.swap;
+    if (pair && gemm_2sm_supported(g)) return map_launch(launch_grouped_gemm_2sm(g, st));
     return map_launch(launch_grouped_gemm(g, st));
 }
 

@@ -54,7 +54,7 @@ struct PhaseArgs {
     int N;        // weight rows per group
     int N_store;  // output columns written (router: E of E_pad)
     int k_blocks;
-    int ksplit;   // weight-major tiles only
+    int ksplit;   // reduction split (partial slices), every tile of the phase
     int kb_per_split;
     int epi;
     int BN;       // token-major: weight rows per tile
@@ -101,7 +101,7 @@ __device__ __forceinline__ bool group_swaps(const DevArgs& a, int p, int64_t row
 __device__ __forceinline__ int tiles_of(const DevArgs& a, int p, int64_t rows) {
     if (rows <= 0) return 0;
     const PhaseArgs& ph = a.ph[p];
-    if (!group_swaps(a, p, rows)) return static_cast<int>(((rows + 127) / 128) * (ph.N / ph.BN));
+    if (!group_swaps(a, p, rows)) return static_cast<int>(((rows + 127) / 128) * (ph.N / ph.BN) * ph.ksplit);
     return static_cast<int>(((rows + a.BNs - 1) / a.BNs) * (ph.N / 128) * ph.ksplit);
 }
 
@@ -125,15 +125,19 @@ __device__ __forceinline__ Tile decode_tile(const DevArgs& a, int tile, const in
     const int64_t rows_g = off[lo + 1] - base;
     t.swap = group_swaps(a, p, rows_g) ? 1 : 0;
     if (!t.swap) {
+        // a reduction split applies to every tile of the phase, so each
+        // partial slice is written for every row
+        const int s = local % ph.ksplit;
+        const int rest = local / ph.ksplit;
         const int mt = static_cast<int>((rows_g + 127) / 128);
-        const int n = local / mt, m = local - n * mt;  // m fastest: weight tile reused from L2
+        const int n = rest / mt, m = rest - n * mt;  // m fastest: weight tile reused from L2
         const int64_t r0 = static_cast<int64_t>(m) * 128;
         t.row0 = base + r0;
         t.rows = static_cast<int>(rows_g - r0 < 128 ? rows_g - r0 : 128);
         t.n0 = n * ph.BN;
-        t.kb0 = 0;
-        t.kb1 = ph.k_blocks;
-        t.split = 0;
+        t.kb0 = s * ph.kb_per_split;
+        t.kb1 = min(ph.k_blocks, t.kb0 + ph.kb_per_split);
+        t.split = s;
     } else {
         const int nch = static_cast<int>((rows_g + a.BNs - 1) / a.BNs);
         const int s = local % ph.ksplit;
@@ -151,7 +155,11 @@ __device__ __forceinline__ Tile decode_tile(const DevArgs& a, int tile, const in
     return t;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast exp and divide intrinsics: the
+// result is rounded to bf16 (8-bit mantissa) right after, far coarser than
+// their few-ulp error.  For g < -87, e^-g overflows to inf and the quotient
+// is 0, the limit of silu.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
@@ -438,7 +446,8 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                         dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     } else {
                         const int col0 = t.n0 + c * 32;
-                        float* Y = static_cast<float*>(pa.out) + grow * pa.ldo + col0;
+                        float* Y = static_cast<float*>(pa.out) + static_cast<int64_t>(t.split) * pa.split_stride +
+                                   grow * pa.ldo + col0;
                         if (col0 + 32 <= pa.N_store && (pa.ldo & 3) == 0) {  // float4 rows need 16 B alignment
                             float4* dst = reinterpret_cast<float4*>(Y);
 #pragma unroll
@@ -589,7 +598,7 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         for (int c : {256, 128, 64, 32})
             if (c <= bn_cap && g.N % c == 0) { bn = c; break; }
         if (bn == 0) return -2;
-        if (g.epi == EPI_SWIGLU_BF16 && g.N % 32 != 0) return -2;
+        if (g.epi == EPI_SWIGLU_BF16 && (g.N % 32 != 0 || g.ksplit > 1)) return -2;
         ph.BN = bn;
         int ks = g.ksplit < 1 ? 1 : g.ksplit;
         if (ks > ph.k_blocks) ks = ph.k_blocks;
@@ -637,7 +646,7 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
     for (int p = 0; p < L.nphase; ++p) {
         const GemmPhase& g = L.ph[p];
         const int64_t rows_total = L.group_off ? g.tok_rows : L.dense_rows;
-        const int64_t tm = ((rows_total + 127) / 128 + L.G) * (g.N / a.ph[p].BN);
+        const int64_t tm = ((rows_total + 127) / 128 + L.G) * (g.N / a.ph[p].BN) * a.ph[p].ksplit;
         const int64_t sw =
             (g.N % 128 == 0) ? ((rows_total + a.BNs - 1) / a.BNs + L.G) * (g.N / 128) * a.ph[p].ksplit : 0;
         bound += tm > sw ? tm : sw;

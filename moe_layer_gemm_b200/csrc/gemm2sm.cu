@@ -14,6 +14,14 @@
 // a single-CTA 128 x 256 tile needed 48 KB for, so the ring is deeper and the
 // weight tile is fetched by half as many CTAs.
 //
+// Small groups use weight-major pair tiles instead: the MMA's M side is 256
+// weight rows (CTA r loads the 128-row weight tile n0 + 128 r), its N side
+// the group's tokens, of which each CTA loads half.  Against single-CTA
+// weight-major tiles this halves the token traffic and the MMA instructions
+// per SM, and when no group can take token-major tiles the token slot is
+// only 8 KB, so the weight ring is deeper.  The down projection's reduction
+// can be split as in gemm.cu.
+//
 // Pair protocol (barriers live in each CTA; "leader" means rank 0's copy):
 //   full[s]    leader only: the leader registers the pair's bytes, both CTAs'
 //              TMA loads complete on it
@@ -45,8 +53,10 @@ constexpr int kRing = 8;
 struct Phase2 {
     int N, k_blocks, epi;
     int64_t nb;  // 128-row weight blocks per group
+    int ksplit, kb_per_split;  // weight-major tiles only
     void* out;
     int64_t ldo;
+    int64_t split_stride;
 };
 
 struct Args2 {
@@ -54,22 +64,27 @@ struct Args2 {
     int G;
     int nphase;
     int dep;
+    int swap_max_rows;  // groups with at most this many rows take weight-major pair tiles
+    int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 128)
     Phase2 ph[2];
     int stages;
+    uint32_t b_slot;    // bytes of the second operand slot per stage
     int* status;
     int* sched;
 };
 
 struct Maps2 {
     CUtensorMap tok[2];  // token rows, box 128, 128-byte swizzle
+    CUtensorMap tok16[2];  // token rows, box 16, 128-byte swizzle (weight-major halves)
     CUtensorMap w[2];    // tiled weights as [rows, 64], box 128, no swizzle (tiles are pre-swizzled)
 };
 
 struct Tile2 {
-    int phase, g;
-    int64_t row0;  // first token row of the pair's 256-row tile
-    int rows;      // valid rows of the 256
+    int phase, g, swap;
+    int64_t row0;  // first token row of the pair's tile
+    int rows;      // valid token rows (<= 256 token-major, <= BNs weight-major)
     int n0;        // first weight row (multiple of 256)
+    int kb0, kb1, split;
 };
 
 // ---- cluster helpers
@@ -117,9 +132,12 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
                  : "memory");
 }
 
+__device__ __forceinline__ bool swaps2(const Args2& a, int64_t rows) { return rows <= a.swap_max_rows; }
+
 __device__ __forceinline__ int tiles_of2(const Args2& a, int p, int64_t rows) {
     if (rows <= 0) return 0;
-    return static_cast<int>(((rows + 255) / 256) * (a.ph[p].N / 256));
+    const int64_t chunks = swaps2(a, rows) ? (rows + a.BNs - 1) / a.BNs : (rows + 255) / 256;
+    return static_cast<int>(chunks * (a.ph[p].N / 256) * a.ph[p].ksplit);
 }
 
 __device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* tstart, const int64_t* off) {
@@ -133,17 +151,27 @@ __device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* ts
         const int mid = (lo + hi) >> 1;
         if (ts[mid] <= tile) lo = mid; else hi = mid;
     }
+    const Phase2& ph = a.ph[p];
     t.phase = p;
     t.g = lo;
     const int local = tile - ts[lo];
     const int64_t base = off[lo];
     const int64_t rows_g = off[lo + 1] - base;
-    const int mt = static_cast<int>((rows_g + 255) / 256);
-    const int n = local / mt, m = local - n * mt;  // m fastest: weight tile reused from L2
-    const int64_t r0 = static_cast<int64_t>(m) * 256;
+    t.swap = swaps2(a, rows_g) ? 1 : 0;
+    // token chunk fastest (the weight tile is reused from L2), then the
+    // weight tile; the reduction split is outermost within a chunk's tiles
+    const int chunk = t.swap ? a.BNs : 256;
+    const int nch = static_cast<int>((rows_g + chunk - 1) / chunk);
+    const int sp = local % ph.ksplit;
+    const int rest = local / ph.ksplit;
+    const int c = rest % nch;
+    const int64_t r0 = static_cast<int64_t>(c) * chunk;
     t.row0 = base + r0;
-    t.rows = static_cast<int>(rows_g - r0 < 256 ? rows_g - r0 : 256);
-    t.n0 = n * 256;
+    t.rows = static_cast<int>(rows_g - r0 < chunk ? rows_g - r0 : chunk);
+    t.n0 = (rest / nch) * 256;
+    t.kb0 = sp * ph.kb_per_split;
+    t.kb1 = min(ph.k_blocks, t.kb0 + ph.kb_per_split);
+    t.split = sp;
     return t;
 }
 
@@ -153,7 +181,11 @@ __device__ __forceinline__ int ld_acquire2(const int* p) {
     return v;
 }
 
-__device__ __forceinline__ float silu2(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast exp and divide intrinsics: the
+// result is rounded to bf16 (8-bit mantissa) right after, far coarser than
+// their few-ulp error.  For g < -87, e^-g overflows to inf and the quotient
+// is 0, the limit of silu.
+__device__ __forceinline__ float silu2(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
@@ -166,9 +198,9 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int S = a.stages;
-    uint8_t* sA = smem;                                  // [S][16 KB] token rows (this CTA's M half)
-    uint8_t* sB = smem + static_cast<size_t>(S) * kHalf;  // [S][16 KB] weight rows (this CTA's N half)
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + static_cast<size_t>(S) * kHalf);
+    uint8_t* sA = smem;                                   // [S][16 KB] M-side rows of this CTA (tokens or weights)
+    uint8_t* sB = smem + static_cast<size_t>(S) * kHalf;  // [S][b_slot] N-side rows of this CTA (weights or tokens)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + static_cast<size_t>(S) * a.b_slot);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
@@ -207,6 +239,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     if (warp == 0 && lane == 0)
         for (int p = 0; p < a.nphase; ++p) {
             tma_prefetch_desc(&maps.tok[p]);
+            tma_prefetch_desc(&maps.tok16[p]);
             tma_prefetch_desc(&maps.w[p]);
         }
     if (warp == 1) {
@@ -304,19 +337,31 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                     if (!ok) break;
                 }
-                const int32_t tok_row = static_cast<int32_t>(t.row0 + 128 * rank);
                 const int64_t wblk = static_cast<int64_t>(t.g) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
-                for (int kb = 0; kb < pa.k_blocks; ++kb) {
+                // weight-major: this CTA's half of the tile's token columns, in 16-row boxes
+                const int nb16 = t.swap ? (t.rows + 31) / 32 : 0;
+                const uint32_t pair_bytes = t.swap ? 2u * (kHalf + static_cast<uint32_t>(nb16) * 2048u) : 4u * kHalf;
+                for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (leader) mbar_arrive_expect_tx(&full[s], 4u * kHalf);  // both CTAs' A and B halves
+                    if (leader) mbar_arrive_expect_tx(&full[s], pair_bytes);
                     const uint32_t bar = leader_full0 + 8u * s;
-                    tma_load_pair(&maps.tok[t.phase], sA + static_cast<size_t>(s) * kHalf, bar, kb * kBK, tok_row,
-                                  pol_last);
-                    tma_load_pair(&maps.w[t.phase], sB + static_cast<size_t>(s) * kHalf, bar, 0,
-                                  static_cast<int32_t>((wblk * pa.k_blocks + kb) * 128), pol_first);
+                    uint8_t* dA = sA + static_cast<size_t>(s) * kHalf;
+                    uint8_t* dB = sB + static_cast<size_t>(s) * a.b_slot;
+                    const int32_t wrow = static_cast<int32_t>((wblk * pa.k_blocks + kb) * 128);
+                    if (!t.swap) {
+                        tma_load_pair(&maps.tok[t.phase], dA, bar, kb * kBK,
+                                      static_cast<int32_t>(t.row0 + 128 * rank), pol_last);
+                        tma_load_pair(&maps.w[t.phase], dB, bar, 0, wrow, pol_first);
+                    } else {
+                        tma_load_pair(&maps.w[t.phase], dA, bar, 0, wrow, pol_first);
+                        const int64_t trow = t.row0 + static_cast<int64_t>(rank) * 16 * nb16;
+                        for (int j = 0; j < nb16; ++j)
+                            tma_load_pair(&maps.tok16[t.phase], dB + j * 2048, bar, kb * kBK,
+                                          static_cast<int32_t>(trow + 16 * j), pol_last);
+                    }
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
             }
@@ -336,7 +381,6 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             uint32_t s = 0, ph = 0, r = 0, rph = 0;
             int it = 0;
             bool ok = true;
-            const uint32_t idesc = umma_idesc_bf16(256, 256);
             while (ok) {
                 if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) break;
                 const int tile = ring[r];
@@ -350,19 +394,20 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
-                const int kbs = a.ph[t.phase].k_blocks;
-                for (int kb = 0; kb < kbs; ++kb) {
+                const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 31) / 32) * 32u : 256u;
+                const uint32_t idesc = umma_idesc_bf16(256, n_mma);
+                for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(sA + static_cast<size_t>(s) * kHalf);
-                    const uint32_t b_base = smem_u32(sB + static_cast<size_t>(s) * kHalf);
+                    const uint32_t b_base = smem_u32(sB + static_cast<size_t>(s) * a.b_slot);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
                         umma_pair(d_tmem, umma_desc_sw128(a_base + kk * 32), umma_desc_sw128(b_base + kk * 32), idesc,
-                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                                  (kb > t.kb0 || kk > 0) ? 1u : 0u);
                     umma_commit_pair(&empty[s]);
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
@@ -393,26 +438,56 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             if (!mbar_wait(&tfull[buf], use & 1u, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf) * 256u + (static_cast<uint32_t>(q * 32) << 16);
-            const int rr = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the pair's 256
-            const bool valid = rr < t.rows;
-            const int64_t grow = t.row0 + rr;
             float v[32];
-            for (int c = 0; c < 8; ++c) {
-                tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
-                if (!valid) continue;
-                if (pa.epi == EPI_SWIGLU_BF16) {
-                    uint32_t pk[8];
+            if (!t.swap) {
+                const int rr = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the pair's 256
+                const bool valid = rr < t.rows;
+                const int64_t grow = t.row0 + rr;
+                for (int c = 0; c < 8; ++c) {
+                    tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                    if (!valid) continue;
+                    if (pa.epi == EPI_SWIGLU_BF16) {
+                        uint32_t pk[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = pack2(silu2(v[2 * i]) * v[16 + 2 * i], silu2(v[2 * i + 1]) * v[16 + 2 * i + 1]);
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(pa.out) + grow * pa.ldo +
-                                                          (t.n0 / 2 + c * 16));
-                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pa.out) + grow * pa.ldo + t.n0 + c * 32);
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = pack2(silu2(v[2 * i]) * v[16 + 2 * i], silu2(v[2 * i + 1]) * v[16 + 2 * i + 1]);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(pa.out) + grow * pa.ldo +
+                                                              (t.n0 / 2 + c * 16));
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pa.out) +
+                                                                static_cast<int64_t>(t.split) * pa.split_stride +
+                                                                grow * pa.ldo + t.n0 + c * 32);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+            } else {
+                // lanes are this CTA's 128 weight rows n0 + 128 rank + .., columns the tile's tokens
+                const int nwr = t.n0 + 128 * static_cast<int>(rank);
+                const int nbk = (t.rows + 31) / 32;
+                for (int c = 0; c < nbk; ++c) {
+                    tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                    if (pa.epi == EPI_SWIGLU_BF16) {
+                        const int f = nwr / 2 + q * 16 + (lane & 15);
+                        bf16* H = static_cast<bf16*>(pa.out);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float u = __shfl_xor_sync(0xffffffffu, v[j], 16);
+                            const int tok = c * 32 + j;
+                            if (lane < 16 && tok < t.rows)
+                                H[(t.row0 + tok) * pa.ldo + f] = __float2bfloat16_rn(silu2(v[j]) * u);
+                        }
+                    } else {
+                        float* Y = static_cast<float*>(pa.out) + static_cast<int64_t>(t.split) * pa.split_stride;
+                        const int col = nwr + q * 32 + lane;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int tok = c * 32 + j;
+                            if (tok < t.rows) Y[(t.row0 + tok) * pa.ldo + col] = v[j];
+                        }
+                    }
                 }
             }
             tc_fence_before();
@@ -451,12 +526,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder2() {
     return fn;
 }
 
-bool map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, bool swizzle) {
+bool map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, bool swizzle) {
     auto enc = encoder2();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64u, 128u};
+    cuuint32_t box[2] = {64u, box_rows};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -467,11 +542,11 @@ bool map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, bool s
 
 bool gemm_2sm_supported(const GemmLaunch& L) {
     if (L.nphase < 1 || L.nphase > 2 || L.G < 1 || L.G > kMaxGroups || L.group_off == nullptr) return false;
-    if (L.swap_max_rows > 0) return false;
-    for (int p = 0; p < L.nphase; ++p)
-        if (L.ph[p].N % 256 != 0 || L.ph[p].Kdim % 8 != 0 || L.ph[p].Kdim < 16 || L.ph[p].ksplit > 1 ||
-            L.ph[p].N_store != L.ph[p].N || (L.ph[p].ldo & 3) != 0)
-            return false;
+    for (int p = 0; p < L.nphase; ++p) {
+        const GemmPhase& g = L.ph[p];
+        if (g.N % 256 != 0 || g.Kdim % 8 != 0 || g.Kdim < 16 || g.N_store != g.N || (g.ldo & 3) != 0) return false;
+        if (g.ksplit > 1 && g.epi != EPI_F32) return false;  // SwiGLU needs the whole reduction
+    }
     return true;
 }
 
@@ -484,27 +559,46 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     a.dep = L.nphase == 2 ? 1 : 0;
     a.status = L.status;
     a.sched = L.sched;
+    const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
+    a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
+    {
+        const int64_t lim = mx < a.swap_max_rows ? mx : a.swap_max_rows;
+        a.BNs = static_cast<int>(lim >= 128 ? 128 : ((lim + 31) / 32) * 32);
+        if (a.BNs < 32) a.BNs = 32;
+    }
+    // The N-side slot holds a 128-row weight half (token-major tiles) or
+    // BNs / 2 token rows (weight-major tiles).
+    const bool token_major_possible = mx > a.swap_max_rows;
+    a.b_slot = token_major_possible ? kHalf : static_cast<uint32_t>(a.BNs) * 64u;
     Maps2 maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int p = 0; p < L.nphase; ++p) {
         const GemmPhase& g = L.ph[p];
-        a.ph[p].N = g.N;
-        a.ph[p].k_blocks = (g.Kdim + kBK - 1) / kBK;
-        a.ph[p].epi = g.epi;
-        a.ph[p].nb = g.N / 128;
-        a.ph[p].out = g.out;
-        a.ph[p].ldo = g.ldo;
-        if (!map2(&maps.tok[p], g.tok, static_cast<uint64_t>(g.tok_rows), g.Kdim, true)) return -3;
-        const uint64_t wrows = static_cast<uint64_t>(L.G) * a.ph[p].nb * a.ph[p].k_blocks * 128;
-        if (!map2(&maps.w[p], g.w, wrows, 64, false)) return -3;
+        Phase2& ph = a.ph[p];
+        ph.N = g.N;
+        ph.k_blocks = (g.Kdim + kBK - 1) / kBK;
+        ph.epi = g.epi;
+        ph.nb = g.N / 128;
+        ph.out = g.out;
+        ph.ldo = g.ldo;
+        ph.split_stride = g.split_stride;
+        int ks = g.ksplit < 1 ? 1 : g.ksplit;
+        if (ks > ph.k_blocks) ks = ph.k_blocks;
+        ph.kb_per_split = (ph.k_blocks + ks - 1) / ks;
+        ph.ksplit = (ph.k_blocks + ph.kb_per_split - 1) / ph.kb_per_split;
+        const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
+        if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
+        if (!map2(&maps.tok16[p], g.tok, trows, g.Kdim, 16u, true)) return -3;
+        const uint64_t wrows = static_cast<uint64_t>(L.G) * ph.nb * ph.k_blocks * 128;
+        if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
     }
     const size_t fixed = 1024 + static_cast<size_t>(2 * 16 + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
                          static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + 64;
-    int stages = static_cast<int>((227 * 1024 - fixed) / (2 * kHalf));
+    int stages = static_cast<int>((227 * 1024 - fixed) / (kHalf + a.b_slot));
     if (stages > 16) stages = 16;
     if (stages < 2) return -2;
     a.stages = stages;
-    const size_t smem = fixed + static_cast<size_t>(stages) * 2 * kHalf;
+    const size_t smem = fixed + static_cast<size_t>(stages) * (kHalf + a.b_slot);
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=

@@ -24,7 +24,7 @@ struct GemmPhase {
     int N;                // weight rows per group
     int N_store;          // output columns actually written (<= N)
     int Kdim;
-    int ksplit;           // reduction split of weight-major tiles (partial slices)
+    int ksplit;           // reduction split into partial slices (every tile of the phase)
     int epi;
     void* out;
     int64_t ldo;          // output row stride (elements)
@@ -48,8 +48,8 @@ struct GemmLaunch {
 };
 
 size_t gemm_sched_bytes(int G);
-// CTA-pair (cta_group::2) kernel for launches whose groups all take
-// token-major tiles and whose widths are multiples of 256.
+// CTA-pair (cta_group::2) kernel: 256-wide tiles, so both phases' widths
+// must be multiples of 256.
 bool gemm_2sm_supported(const GemmLaunch& L);
 int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st);
 int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st);

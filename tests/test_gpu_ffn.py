@@ -67,6 +67,10 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (130, 128, 128, 1, 1, 0.0),       # single expert = dense FFN
     (2100, 512, 256, 4, 2, 0.0),      # mean group >= 1024 rows, widths x256: CTA-pair tiles, ragged tail
     (6200, 256, 384, 6, 1, 1.5),      # CTA-pair tiles with skewed groups (the smallest may be tiny)
+    (256, 256, 1024, 8, 2, 1.5),      # decode-like CTA pairs, 4-way split, one group > 128 rows (token-major)
+    (256, 384, 768, 8, 2, 1.5),       # single-CTA, 2-way split, one group > 128 rows (token-major)
+    (40, 256, 512, 8, 2, 0.0),        # CTA pairs, groups under 16 rows, 2-way split
+    (600, 256, 256, 16, 4, 1.2),      # CTA pairs, weight- and token-major groups in one launch
 ])
 def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
     r = _run(T, d, f, E, K, skew)
