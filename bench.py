@@ -137,22 +137,24 @@ def layer_algorithmic(wl, counts: np.ndarray, kept: np.ndarray):
                 gemm_bytes=gemm_bytes, gemm_flops=gemm_flops)
 
 
-def profile_traffic(workload: str):
-    """DRAM bytes per step of the expert GEMMs from the committed ncu summary,
-    or None when it is missing or was taken on a different kernel source."""
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of the expert-GEMM kernel from the committed ncu
+    summary profiles/<kernel>_<workload>.txt, or None when it is missing or
+    was taken on a different kernel source."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"grouped_gemm_{workload}.txt")
+    stem = kernel[:-len("_kernel")] if kernel.endswith("_kernel") else kernel
+    path = os.path.join(ROOT, "profiles", f"{stem}_{workload}.txt")
     try:
         vals = {}
         for line in open(path):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-        src = os.path.join(ROOT, "moe_layer_gemm_b200", "csrc", vals.get("source", "gemm.cu"))
+        src = os.path.join(ROOT, "moe_layer_gemm_b200", "csrc", vals["source"])
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if vals.get("gemm_cu_sha256_16") != h:
+        if vals.get("source_sha256_16") != h:
             return None
-        return int(float(vals["dram_bytes_per_step"]))
+        return int(float(vals["dram_bytes_per_launch"]))
     except Exception:
         return None
 
@@ -356,8 +358,9 @@ def run_ours(args):
         achieved = alg["gemm_flops"] / (gemm_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
                 "frac": achieved / tensor_peak}
-    traffic = profile_traffic(wl.name)
-    roof.update({"traffic": traffic, "kernel": "grouped_gemm_kernel (gate/up and down in one launch)",
+    kernel = abi.moe_ffn_kernel(dims)
+    traffic = profile_traffic(kernel, wl.name)
+    roof.update({"traffic": traffic, "kernel": f"{kernel} (gate/up and down in one launch)",
                  "algorithmic_per_step": alg["gemm_bytes"] if roof["bound"] == "hbm" else alg["gemm_flops"],
                  "ms_per_step": gemm_ms, "peak_source": f"{peak_src}" + (" sustained" if sustained and roof["bound"] == "tensor" else "")})
 

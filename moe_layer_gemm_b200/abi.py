@@ -31,7 +31,7 @@ EXPORTED = [
     "moe_status_str", "moe_version", "moe_capacity", "moe_workspace_size", "moe_reset_device_status",
     "moe_get_device_status", "moe_pack_weights", "moe_route", "moe_route_from_logits", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
-    "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc",
+    "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc", "moe_ffn_kernel",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -85,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_layer_launch_count": (I, [dims_p, I, I]),
         "moe_packed_weight_bytes": (I, [dims_p, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
         "moe_permute_noalloc": (I, [dims_p, P, P, P, P, P, P, P, P, P, P]),
+        "moe_ffn_kernel": (I, [dims_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -271,6 +272,17 @@ def moe_layer_launch_count(dims, stats: bool, bias_update: bool) -> int:
     if n < 0:
         raise MoEError("moe_layer_launch_count", n, "invalid dims")
     return n
+
+
+FFN_KERNELS = ("grouped_gemm_kernel", "grouped_gemm_2sm_kernel")
+
+
+def moe_ffn_kernel(dims) -> str:
+    """Name of the grouped-GEMM kernel the expert FFN launches for these dims."""
+    k = load().moe_ffn_kernel(ctypes.byref(_dims(dims)))
+    if k < 0:
+        raise MoEError("moe_ffn_kernel", k, "invalid dims")
+    return FFN_KERNELS[k]
 
 
 # ---------------------------------------------------------------- helpers

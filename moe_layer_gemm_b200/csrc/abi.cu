@@ -191,11 +191,9 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
     return MOE_OK;
 }
 
-// Both expert GEMMs in one launch.  The scheduler words at L.sched_ffn must
-// be zero when it starts (the dispatch kernels clear them; the standalone
-// entry point clears them with a memset).
-int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
-           const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st) {
+// The launch description of both expert GEMMs (gate/up + SwiGLU, then down).
+GemmLaunch ffn_launch(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
+                      const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws) {
     const int64_t A = d->T * d->K;
     int64_t maxrows = d->T;
     const int64_t C = capacity_of(d);
@@ -232,15 +230,26 @@ int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t*
     p1.out = yout;
     p1.ldo = d->d_model;
     p1.split_stride = A * d->d_model;
-    g.status = at<int>(ws, L.status);
-    g.sched = at<int>(ws, L.sched_ffn);
-    // CTA-pair tiles: token-major pairs are 256 token rows, worth it when
-    // groups are large (ragged 256-row tails of mid-sized groups cost more
-    // than they save); weight-major pairs halve the token traffic of
-    // decode-sized groups.
+    g.status = ws ? at<int>(ws, L.status) : nullptr;
+    g.sched = ws ? at<int>(ws, L.sched_ffn) : nullptr;
+    return g;
+}
+
+// CTA-pair tiles: token-major pairs are 256 token rows, worth it when groups
+// are large (ragged 256-row tails of mid-sized groups cost more than they
+// save); weight-major pairs halve the token traffic of decode-sized groups.
+bool ffn_uses_pair(const moe_dims* d, const Layout& L, const GemmLaunch& g) {
     const bool large_groups = d->T * d->K >= static_cast<int64_t>(d->E) * 1024;
-    const bool pair = large_groups || L.swap;
-    if (pair && gemm_2sm_supported(g)) return map_launch(launch_grouped_gemm_2sm(g, st));
+    return (large_groups || L.swap) && gemm_2sm_supported(g);
+}
+
+// Both expert GEMMs in one launch.  The scheduler words at L.sched_ffn must
+// be zero when it starts (the dispatch kernels clear them; the standalone
+// entry point clears them with a memset).
+int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
+           const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st) {
+    const GemmLaunch g = ffn_launch(d, L, xperm, offsets, W13p, W2p, h, yout, nsplit, ws);
+    if (ffn_uses_pair(d, L, g)) return map_launch(launch_grouped_gemm_2sm(g, st));
     return map_launch(launch_grouped_gemm(g, st));
 }
 
@@ -465,6 +474,16 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
         MOE_TRY(map_launch(launch_bias_update(counts, dims->T, dims->E, dims->K, alpha, bias, st)));
     mark(5);
     return MOE_OK;
+}
+
+int moe_ffn_kernel(const moe_dims* dims) {
+    MOE_TRY(check_dims(dims));
+    const Layout L = layout_of(dims);
+    // placeholder (never dereferenced) pointers: only the shape decides
+    static const int32_t dummy_offsets[1] = {0};
+    const GemmLaunch g = ffn_launch(dims, L, nullptr, dummy_offsets, nullptr, nullptr, nullptr, nullptr, L.nsplit,
+                                    nullptr);
+    return ffn_uses_pair(dims, L, g) ? 1 : 0;
 }
 
 int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update) {

@@ -101,3 +101,17 @@ def test_noalloc_dispatch_rejects_oversize_on_the_host(lib):
     st = lib.moe_permute_noalloc(ctypes.byref(d), fake, None, fake, fake, fake, fake, fake, None, None, None)
     assert st == abi.MOE_ESCRATCH
     assert abi.moe_status_str(abi.MOE_ESCRATCH).startswith("MOE_ESCRATCH")
+
+
+def test_ffn_kernel_choice_by_shape(lib):
+    # decode-sized groups with 256-multiple widths: weight-major CTA pairs
+    assert abi.moe_ffn_kernel(abi.Dims(256, 4096, 14336, 8, 2)) == "grouped_gemm_2sm_kernel"
+    # prefill-sized groups: token-major CTA pairs
+    assert abi.moe_ffn_kernel(abi.Dims(16384, 4096, 14336, 8, 2)) == "grouped_gemm_2sm_kernel"
+    # mid-sized groups (mean 546 rows) keep single-CTA tiles
+    assert abi.moe_ffn_kernel(abi.Dims(8192, 2048, 1408, 60, 4, 1.0)) == "grouped_gemm_kernel"
+    # widths that are not multiples of 256 cannot take 256-wide pair tiles
+    assert abi.moe_ffn_kernel(abi.Dims(64, 128, 256, 8, 2)) == "grouped_gemm_kernel"
+    bad = abi.Dims(0, 4096, 14336, 8, 2)
+    with pytest.raises(abi.MoEError):
+        abi.moe_ffn_kernel(bad)
