@@ -243,7 +243,8 @@ typedef struct moe_layer_outputs {
      * layer records, on `stream`: [0] before routing, [1] after routing,
      * [2] after dispatch, [3] after the expert GEMMs (gate/up and down run
      * in one launch), [4] after combine, [5] after statistics and the bias
-     * update.  For per-stage timing. */
+     * update (these run in one extra CTA of the combine launch, so [4] and
+     * [5] mark the same point).  For per-stage timing. */
     void* const* stage_events; /* [MOE_NUM_STAGE_EVENTS] */
 } moe_layer_outputs;
 

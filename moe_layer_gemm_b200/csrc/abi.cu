@@ -74,14 +74,17 @@ int choose_swap(const moe_dims* d) {
     return (avg <= 256 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
 }
 
-// Reduction split of weight-major down-projection tiles: about as many
-// weight bytes per tile as a gate/up tile (128 x d_model), so the dynamic
-// scheduler's last tiles are short.
+// Reduction split of the down projection when groups are decode-sized: a
+// tile then holds at most about twice the weight bytes of a gate/up tile
+// (reduction length 2 d_model instead of d_ff), so the dynamic scheduler's
+// last tiles are short, while the fp32 partial slices the split writes and
+// the combine reads stay few (a same-box A/B at the Mixtral decode shape:
+// 2 slices beat 3 and 4).
 int choose_nsplit(const moe_dims* d, int swap) {
     if (!swap) return 1;
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
     if (avg > kSwapMaxRows) return 1;
-    int ks = static_cast<int>((d->d_ff + d->d_model - 1) / d->d_model);
+    int ks = static_cast<int>((d->d_ff + 2 * d->d_model - 1) / (2 * d->d_model));
     if (ks < 1) ks = 1;
     if (ks > 8) ks = 8;
     return ks;
@@ -464,14 +467,26 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
     MOE_TRY(do_ffn(dims, L, at<bf16>(ws, L.xperm), offsets, reinterpret_cast<const bf16*>(W13p),
                    reinterpret_cast<const bf16*>(W2p), at<bf16>(ws, L.h), yp, L.nsplit, ws, st));
     mark(3);
+    // statistics and the bias update ride on the combine launch as one extra CTA
+    StatsTail tail{};
+    if (want_stats || (bias && alpha != 0.0f)) {
+        tail.counts = counts;
+        tail.E = dims->E;
+        if (want_stats) {
+            tail.part = at<float>(ws, L.prob_part);
+            tail.nblocks = L.route_nb;
+            tail.P = P;
+            tail.f = o.f;
+            tail.aux = o.aux;
+        }
+        if (bias && alpha != 0.0f) {
+            tail.bias = bias;
+            tail.alpha = alpha;
+        }
+    }
     MOE_TRY(map_launch(launch_combine(yp, L.nsplit, dims->T * dims->K * dims->d_model, inv, w, dims->T,
-                                      dims->d_model, dims->K, y, st)));
+                                      dims->d_model, dims->K, y, st, &tail)));
     mark(4);
-    if (want_stats)
-        MOE_TRY(map_launch(launch_finalize_stats(at<float>(ws, L.prob_part), L.route_nb, counts, dims->T, dims->E,
-                                                 dims->K, P, o.f, o.aux, st)));
-    if (bias && alpha != 0.0f)
-        MOE_TRY(map_launch(launch_bias_update(counts, dims->T, dims->E, dims->K, alpha, bias, st)));
     mark(5);
     return MOE_OK;
 }
@@ -492,9 +507,9 @@ int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update) {
     int n = L.fused_router ? 1 : 3;  // fused router, or transpose + logits GEMM + top-K
     n += launch_count(dims->T) + 1;  // dispatch kernels + row gather
     n += 1;                          // both expert GEMMs in one persistent launch
-    n += 1;                          // combine
-    if (stats) n += 1;               // P_i, f_i and aux
-    if (bias_update) n += 1;
+    n += 1;                          // combine, with P_i, f_i, aux and the bias update in one extra CTA
+    (void)stats;
+    (void)bias_update;
     return n;
 }
 

@@ -25,15 +25,75 @@ constexpr int kMaxK = 16;
 
 constexpr int kMaxSplit = 8;
 
+__device__ __forceinline__ float warp_sum_fixed(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// The statistics tail (one CTA of any multiple of 32 threads): warp w
+// reduces experts w, w + nw, ...: lane l adds router blocks l, l + 32, ...
+// in order, then a fixed butterfly; P_i = sum / T, f_i = counts_i / (T K);
+// aux = E * sum_i f_i P_i summed per warp in expert order, then over warps
+// in warp order.  Then the bias update, one expert per thread.  Every sum
+// has a fixed order, so results are reproducible.
+__device__ void stats_tail(const StatsTail& s, int64_t T, int K) {
+    __shared__ float red[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int E = s.E;
+    if (s.part) {
+        const float invT = 1.0f / static_cast<float>(T);
+        const float invA = 1.0f / static_cast<float>(T * K);
+        float acc = 0.f;
+        for (int e = warp; e < E; e += nw) {
+            float sum = 0.f;
+            for (int b = lane; b < s.nblocks; b += 32) sum += s.part[static_cast<int64_t>(b) * E + e];
+            sum = warp_sum_fixed(sum);
+            const float pe = sum * invT;
+            const float fe = static_cast<float>(s.counts[e]) * invA;
+            if (lane == 0) {
+                s.P[e] = pe;
+                if (s.f) s.f[e] = fe;
+                acc += fe * pe;
+            }
+        }
+        if (lane == 0) red[warp] = acc;
+        __syncthreads();
+        if (threadIdx.x == 0 && s.aux) {
+            float a = 0.f;
+            for (int i = 0; i < nw; ++i) a += red[i];
+            *s.aux = static_cast<float>(E) * a;
+        }
+    }
+    if (s.bias && s.alpha != 0.0f) {
+        const int64_t TK = T * K;
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const int64_t lhs = static_cast<int64_t>(s.counts[e]) * E;
+            float b = s.bias[e];
+            if (lhs > TK) b = __fsub_rn(b, s.alpha);
+            else if (lhs < TK) b = __fadd_rn(b, s.alpha);
+            s.bias[e] = b;
+        }
+    }
+}
+
 // S >= nsplit slots for partial slices (S == nsplit except the 8-slot
 // fallback, which reads only the nsplit slices that exist).
 template <int S>
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, const int32_t* __restrict__ inv,
-               const float* __restrict__ w, int64_t T, int d, int K, float* __restrict__ y) {
+               const float* __restrict__ w, int64_t T, int d, int K, float* __restrict__ y, const StatsTail tail) {
+    pdl_trigger();
+    pdl_wait();
+    // with a statistics tail the last CTA does only that
+    const int ntok_blocks = static_cast<int>(gridDim.x) - (tail.counts ? 1 : 0);
+    if (tail.counts && static_cast<int>(blockIdx.x) == ntok_blocks) {
+        stats_tail(tail, T, K);
+        return;
+    }
     const int nvec = d / 4;
     const int64_t svec = split_stride / 4;
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    for (int64_t t = blockIdx.x; t < T; t += ntok_blocks) {
         int32_t rows[kMaxK];
         float ws[kMaxK];
         for (int k = 0; k < K; ++k) {
@@ -83,6 +143,8 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
 __global__ void __launch_bounds__(256)
 reduce_splits_kernel(const float* __restrict__ part, int nsplit, int64_t split_stride,
                      const int32_t* __restrict__ offsets, int E, int d, float* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t n = static_cast<int64_t>(offsets[E]) * (d / 4);
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -99,6 +161,8 @@ reduce_splits_kernel(const float* __restrict__ part, int nsplit, int64_t split_s
 __global__ void __launch_bounds__(256)
 stats_kernel(const int32_t* __restrict__ counts, const float* __restrict__ P, int64_t T, int E, int K,
              float* __restrict__ f, float* __restrict__ aux) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ float red[256];
     const float inv = 1.0f / static_cast<float>(T * K);
     float part = 0.f;
@@ -116,47 +180,11 @@ stats_kernel(const int32_t* __restrict__ counts, const float* __restrict__ P, in
     if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
 }
 
-// One block of 1024 threads: P_i = (sum over router blocks of the per-block
-// sums) / T.  Warp w reduces experts w, w+32, ...: lane l adds blocks l,
-// l+32, ... in order, then a fixed butterfly across lanes; f_i and aux as in
-// stats_kernel.  Every sum has a fixed order, so results are reproducible.
-__device__ __forceinline__ float warp_sum_fixed(float x) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-__global__ void __launch_bounds__(1024)
-finalize_stats_kernel(const float* __restrict__ part, int nblocks, const int32_t* __restrict__ counts, int64_t T,
-                      int E, int K, float* __restrict__ P, float* __restrict__ f, float* __restrict__ aux) {
-    __shared__ float red[1024];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    const float invT = 1.0f / static_cast<float>(T);
-    const float invA = 1.0f / static_cast<float>(T * K);
-    float acc = 0.f;
-    for (int e = warp; e < E; e += nw) {
-        float s = 0.f;
-        for (int b = lane; b < nblocks; b += 32) s += part[static_cast<int64_t>(b) * E + e];
-        s = warp_sum_fixed(s);
-        const float pe = s * invT;
-        const float fe = static_cast<float>(counts[e]) * invA;
-        if (lane == 0) {
-            if (P) P[e] = pe;
-            if (f) f[e] = fe;
-            acc += fe * pe;
-        }
-    }
-    red[threadIdx.x] = acc;
-    __syncthreads();
-    for (int st = blockDim.x / 2; st > 0; st >>= 1) {
-        if (threadIdx.x < st) red[threadIdx.x] += red[threadIdx.x + st];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0 && aux) *aux = static_cast<float>(E) * red[0];
-}
 
 __global__ void bias_update_kernel(const int32_t* __restrict__ counts, int64_t TK, int E, float alpha,
                                    float* __restrict__ bias) {
+    pdl_trigger();
+    pdl_wait();
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= E) return;
     const int64_t lhs = static_cast<int64_t>(counts[e]) * E;
@@ -217,19 +245,25 @@ __global__ void pack_w2_kernel(const __nv_bfloat16* __restrict__ W2, int d, int 
 }  // namespace
 
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv, const float* w,
-                   int64_t T, int d, int K, float* y, cudaStream_t st) {
+                   int64_t T, int d, int K, float* y, cudaStream_t st, const StatsTail* tail_in) {
     if (K > kMaxK || d % 4 != 0 || nsplit < 1 || nsplit > kMaxSplit) return -2;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     int64_t grid = T < static_cast<int64_t>(sms) * 16 ? T : static_cast<int64_t>(sms) * 16;
     if (grid < 1) grid = 1;
     const int threads = d / 4 >= 256 ? 256 : ((d / 4 + 31) / 32) * 32;
+    StatsTail tail{};
+    if (tail_in && tail_in->counts) {
+        tail = *tail_in;
+        if (tail.part && !tail.P) return -2;
+        ++grid;  // one extra CTA for the tail
+    }
     const int g = static_cast<int>(grid);
     switch (nsplit) {
-        case 1: combine_kernel<1><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
-        case 2: combine_kernel<2><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
-        case 3: combine_kernel<3><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
-        case 4: combine_kernel<4><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
-        default: combine_kernel<8><<<g, threads, 0, st>>>(y_perm, nsplit, split_stride, inv, w, T, d, K, y); break;
+        case 1: (void)launch_pdl(combine_kernel<1>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        case 2: (void)launch_pdl(combine_kernel<2>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        case 3: (void)launch_pdl(combine_kernel<3>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        case 4: (void)launch_pdl(combine_kernel<4>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        default: (void)launch_pdl(combine_kernel<8>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
     }
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
@@ -237,24 +271,19 @@ int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const 
 int launch_reduce_splits(const float* part, int nsplit, int64_t split_stride, const int32_t* offsets, int E, int d,
                          float* y_perm, cudaStream_t st) {
     const int sms = num_sms() > 0 ? num_sms() : 148;
-    reduce_splits_kernel<<<sms * 4, 256, 0, st>>>(part, nsplit, split_stride, offsets, E, d, y_perm);
+    (void)launch_pdl(reduce_splits_kernel, dim3(sms * 4), dim3(256), 0, st, part, nsplit, split_stride, offsets, E, d, y_perm);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
 int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E, int K, float* f, float* aux,
                  const float*, cudaStream_t st) {
-    stats_kernel<<<1, 256, 0, st>>>(counts, prob_mean, T, E, K, f, aux);
+    (void)launch_pdl(stats_kernel, dim3(1), dim3(256), 0, st, counts, prob_mean, T, E, K, f, aux);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
-int launch_finalize_stats(const float* prob_part, int nblocks, const int32_t* counts, int64_t T, int E, int K,
-                          float* P, float* f, float* aux, cudaStream_t st) {
-    finalize_stats_kernel<<<1, 1024, 0, st>>>(prob_part, nblocks, counts, T, E, K, P, f, aux);
-    return cudaGetLastError() == cudaSuccess ? 0 : -3;
-}
 
 int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias, cudaStream_t st) {
-    bias_update_kernel<<<(E + 255) / 256, 256, 0, st>>>(counts, T * K, E, alpha, bias);
+    (void)launch_pdl(bias_update_kernel, dim3((E + 255) / 256), dim3(256), 0, st, counts, T * K, E, alpha, bias);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

@@ -231,6 +231,9 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         }
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    // group offsets, scheduler words and token rows come from earlier kernels;
+    // no early trigger: the next kernel launches as this one drains
+    pdl_wait();
     for (int g = threadIdx.x; g <= G; g += blockDim.x)
         off[g] = a.group_off ? static_cast<int64_t>(a.group_off[g]) : (g == 0 ? 0 : a.dense_rows);
     __syncthreads();
@@ -652,7 +655,7 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         bound += tm > sw ? tm : sw;
     }
     const int grid = static_cast<int>(bound < sms ? (bound < 1 ? 1 : bound) : sms);
-    grouped_gemm_kernel<<<grid, kThreads, smem, st>>>(maps, a);
+    if (launch_pdl(grouped_gemm_kernel, dim3(grid), dim3(kThreads), smem, st, maps, a) != cudaSuccess) return -3;
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

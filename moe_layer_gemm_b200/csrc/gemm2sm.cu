@@ -18,9 +18,14 @@
 // weight rows (CTA r loads the 128-row weight tile n0 + 128 r), its N side
 // the group's tokens, of which each CTA loads half.  Against single-CTA
 // weight-major tiles this halves the token traffic and the MMA instructions
-// per SM, and when no group can take token-major tiles the token slot is
-// only 8 KB, so the weight ring is deeper.  The down projection's reduction
-// can be split as in gemm.cu.
+// per SM.  Where the phase has tiles to spare, a weight-major pair tile
+// covers two such 256-row sub-tiles that share one token load, issuing two
+// MMAs into two TMEM accumulators, which halves the token traffic again.
+// The down projection's reduction can be split as in gemm.cu.
+//
+// Stage layout (per CTA): token-major tiles put their 128 token rows at 0
+// and their 128 weight rows at 16 KB; weight-major tiles put weight
+// sub-tile j at 16 KB j and their token rows at xoff.
 //
 // Pair protocol (barriers live in each CTA; "leader" means rank 0's copy):
 //   full[s]    leader only: the leader registers the pair's bytes, both CTAs'
@@ -53,7 +58,8 @@ constexpr int kRing = 8;
 struct Phase2 {
     int N, k_blocks, epi;
     int64_t nb;  // 128-row weight blocks per group
-    int ksplit, kb_per_split;  // weight-major tiles only
+    int ksplit, kb_per_split;  // reduction split (every tile of the phase)
+    int wt;                    // weight-major tiles: 256-row weight sub-tiles per pair tile (1 or 2)
     void* out;
     int64_t ldo;
     int64_t split_stride;
@@ -68,7 +74,8 @@ struct Args2 {
     int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 128)
     Phase2 ph[2];
     int stages;
-    uint32_t b_slot;    // bytes of the second operand slot per stage
+    uint32_t stage_bytes;  // per stage and CTA
+    uint32_t xoff;         // weight-major tiles: offset of the token rows in a stage
     int* status;
     int* sched;
 };
@@ -85,6 +92,7 @@ struct Tile2 {
     int rows;      // valid token rows (<= 256 token-major, <= BNs weight-major)
     int n0;        // first weight row (multiple of 256)
     int kb0, kb1, split;
+    int wt;  // weight sub-tiles (weight-major tiles), else 1
 };
 
 // ---- cluster helpers
@@ -136,8 +144,9 @@ __device__ __forceinline__ bool swaps2(const Args2& a, int64_t rows) { return ro
 
 __device__ __forceinline__ int tiles_of2(const Args2& a, int p, int64_t rows) {
     if (rows <= 0) return 0;
-    const int64_t chunks = swaps2(a, rows) ? (rows + a.BNs - 1) / a.BNs : (rows + 255) / 256;
-    return static_cast<int>(chunks * (a.ph[p].N / 256) * a.ph[p].ksplit);
+    const Phase2& ph = a.ph[p];
+    if (!swaps2(a, rows)) return static_cast<int>(((rows + 255) / 256) * (ph.N / 256) * ph.ksplit);
+    return static_cast<int>(((rows + a.BNs - 1) / a.BNs) * (ph.N / (256 * ph.wt)) * ph.ksplit);
 }
 
 __device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* tstart, const int64_t* off) {
@@ -158,8 +167,9 @@ __device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* ts
     const int64_t base = off[lo];
     const int64_t rows_g = off[lo + 1] - base;
     t.swap = swaps2(a, rows_g) ? 1 : 0;
-    // token chunk fastest (the weight tile is reused from L2), then the
-    // weight tile; the reduction split is outermost within a chunk's tiles
+    t.wt = t.swap ? ph.wt : 1;
+    // reduction split fastest, then the token chunk (the weight tile is
+    // reused from L2), then the weight tile
     const int chunk = t.swap ? a.BNs : 256;
     const int nch = static_cast<int>((rows_g + chunk - 1) / chunk);
     const int sp = local % ph.ksplit;
@@ -168,7 +178,7 @@ __device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* ts
     const int64_t r0 = static_cast<int64_t>(c) * chunk;
     t.row0 = base + r0;
     t.rows = static_cast<int>(rows_g - r0 < chunk ? rows_g - r0 : chunk);
-    t.n0 = (rest / nch) * 256;
+    t.n0 = (rest / nch) * 256 * t.wt;
     t.kb0 = sp * ph.kb_per_split;
     t.kb1 = min(ph.k_blocks, t.kb0 + ph.kb_per_split);
     t.split = sp;
@@ -198,9 +208,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int S = a.stages;
-    uint8_t* sA = smem;                                   // [S][16 KB] M-side rows of this CTA (tokens or weights)
-    uint8_t* sB = smem + static_cast<size_t>(S) * kHalf;  // [S][b_slot] N-side rows of this CTA (weights or tokens)
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + static_cast<size_t>(S) * a.b_slot);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * a.stage_bytes);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
@@ -247,6 +255,9 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
+    // group offsets, scheduler words and token rows come from earlier kernels;
+    // no early trigger: the next kernel launches as this one drains
+    pdl_wait();
     for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
     __syncthreads();
     if (warp == 0) {
@@ -337,10 +348,12 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                     if (!ok) break;
                 }
-                const int64_t wblk = static_cast<int64_t>(t.g) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
+                // this CTA's 128-row weight block of (sub-)tile j: rows n0 + 256 j + 128 rank
+                const int64_t wblk0 = static_cast<int64_t>(t.g) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
                 // weight-major: this CTA's half of the tile's token columns, in 16-row boxes
                 const int nb16 = t.swap ? (t.rows + 31) / 32 : 0;
-                const uint32_t pair_bytes = t.swap ? 2u * (kHalf + static_cast<uint32_t>(nb16) * 2048u) : 4u * kHalf;
+                const uint32_t pair_bytes =
+                    t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(nb16) * 2048u) : 4u * kHalf;
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
                         ok = false;
@@ -348,18 +361,19 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     }
                     if (leader) mbar_arrive_expect_tx(&full[s], pair_bytes);
                     const uint32_t bar = leader_full0 + 8u * s;
-                    uint8_t* dA = sA + static_cast<size_t>(s) * kHalf;
-                    uint8_t* dB = sB + static_cast<size_t>(s) * a.b_slot;
-                    const int32_t wrow = static_cast<int32_t>((wblk * pa.k_blocks + kb) * 128);
+                    uint8_t* stage = smem + static_cast<size_t>(s) * a.stage_bytes;
                     if (!t.swap) {
-                        tma_load_pair(&maps.tok[t.phase], dA, bar, kb * kBK,
+                        tma_load_pair(&maps.tok[t.phase], stage, bar, kb * kBK,
                                       static_cast<int32_t>(t.row0 + 128 * rank), pol_last);
-                        tma_load_pair(&maps.w[t.phase], dB, bar, 0, wrow, pol_first);
+                        tma_load_pair(&maps.w[t.phase], stage + kHalf, bar, 0,
+                                      static_cast<int32_t>((wblk0 * pa.k_blocks + kb) * 128), pol_first);
                     } else {
-                        tma_load_pair(&maps.w[t.phase], dA, bar, 0, wrow, pol_first);
+                        for (int j = 0; j < t.wt; ++j)
+                            tma_load_pair(&maps.w[t.phase], stage + j * kHalf, bar, 0,
+                                          static_cast<int32_t>(((wblk0 + 2 * j) * pa.k_blocks + kb) * 128), pol_first);
                         const int64_t trow = t.row0 + static_cast<int64_t>(rank) * 16 * nb16;
                         for (int j = 0; j < nb16; ++j)
-                            tma_load_pair(&maps.tok16[t.phase], dB + j * 2048, bar, kb * kBK,
+                            tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + j * 2048, bar, kb * kBK,
                                           static_cast<int32_t>(trow + 16 * j), pol_last);
                     }
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
@@ -402,12 +416,22 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(sA + static_cast<size_t>(s) * kHalf);
-                    const uint32_t b_base = smem_u32(sB + static_cast<size_t>(s) * a.b_slot);
+                    const uint32_t stage = smem_u32(smem + static_cast<size_t>(s) * a.stage_bytes);
+                    if (!t.swap) {
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        umma_pair(d_tmem, umma_desc_sw128(a_base + kk * 32), umma_desc_sw128(b_base + kk * 32), idesc,
-                                  (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            umma_pair(d_tmem, umma_desc_sw128(stage + kk * 32), umma_desc_sw128(stage + kHalf + kk * 32),
+                                      idesc, (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        // sub-tile j accumulates into columns 128 j .. of the buffer
+                        for (int j = 0; j < t.wt; ++j) {
+#pragma unroll
+                            for (int kk = 0; kk < kBK / 16; ++kk)
+                                umma_pair(d_tmem + 128u * j, umma_desc_sw128(stage + j * kHalf + kk * 32),
+                                          umma_desc_sw128(stage + a.xoff + kk * 32), idesc,
+                                          (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
                     umma_commit_pair(&empty[s]);
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
@@ -464,11 +488,13 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     }
                 }
             } else {
-                // lanes are this CTA's 128 weight rows n0 + 128 rank + .., columns the tile's tokens
-                const int nwr = t.n0 + 128 * static_cast<int>(rank);
+                // accumulator `sub`: lanes are this CTA's 128 weight rows n0 + 256 sub + 128 rank + ..,
+                // columns 128 sub + (the tile's tokens)
                 const int nbk = (t.rows + 31) / 32;
-                for (int c = 0; c < nbk; ++c) {
-                    tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                for (int cc = 0; cc < t.wt * nbk; ++cc) {
+                    const int sub = cc / nbk, c = cc - sub * nbk;
+                    const int nwr = t.n0 + 256 * sub + 128 * static_cast<int>(rank);
+                    tmem_ld32(taddr + static_cast<uint32_t>(128 * sub + c * 32), v);
                     if (pa.epi == EPI_SWIGLU_BF16) {
                         const int f = nwr / 2 + q * 16 + (lane & 15);
                         bf16* H = static_cast<bf16*>(pa.out);
@@ -566,10 +592,11 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         a.BNs = static_cast<int>(lim >= 128 ? 128 : ((lim + 31) / 32) * 32);
         if (a.BNs < 32) a.BNs = 32;
     }
-    // The N-side slot holds a 128-row weight half (token-major tiles) or
-    // BNs / 2 token rows (weight-major tiles).
     const bool token_major_possible = mx > a.swap_max_rows;
-    a.b_slot = token_major_possible ? kHalf : static_cast<uint32_t>(a.BNs) * 64u;
+    const bool weight_major_possible = a.swap_max_rows > 0;
+    const int sms = num_sms();
+    if (sms <= 1) return -3;
+    const int clusters = sms / 2;
     Maps2 maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int p = 0; p < L.nphase; ++p) {
@@ -586,6 +613,11 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         if (ks > ph.k_blocks) ks = ph.k_blocks;
         ph.kb_per_split = (ph.k_blocks + ks - 1) / ks;
         ph.ksplit = (ph.k_blocks + ph.kb_per_split - 1) / ph.kb_per_split;
+        // two 256-row weight sub-tiles per weight-major tile when the width
+        // allows and the phase still has at least 4 tiles per cluster with
+        // every group active
+        ph.wt = (weight_major_possible && g.N % 512 == 0 &&
+                 static_cast<int64_t>(L.G) * (g.N / 512) * ph.ksplit >= 4LL * clusters) ? 2 : 1;
         const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
         if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
         if (!map2(&maps.tok16[p], g.tok, trows, g.Kdim, 16u, true)) return -3;
@@ -594,11 +626,22 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     }
     const size_t fixed = 1024 + static_cast<size_t>(2 * 16 + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
                          static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + 64;
-    int stages = static_cast<int>((227 * 1024 - fixed) / (kHalf + a.b_slot));
+    // stage: token-major tiles need 2 x 16 KB; weight-major tiles wt x 16 KB
+    // of weights and BNs / 2 token rows
+    int wt_max = 1;
+    for (int p = 0; p < L.nphase; ++p) wt_max = a.ph[p].wt > wt_max ? a.ph[p].wt : wt_max;
+    a.xoff = static_cast<uint32_t>(wt_max) * kHalf;
+    uint32_t stage_bytes = token_major_possible ? 2u * kHalf : 0u;
+    if (weight_major_possible) {
+        const uint32_t wm = a.xoff + static_cast<uint32_t>(a.BNs) * 64u;
+        stage_bytes = wm > stage_bytes ? wm : stage_bytes;
+    }
+    a.stage_bytes = stage_bytes;
+    int stages = static_cast<int>((227 * 1024 - fixed) / stage_bytes);
     if (stages > 16) stages = 16;
     if (stages < 2) return -2;
     a.stages = stages;
-    const size_t smem = fixed + static_cast<size_t>(stages) * (kHalf + a.b_slot);
+    const size_t smem = fixed + static_cast<size_t>(stages) * stage_bytes;
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
@@ -606,21 +649,20 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
             return -3;
         attr = true;
     }
-    const int sms = num_sms();
-    if (sms <= 1) return -3;
-    int clusters = sms / 2;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * clusters, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attrs[1];
+    cudaLaunchAttribute attrs[2];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
     attrs[0].val.clusterDim.x = 2;
     attrs[0].val.clusterDim.y = 1;
     attrs[0].val.clusterDim.z = 1;
+    attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // pdl_wait in the kernel
+    attrs[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, grouped_gemm_2sm_kernel, maps, a) != cudaSuccess) return -3;
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }

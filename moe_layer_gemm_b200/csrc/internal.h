@@ -16,6 +16,25 @@ enum GemmEpilogue : int {
 };
 
 // One matrix product over all groups: out[rows of g] = tok[rows of g] . w[g]^T.
+// Launch `kernel` with programmatic stream serialization: it may begin
+// while the previous kernel on `st` drains, so it must call pdl_wait()
+// before using that kernel's results (see ptx.cuh).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct GemmPhase {
     const bf16* tok;      // [tok_rows, Kdim] bf16, K contiguous
     int64_t tok_rows;
@@ -76,14 +95,29 @@ int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, i
                    int zero_count, cudaStream_t st);
 
 // ------------------------------------------------------------ combine / stats
+// Work folded into the combine launch as one extra CTA: the load statistics
+// (P_i from the router's per-block sums, f_i, aux) and the aux-free bias
+// update.  Both need only routing results, which are complete when the
+// combine starts.
+struct StatsTail {
+    const float* part;      // router per-block probability sums [nblocks, E]; nullptr: no statistics
+    int nblocks;
+    const int32_t* counts;  // nullptr: no tail CTA at all
+    float* P;               // required with part
+    float* f;               // may be nullptr
+    float* aux;             // may be nullptr
+    float* bias;            // updated in place when non-null and alpha != 0
+    float alpha;
+    int E;
+};
+
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv,
-                   const float* w, int64_t T, int d, int K, float* y, cudaStream_t st);
+                   const float* w, int64_t T, int d, int K, float* y, cudaStream_t st,
+                   const StatsTail* tail = nullptr);
 int launch_reduce_splits(const float* part, int nsplit, int64_t split_stride, const int32_t* offsets,
                          int E, int d, float* y_perm, cudaStream_t st);
 int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E, int K,
                  float* f, float* aux, const float* alpha_bias_unused, cudaStream_t st);
-int launch_finalize_stats(const float* prob_part, int nblocks, const int32_t* counts, int64_t T, int E, int K,
-                          float* P, float* f, float* aux, cudaStream_t st);
 int launch_count(int64_t T);  // kernels launch_permute enqueues before the row gather
 int64_t permute_static_max_hist();
 int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,

@@ -32,6 +32,17 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch.  pdl_wait blocks until the grids this one
+// depends on (the previous kernel on the stream, when this one was launched
+// with programmatic stream serialization) have completed and their memory is
+// visible; without that launch attribute it returns at once.  Every kernel
+// launched that way calls it, unconditionally and before touching any
+// buffer another kernel writes or reads, so completion stays transitive
+// along the stream.  pdl_trigger lets the next such kernel start launching
+// once every CTA of this grid has called it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

@@ -157,6 +157,8 @@ route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
                    const float* __restrict__ bias, int64_t T, int d, int E, int K,
                    float* __restrict__ logits, int32_t* __restrict__ idx, float* __restrict__ w,
                    float* __restrict__ prob_part) {
+    pdl_trigger();
+    pdl_wait();
     constexpr int EP = EV * 8;  // padded experts per row
     extern __shared__ uint4 swr_raw[];
     // 16-byte slot s of chunk c (8 rows = 8*EV slots) lives at s ^ (c & 7):
@@ -246,6 +248,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 route_split_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr,
                    const float* __restrict__ bias, int64_t T, int d, int E, int K, float* __restrict__ logits,
                    int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ prob_part) {
+    pdl_trigger();
+    pdl_wait();
     constexpr int EP = EV * 8;
     __shared__ float part[kRouteWarps][EP];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -257,31 +261,37 @@ route_split_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
 #pragma unroll
         for (int e = 0; e < EP; ++e) acc[e] = 0.f;
         const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
-        for (int c0 = c_beg + lane; c0 < c_end; c0 += 32 * kXBatch) {
-            uint4 xv[kXBatch];
+        if (E == EP) {
+            // A W_r row is EV 16-byte vectors, so the 8 rows of one x vector
+            // are 8 EV contiguous vectors.  Every load of a batch is issued
+            // before any arithmetic: one round of L2 latency per batch.
+            constexpr int VB = EV == 1 ? 2 : 1;  // x vectors per lane per batch
+            const uint4* wr4 = reinterpret_cast<const uint4*>(Wr);
+            for (int c0 = c_beg + lane; c0 < c_end; c0 += 32 * VB) {
+                uint4 xv[VB];
+                uint4 wv[VB][8 * EV];
 #pragma unroll
-            for (int b = 0; b < kXBatch; ++b) {
-                const int c = c0 + 32 * b;
-                xv[b] = c < c_end ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
-            }
+                for (int b = 0; b < VB; ++b) {
+                    const int c = c0 + 32 * b;
+                    const bool ok = c < c_end;
+                    xv[b] = ok ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int b = 0; b < kXBatch; ++b) {
-                const int c = c0 + 32 * b;
-                if (c >= c_end) break;
-                const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv[b]);
+                    for (int j = 0; j < 8 * EV; ++j)
+                        wv[b][j] = ok ? __ldg(wr4 + static_cast<int64_t>(c) * 8 * EV + j) : make_uint4(0, 0, 0, 0);
+                }
 #pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2) {
-                    const float2 xf = __bfloat1622float2(xp[i2]);
+                for (int b = 0; b < VB; ++b) {
+                    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv[b]);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const float xs = half ? xf.y : xf.x;
-                        const int row = c * 8 + 2 * i2 + half;
-                        if (E == EP) {  // a W_r row is EV whole 16-byte vectors
-                            const uint4* wrow = reinterpret_cast<const uint4*>(Wr + static_cast<int64_t>(row) * EP);
+                    for (int i2 = 0; i2 < 4; ++i2) {
+                        const float2 xf = __bfloat1622float2(xp[i2]);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const float xs = half ? xf.y : xf.x;
 #pragma unroll
                             for (int vv = 0; vv < EV; ++vv) {
-                                const uint4 wv = __ldg(wrow + vv);
-                                const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&wv);
+                                const __nv_bfloat162* wp =
+                                    reinterpret_cast<const __nv_bfloat162*>(&wv[b][(2 * i2 + half) * EV + vv]);
 #pragma unroll
                                 for (int h = 0; h < 4; ++h) {
                                     const float2 w2 = __bfloat1622float2(wp[h]);
@@ -289,7 +299,30 @@ route_split_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
                                     acc[vv * 8 + 2 * h + 1] = fmaf(xs, w2.y, acc[vv * 8 + 2 * h + 1]);
                                 }
                             }
-                        } else {
+                        }
+                    }
+                }
+            }
+        } else {
+            for (int c0 = c_beg + lane; c0 < c_end; c0 += 32 * kXBatch) {
+                uint4 xv[kXBatch];
+#pragma unroll
+                for (int b = 0; b < kXBatch; ++b) {
+                    const int c = c0 + 32 * b;
+                    xv[b] = c < c_end ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int b = 0; b < kXBatch; ++b) {
+                    const int c = c0 + 32 * b;
+                    if (c >= c_end) break;
+                    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv[b]);
+#pragma unroll
+                    for (int i2 = 0; i2 < 4; ++i2) {
+                        const float2 xf = __bfloat1622float2(xp[i2]);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const float xs = half ? xf.y : xf.x;
+                            const int row = c * 8 + 2 * i2 + half;
 #pragma unroll
                             for (int e = 0; e < EP; ++e) {
                                 const float wv =
@@ -329,6 +362,8 @@ template <int J>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 topk_from_logits_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int64_t T, int E,
                         int K, int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ prob_part) {
+    pdl_trigger();
+    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kRouteWarps;
     float psum[J];
@@ -353,6 +388,8 @@ topk_from_logits_kernel(const float* __restrict__ logits, const float* __restric
 // l+32, ... in order, then a fixed butterfly (reproducible).
 __global__ void __launch_bounds__(1024)
 prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float invT, float* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int e = warp; e < E; e += nw) {
         float s = 0.f;
@@ -365,6 +402,8 @@ prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float i
 // WrT[e][k] = Wr[k][e] for e < E, 0 for E <= e < E_pad.
 __global__ void transpose_router_kernel(const __nv_bfloat16* __restrict__ Wr, int d, int E, int E_pad,
                                         __nv_bfloat16* __restrict__ WrT) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ __nv_bfloat16 tile[32][33];
     const int k0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -406,7 +445,7 @@ int launch_fused_ev(const bf16* x, const bf16* Wr, const float* bias, int64_t T,
         attr = true;
     }
     const size_t smem = static_cast<size_t>(d) * EV * 8 * 2;
-    route_fused_kernel<EV><<<nblocks, kRouteWarps * 32, smem, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+    (void)launch_pdl(route_fused_kernel<EV>, dim3(nblocks), dim3(kRouteWarps * 32), smem, st, x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
@@ -416,11 +455,14 @@ int launch_route_fused(const bf16* x, const bf16* Wr, const float* bias, int64_t
         // nblocks == T here (route_blocks): one CTA per token
         const int th = kRouteWarps * 32;
         if (E <= 8)
-            route_split_kernel<1><<<static_cast<int>(T), th, 0, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+            (void)launch_pdl(route_split_kernel<1>, dim3(static_cast<unsigned>(T)), dim3(th), 0, st, x, Wr, bias, T, d, E, K, logits,
+                             idx, w, prob_part);
         else if (E <= 16)
-            route_split_kernel<2><<<static_cast<int>(T), th, 0, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+            (void)launch_pdl(route_split_kernel<2>, dim3(static_cast<unsigned>(T)), dim3(th), 0, st, x, Wr, bias, T, d, E, K, logits,
+                             idx, w, prob_part);
         else
-            route_split_kernel<4><<<static_cast<int>(T), th, 0, st>>>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
+            (void)launch_pdl(route_split_kernel<4>, dim3(static_cast<unsigned>(T)), dim3(th), 0, st, x, Wr, bias, T, d, E, K, logits,
+                             idx, w, prob_part);
         return cudaGetLastError() == cudaSuccess ? 0 : -3;
     }
     if (E <= 8) return launch_fused_ev<1>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
@@ -432,26 +474,26 @@ int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, i
                             float* w, float* prob_part, int nblocks, cudaStream_t st) {
     const int th = kRouteWarps * 32;
     if (E <= 32)
-        topk_from_logits_kernel<1><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<1>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
     else if (E <= 64)
-        topk_from_logits_kernel<2><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<2>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
     else if (E <= 128)
-        topk_from_logits_kernel<4><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<4>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
     else if (E <= 256)
-        topk_from_logits_kernel<8><<<nblocks, th, 0, st>>>(logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<8>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
     else
         return -2;
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
 int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, float* prob_mean, cudaStream_t st) {
-    prob_finalize_kernel<<<1, 1024, 0, st>>>(prob_part, nblocks, E, 1.0f / static_cast<float>(T), prob_mean);
+    (void)launch_pdl(prob_finalize_kernel, dim3(1), dim3(1024), 0, st, prob_part, nblocks, E, 1.0f / static_cast<float>(T), prob_mean);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
 int launch_transpose_router(const bf16* Wr, int d, int E, int E_pad, bf16* WrT, cudaStream_t st) {
     dim3 grid(((d + 63) / 64) * 2, (E_pad + 31) / 32), block(32, 8);  // columns up to the tile padding
-    transpose_router_kernel<<<grid, block, 0, st>>>(Wr, d, E, E_pad, WrT);
+    (void)launch_pdl(transpose_router_kernel, dim3(grid), dim3(block), 0, st, Wr, d, E, E_pad, WrT);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
