@@ -74,17 +74,16 @@ int choose_swap(const moe_dims* d) {
     return (avg <= 256 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
 }
 
-// Reduction split of the down projection when groups are decode-sized: a
-// tile then holds at most about twice the weight bytes of a gate/up tile
-// (reduction length 2 d_model instead of d_ff), so the dynamic scheduler's
-// last tiles are short, while the fp32 partial slices the split writes and
-// the combine reads stay few (a same-box A/B at the Mixtral decode shape:
-// 2 slices beat 3 and 4).
+// Reduction split of the down projection when groups are decode-sized:
+// about as many weight bytes per tile as a gate/up tile (reduction length
+// d_model instead of d_ff), so the dynamic scheduler's last tiles are short
+// and there are tiles enough for the CTA-pair kernel to give each weight-
+// major tile two weight sub-tiles (half the token reads).
 int choose_nsplit(const moe_dims* d, int swap) {
     if (!swap) return 1;
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
     if (avg > kSwapMaxRows) return 1;
-    int ks = static_cast<int>((d->d_ff + 2 * d->d_model - 1) / (2 * d->d_model));
+    int ks = static_cast<int>((d->d_ff + d->d_model - 1) / d->d_model);
     if (ks < 1) ks = 1;
     if (ks > 8) ks = 8;
     return ks;

@@ -613,11 +613,14 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         if (ks > ph.k_blocks) ks = ph.k_blocks;
         ph.kb_per_split = (ph.k_blocks + ks - 1) / ks;
         ph.ksplit = (ph.k_blocks + ph.kb_per_split - 1) / ph.kb_per_split;
-        // two 256-row weight sub-tiles per weight-major tile when the width
-        // allows and the phase still has at least 4 tiles per cluster with
-        // every group active
+        // Two 256-row weight sub-tiles per weight-major tile when the width
+        // allows and the phase still has at least 3 tiles per cluster with
+        // every group active.  (Single sub-tiles for the groups scheduled
+        // last, to shorten the final tiles, measured slower at the Mixtral
+        // decode shape: their extra token reads cost more than the shorter
+        // tail saved.)
         ph.wt = (weight_major_possible && g.N % 512 == 0 &&
-                 static_cast<int64_t>(L.G) * (g.N / 512) * ph.ksplit >= 4LL * clusters) ? 2 : 1;
+                 static_cast<int64_t>(L.G) * (g.N / 512) * ph.ksplit >= 3LL * clusters) ? 2 : 1;
         const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
         if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
         if (!map2(&maps.tok16[p], g.tok, trows, g.Kdim, 16u, true)) return -3;

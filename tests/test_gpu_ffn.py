@@ -67,14 +67,14 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (130, 128, 128, 1, 1, 0.0),       # single expert = dense FFN
     (2100, 512, 256, 4, 2, 0.0),      # mean group >= 1024 rows, widths x256: CTA-pair tiles, ragged tail
     (6200, 256, 384, 6, 1, 1.5),      # CTA-pair tiles with skewed groups (the smallest may be tiny)
-    (256, 256, 1024, 8, 2, 1.5),      # decode-like CTA pairs, 2-way split, one group > 128 rows (token-major)
-    (256, 256, 1408, 8, 2, 0.0),      # decode-like CTA pairs, 3-way split of 22 k-blocks (8, 8, 6)
-    (256, 384, 1536, 8, 2, 1.5),      # single-CTA, 2-way split, one group > 128 rows (token-major)
-    (256, 128, 1024, 8, 2, 0.0),      # single-CTA, 4-way split
-    (40, 256, 1024, 8, 2, 0.0),       # CTA pairs, groups under 16 rows, 2-way split
+    (256, 256, 1024, 8, 2, 1.5),      # decode-like CTA pairs, 4-way split, one group > 128 rows (token-major)
+    (256, 256, 1408, 8, 2, 0.0),      # decode-like CTA pairs, 6-way split of 22 k-blocks (4, 4, 4, 4, 4, 2)
+    (256, 384, 1536, 8, 2, 1.5),      # single-CTA, 4-way split, one group > 128 rows (token-major)
+    (256, 128, 1024, 8, 2, 0.0),      # single-CTA, 8-way split
+    (40, 256, 1024, 8, 2, 0.0),       # CTA pairs, groups under 16 rows, 4-way split
     (600, 256, 256, 16, 4, 1.2),      # CTA pairs, weight- and token-major groups in one launch
-    (512, 256, 2560, 64, 4, 0.0),     # CTA pairs, gate/up tiles of two 256-row weight sub-tiles, 5-way split
-    (1024, 1024, 1024, 256, 8, 1.1),  # CTA pairs, both phases with two weight sub-tiles, skewed small groups
+    (512, 256, 2560, 64, 4, 0.0),     # CTA pairs, gate/up tiles of two 256-row weight sub-tiles, 8-way split
+    (1024, 1024, 1024, 256, 8, 1.1),  # CTA pairs, two weight sub-tiles in both phases, skewed small groups
 ])
 def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
     # weight scale shrinks with the width so |y| stays O(1), the scale the
