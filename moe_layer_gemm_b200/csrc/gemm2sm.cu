@@ -350,8 +350,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 }
                 // this CTA's 128-row weight block of (sub-)tile j: rows n0 + 256 j + 128 rank
                 const int64_t wblk0 = static_cast<int64_t>(t.g) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
-                // weight-major: this CTA's half of the tile's token columns, in 16-row boxes
-                const int nb16 = t.swap ? (t.rows + 31) / 32 : 0;
+                // weight-major: the MMA's N is the tile's tokens rounded up to 16;
+                // this CTA holds N / 2 of them (a multiple of 8), loaded in 16-row boxes
+                const int half = t.swap ? ((t.rows + 15) / 16) * 8 : 0;
+                const int nb16 = (half + 15) / 16;
                 const uint32_t pair_bytes =
                     t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(nb16) * 2048u) : 4u * kHalf;
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
@@ -371,7 +373,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                         for (int j = 0; j < t.wt; ++j)
                             tma_load_pair(&maps.w[t.phase], stage + j * kHalf, bar, 0,
                                           static_cast<int32_t>(((wblk0 + 2 * j) * pa.k_blocks + kb) * 128), pol_first);
-                        const int64_t trow = t.row0 + static_cast<int64_t>(rank) * 16 * nb16;
+                        const int64_t trow = t.row0 + static_cast<int64_t>(rank) * half;
                         for (int j = 0; j < nb16; ++j)
                             tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + j * 2048, bar, kb * kBK,
                                           static_cast<int32_t>(trow + 16 * j), pol_last);
@@ -408,7 +410,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
-                const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 31) / 32) * 32u : 256u;
+                const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 15) / 16) * 16u : 256u;
                 const uint32_t idesc = umma_idesc_bf16(256, n_mma);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
