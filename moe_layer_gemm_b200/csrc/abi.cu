@@ -456,11 +456,17 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
     MOE_TRY(do_route(dims, L, xb, reinterpret_cast<const bf16*>(Wr), bias, o.logits, idx, w,
                      want_stats ? P : nullptr, ws, st, /*finalize=*/false));
     mark(1);
-    MOE_TRY(map_launch(launch_permute(idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
-                                      at<int32_t>(ws, L.block_hist), counts, kept, offsets, inv,
-                                      at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop,
-                                      at<int32_t>(ws, L.sched_ffn), static_cast<int>(gemm_sched_bytes(dims->E) / 4),
-                                      st)));
+    if (dispatch_gather_fused_supported(dims->T, dims->E, dims->K))
+        MOE_TRY(map_launch(launch_dispatch_gather_small(
+            idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims), counts, kept, offsets, inv,
+            at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop, at<int32_t>(ws, L.sched_ffn),
+            static_cast<int>(gemm_sched_bytes(dims->E) / 4), st)));
+    else
+        MOE_TRY(map_launch(launch_permute(idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
+                                          at<int32_t>(ws, L.block_hist), counts, kept, offsets, inv,
+                                          at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop,
+                                          at<int32_t>(ws, L.sched_ffn),
+                                          static_cast<int>(gemm_sched_bytes(dims->E) / 4), st)));
     mark(2);
     float* yp = at<float>(ws, L.yperm);
     MOE_TRY(do_ffn(dims, L, at<bf16>(ws, L.xperm), offsets, reinterpret_cast<const bf16*>(W13p),
@@ -504,7 +510,8 @@ int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update) {
     if (check_dims(dims) != MOE_OK) return -1;
     const Layout L = layout_of(dims);
     int n = L.fused_router ? 1 : 3;  // fused router, or transpose + logits GEMM + top-K
-    n += launch_count(dims->T) + 1;  // dispatch kernels + row gather
+    // dispatch kernels + row gather (one fused launch for small batches)
+    n += dispatch_gather_fused_supported(dims->T, dims->E, dims->K) ? 1 : launch_count(dims->T) + 1;
     n += 1;                          // both expert GEMMs in one persistent launch
     n += 1;                          // combine, with P_i, f_i, aux and the bias update in one extra CTA
     (void)stats;

@@ -119,6 +119,13 @@ int launch_reduce_splits(const float* part, int nsplit, int64_t split_stride, co
 int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E, int K,
                  float* f, float* aux, const float* alpha_bias_unused, cudaStream_t st);
 int launch_count(int64_t T);  // kernels launch_permute enqueues before the row gather
+// The layer's small-batch dispatch: counts, ranks and the row gather in one
+// launch (results identical to launch_permute's).
+bool dispatch_gather_fused_supported(int64_t T, int E, int K);
+int launch_dispatch_gather_small(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
+                                 int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
+                                 bf16* x_perm, int32_t* n_dropped, int32_t* zero_out, int zero_count,
+                                 cudaStream_t st);
 int64_t permute_static_max_hist();
 int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                           int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,

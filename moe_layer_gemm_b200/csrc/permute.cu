@@ -23,6 +23,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -284,6 +285,131 @@ gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ i
     }
 }
 
+// Dispatch and row gather of a batch of T <= kSmallT tokens in one launch
+// (the layer's path; moe_permute keeps the two-kernel form).  Every CTA
+// computes the whole dispatch in shared memory, exactly as
+// dispatch_small_kernel does (same counts, ranks and rows); CTA 0 also
+// writes the results out.  Each CTA then copies its share of (token, slice)
+// jobs straight from its shared copy of the rows, so the gather needs no
+// second launch and no global read of inv.
+__global__ void __launch_bounds__(kSmallThreads)
+dispatch_gather_small_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ x, int T, int d,
+                             int E, int K, int64_t C, int parts, int32_t* __restrict__ counts,
+                             int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ inv,
+                             int32_t* __restrict__ src, int32_t* __restrict__ n_dropped,
+                             __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ zero_out, int zero_count) {
+    pdl_trigger();
+    pdl_wait();
+    constexpr int W = kSmallThreads / 32;
+    const bool writer = blockIdx.x == 0;
+    if (writer)
+        for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_out[i] = 0;  // next kernel's scheduler words
+    extern __shared__ int32_t sm[];
+    int32_t* wh = sm;                                              // [W][E]
+    unsigned* tmask = reinterpret_cast<unsigned*>(wh + W * E);     // [W][E]
+    int* tag = reinterpret_cast<int*>(tmask + W * E);              // [W][E]
+    int32_t* soff = tag + W * E;                                   // [E+1]
+    int32_t* srow = soff + E + 1;                                  // [T][K] row of (t, k), or -1
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = threadIdx.x;
+    const bool live = t < T;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) {
+        wh[i] = 0;
+        tag[i] = 0;
+    }
+    __syncthreads();
+    int my[kMaxK];
+    for (int k = 0; k < K; ++k) {
+        my[k] = live ? idx[t * K + k] : -1;
+        if (live) atomicAdd(&wh[warp * E + my[k]], 1);
+    }
+    int pre[kMaxK];
+    warp_prefix(my, K, lane, WarpTable{tmask + warp * E, tag + warp * E}, 1, pre);
+    __syncthreads();
+    if (warp == 0) {
+        // totals, capacity, exclusive scan of kept counts, drops
+        const int per = (E + 31) / 32;
+        int s = 0, dsum = 0;
+        int kp_local[8];
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            int kp = 0;
+            if (e < E) {
+                int c = 0;
+                for (int w2 = 0; w2 < W; ++w2) c += wh[w2 * E + e];
+                kp = (C >= 0 && c > C) ? static_cast<int>(C) : c;
+                if (writer) {
+                    counts[e] = c;
+                    kept[e] = kp;
+                }
+                dsum += c - kp;
+            }
+            kp_local[i] = kp;
+            s += kp;
+        }
+        int incl = s;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - s;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                soff[e] = run;
+                if (writer) offsets[e] = run;
+            }
+            run += kp_local[i];
+        }
+        for (int o = 16; o >= 1; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+        if (writer && lane == 31) offsets[E] = incl;
+        if (writer && lane == 0 && n_dropped) *n_dropped = dsum;
+    }
+    __syncthreads();
+    if (live) {
+        for (int k = 0; k < K; ++k) {
+            const int e = my[k];
+            int r = pre[k];
+            for (int w2 = 0; w2 < warp; ++w2) r += wh[w2 * E + e];
+            const int row = (C < 0 || r < C) ? soff[e] + r : -1;
+            srow[t * K + k] = row;
+            if (writer) {
+                inv[t * K + k] = row;
+                if (row >= 0) src[row] = t;
+            }
+        }
+    }
+    __syncthreads();
+    // gather: job (token, slice) j = blockIdx.x + gridDim.x * (warp + W * i)
+    const int nvec = d / 8;
+    const int slice = (nvec + parts - 1) / parts;
+    const int jobs = T * parts;
+    for (int job = blockIdx.x + gridDim.x * warp; job < jobs; job += gridDim.x * W) {
+        const int tt = job / parts;
+        const int p = job - tt * parts;
+        const uint4* sx = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(tt) * d);
+        const int c_end = min(nvec, (p + 1) * slice);
+        for (int c0 = p * slice + lane; c0 < c_end; c0 += 32 * kGatherBatch) {
+            uint4 v[kGatherBatch];
+#pragma unroll
+            for (int b = 0; b < kGatherBatch; ++b) {
+                const int c = c0 + 32 * b;
+                if (c < c_end) v[b] = __ldg(sx + c);
+            }
+            for (int k = 0; k < K; ++k) {
+                const int row = srow[tt * K + k];
+                if (row < 0) continue;
+                uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(row) * d);
+#pragma unroll
+                for (int b = 0; b < kGatherBatch; ++b) {
+                    const int c = c0 + 32 * b;
+                    if (c < c_end) dst[c] = v[b];
+                }
+            }
+        }
+    }
+}
+
 }  // namespace
 
 int permute_blocks(int64_t T) { return static_cast<int>((T + kTokPerBlock - 1) / kTokPerBlock); }
@@ -325,6 +451,35 @@ int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, i
 }
 
 int launch_count(int64_t T) { return T <= kSmallT ? 1 : 3; }
+
+bool dispatch_gather_fused_supported(int64_t T, int E, int K) { return T <= kSmallT && E <= kMaxE && K <= kMaxK; }
+
+int launch_dispatch_gather_small(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
+                                 int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
+                                 bf16* x_perm, int32_t* n_dropped, int32_t* zero_out, int zero_count,
+                                 cudaStream_t st) {
+    if (!dispatch_gather_fused_supported(T, E, K) || !x || !x_perm || d % 8 != 0) return -2;
+    const size_t smem = static_cast<size_t>(3 * (kSmallThreads / 32) * E + E + 1 + T * K) * 4;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(dispatch_gather_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1 + kSmallT * kMaxK) * 4) !=
+            cudaSuccess)
+            return -3;
+        attr = true;
+    }
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    // (token, slice) jobs: enough for every warp of the grid
+    int parts = 1;
+    while (parts < 16 && T * parts < static_cast<int64_t>(sms) * 32 && (d / 8) / (parts * 2) >= 32) parts *= 2;
+    const int64_t jobs = T * parts;
+    const int64_t need = (jobs + (kSmallThreads / 32) - 1) / (kSmallThreads / 32);
+    const int grid = static_cast<int>(need < sms ? (need < 1 ? 1 : need) : sms);
+    (void)launch_pdl(dispatch_gather_small_kernel, dim3(grid), dim3(kSmallThreads), smem, st, idx, x,
+                     static_cast<int>(T), d, E, K, C, parts, counts, kept, offsets, inv, src, n_dropped, x_perm,
+                     zero_out, zero_count);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
 
 // ------------------------------------------------------------------------
 // Dispatch without a caller-provided workspace.

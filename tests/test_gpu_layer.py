@@ -74,7 +74,7 @@ def test_layer_tiny_full():
 
 @pytest.mark.parametrize("name,T,ntok", [
     ("mixtral_decode", 256, 24), ("mixtral_decode", 37, 37), ("mixtral_prefill", 1500, 24),
-    ("qwen_capacity", 2000, 48), ("deepseek_bias", 600, 12)])
+    ("qwen_capacity", 2000, 48), ("qwen_capacity", 700, 32), ("deepseek_bias", 600, 12)])
 def test_layer_reduced_T(name, T, ntok):
     inp = LayerInputs(synth.get_workload(name), T=T)
     bias = None
