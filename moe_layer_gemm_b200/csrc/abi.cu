@@ -169,7 +169,11 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
         g.dense_rows = d->T;
         g.max_group_rows = d->T;
         g.swap_max_rows = 0;
-        g.bn_max = 64;  // narrow tiles: more CTAs share the logits GEMM (N = E_pad is small)
+        // narrow tiles: more CTAs share the logits GEMM (N = E_pad is small);
+        // 32-wide when 64-wide tiles would leave over half the SMs idle
+        const int64_t row_tiles = (d->T + 127) / 128;
+        const int sms = num_sms() > 0 ? num_sms() : 148;
+        g.bn_max = row_tiles * (L.E_pad / 64) < sms / 2 ? 32 : 64;
         g.nphase = 1;
         g.ph[0].tok = x;
         g.ph[0].tok_rows = d->T;

@@ -635,13 +635,8 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         if (!make_map(&maps.tokB[p], g.tok, tok_rows, g.Kdim, 32u)) return -3;
     }
 
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
-            return -3;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (smem_attr_once(reinterpret_cast<const void*>(grouped_gemm_kernel), 227 * 1024, attr_done) != 0) return -3;
     const int sms = num_sms();
     if (sms <= 0) return -3;
     // Upper bound on the tile count, to avoid idle CTAs on tiny problems.

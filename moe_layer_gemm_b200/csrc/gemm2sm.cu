@@ -647,13 +647,8 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     if (stages < 2) return -2;
     a.stages = stages;
     const size_t smem = fixed + static_cast<size_t>(stages) * stage_bytes;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
-            return -3;
-        attr = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (smem_attr_once(reinterpret_cast<const void*>(grouped_gemm_2sm_kernel), 227 * 1024, attr_done) != 0) return -3;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * clusters, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 namespace moe {
 
 using bf16 = __nv_bfloat16;
@@ -16,6 +18,19 @@ enum GemmEpilogue : int {
 };
 
 // One matrix product over all groups: out[rows of g] = tok[rows of g] . w[g]^T.
+// Raise `func`'s dynamic shared memory limit to `bytes` on the current device,
+// once per device (`done` holds one bit per device id < 64).  0, or -3 when
+// the runtime refuses.
+inline int smem_attr_once(const void* func, int bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -3;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return 0;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return -3;
+    if (bit) done.fetch_or(bit, std::memory_order_release);
+    return 0;
+}
+
 // Launch `kernel` with programmatic stream serialization: it may begin
 // while the previous kernel on `st` drains, so it must call pdl_wait()
 // before using that kernel's results (see ptx.cuh).

@@ -421,13 +421,10 @@ int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, i
     if (E > kMaxE || K > kMaxK) return -2;
     if (T <= kSmallT) {
         const size_t smem = static_cast<size_t>(3 * (kSmallThreads / 32) * E + E + 1) * 4;
-        static bool attr = false;
-        if (!attr) {
-            if (cudaFuncSetAttribute(dispatch_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1) * 4) != cudaSuccess)
-                return -3;
-            attr = true;
-        }
+        static std::atomic<unsigned long long> attr_done{0};
+        if (smem_attr_once(reinterpret_cast<const void*>(dispatch_small_kernel),
+                           (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1) * 4, attr_done) != 0)
+            return -3;
         dispatch_small_kernel<<<1, kSmallThreads, smem, st>>>(idx, static_cast<int>(T), E, K, C, counts, kept,
                                                               offsets, inv, src, n_dropped, zero_out, zero_count);
     } else {
@@ -460,14 +457,10 @@ int launch_dispatch_gather_small(const int32_t* idx, const bf16* x, int64_t T, i
                                  cudaStream_t st) {
     if (!dispatch_gather_fused_supported(T, E, K) || !x || !x_perm || d % 8 != 0) return -2;
     const size_t smem = static_cast<size_t>(3 * (kSmallThreads / 32) * E + E + 1 + T * K) * 4;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(dispatch_gather_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1 + kSmallT * kMaxK) * 4) !=
-            cudaSuccess)
-            return -3;
-        attr = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (smem_attr_once(reinterpret_cast<const void*>(dispatch_gather_small_kernel),
+                       (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1 + kSmallT * kMaxK) * 4, attr_done) != 0)
+        return -3;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     // (token, slice) jobs: enough for every warp of the grid
     int parts = 1;

@@ -437,13 +437,8 @@ int route_fused_supported(int d, int E) {
 template <int EV>
 int launch_fused_ev(const bf16* x, const bf16* Wr, const float* bias, int64_t T, int d, int E, int K, float* logits,
                     int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(route_fused_kernel<EV>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
-            cudaSuccess)
-            return -3;
-        attr = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (smem_attr_once(reinterpret_cast<const void*>(route_fused_kernel<EV>), 96 * 1024, attr_done) != 0) return -3;
     const size_t smem = static_cast<size_t>(d) * EV * 8 * 2;
     (void)launch_pdl(route_fused_kernel<EV>, dim3(nblocks), dim3(kRouteWarps * 32), smem, st, x, Wr, bias, T, d, E, K, logits, idx, w, prob_part);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
