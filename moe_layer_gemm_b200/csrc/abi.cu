@@ -361,6 +361,11 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x
     if (x && (!aligned16(x) || !aligned16(x_perm))) return MOE_EUNSUPPORTED;
     MOE_TRY(check_ws(dims, ws, ws_bytes));
     const Layout L = layout_of(dims);
+    if (x && dispatch_gather_fused_supported(dims->T, dims->E, dims->K))  // small batch: one launch
+        return map_launch(launch_dispatch_gather_small(
+            topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
+            counts, kept, offsets, inv, src, reinterpret_cast<bf16*>(x_perm), n_dropped, at<int32_t>(ws, L.sched_ffn),
+            static_cast<int>(gemm_sched_bytes(dims->E) / 4), static_cast<cudaStream_t>(stream)));
     return map_launch(launch_permute(topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model, dims->E,
                                      dims->K, capacity_of(dims), at<int32_t>(ws, L.block_hist), counts, kept,
                                      offsets, inv, src, reinterpret_cast<bf16*>(x_perm), n_dropped,

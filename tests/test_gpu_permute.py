@@ -13,7 +13,9 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("T,E,K,cf,skew", [
     (1, 1, 1, 0.0, 0.0), (1000, 8, 2, 0.0, 0.0), (1000, 8, 2, 1.0, 1.5), (8192, 60, 4, 1.0, 2.0),
     (4096, 256, 8, 0.0, 1.1), (300, 3, 3, 0.5, 0.0), (2049, 16, 16, 1.25, 0.5), (257, 5, 2, 0.0625, 0.0),
-    (16384, 8, 2, 0.0, 0.3)])
+    (16384, 8, 2, 0.0, 0.3),
+    # batches of at most 1024 tokens with a gather take the one-launch dispatch
+    (1024, 256, 16, 0.0, 0.7), (1024, 256, 16, 0.5, 1.0), (513, 33, 7, 0.9, 0.4)])
 def test_permute_bitexact(T, E, K, cf, skew):
     d = dev()
     wts = None
