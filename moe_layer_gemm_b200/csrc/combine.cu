@@ -78,9 +78,12 @@ __device__ void stats_tail(const StatsTail& s, int64_t T, int K) {
 }
 
 // S >= nsplit slots for partial slices (S == nsplit except the 8-slot
-// fallback, which reads only the nsplit slices that exist).
+// fallback, which reads only the nsplit slices that exist).  Slots are
+// handled in groups of G, whose G x S loads are all in flight at once; G
+// shrinks as slices grow so the registers, and with them the resident
+// CTAs, stay put (more loads per thread measured slower at K = 4).
 template <int S>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, S == 1 ? 8 : (S >= 8 ? 2 : 4))  // one slice: 32 registers, 8 CTAs per SM
 combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, const int32_t* __restrict__ inv,
                const float* __restrict__ w, int64_t T, int d, int K, float* __restrict__ y, const StatsTail tail) {
     pdl_trigger();
@@ -93,22 +96,25 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
     }
     const int nvec = d / 4;
     const int64_t svec = split_stride / 4;
+    // the token's rows and weights, read once per CTA
+    __shared__ int32_t rows[kMaxK];
+    __shared__ float ws[kMaxK];
     for (int64_t t = blockIdx.x; t < T; t += ntok_blocks) {
-        int32_t rows[kMaxK];
-        float ws[kMaxK];
-        for (int k = 0; k < K; ++k) {
-            rows[k] = inv[t * K + k];
-            ws[k] = w[t * K + k];
+        if (static_cast<int>(threadIdx.x) < K) {
+            rows[threadIdx.x] = inv[t * K + threadIdx.x];
+            ws[threadIdx.x] = w[t * K + threadIdx.x];
         }
+        __syncthreads();
         for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            // slots in groups of four: a group's loads are all issued before
-            // its arithmetic; slices are summed in slice order and slots
+            // slots in groups of G: a group's loads are all issued before its
+            // arithmetic; slices are summed in slice order and slots
             // accumulated in slot order
-            for (int k0 = 0; k0 < K; k0 += 4) {
-                float4 v[4][S];
+            constexpr int G = S >= 4 ? 2 : 4;
+            for (int k0 = 0; k0 < K; k0 += G) {
+                float4 v[G][S];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < G; ++j) {
                     const int k = k0 + j;
                     const bool live = k < K && rows[k] >= 0;
                     const float4* base =
@@ -118,7 +124,7 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
                         v[j][sl] = (live && sl < nsplit) ? __ldg(base + sl * svec) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < G; ++j) {
                     const int k = k0 + j;
                     if (k < K && rows[k] >= 0) {
                         float4 u = v[j][0];
@@ -136,6 +142,7 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
             }
             reinterpret_cast<float4*>(y + t * d)[c] = acc;
         }
+        __syncthreads();  // rows / ws are rewritten for the next token
     }
 }
 
