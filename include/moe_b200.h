@@ -253,12 +253,14 @@ typedef struct moe_layer_outputs {
 /* Which grouped-GEMM kernel moe_expert_ffn and moe_layer_forward launch for
  * these dims: 0 = single-CTA tiles (grouped_gemm_kernel), 1 = CTA-pair tiles
  * on tcgen05 cta_group::2 (grouped_gemm_2sm_kernel).  The choice depends on
- * the shape only.  Host only, no CUDA call; MOE_EINVAL on bad dims. */
+ * the shape only.  Host only (at most a query of the current device's SM
+ * count); MOE_EINVAL on bad dims. */
 MOE_API int moe_ffn_kernel(const moe_dims* dims);
 
 /* Number of kernel launches one moe_layer_forward call enqueues for these
  * dims and options (stats = P_i / f_i / aux requested, bias_update = bias
- * non-NULL and alpha != 0).  Host only; < 0 on bad dims. */
+ * non-NULL and alpha != 0; neither adds a launch, both run in one extra CTA
+ * of the combine launch).  Host only; < 0 on bad dims. */
 MOE_API int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_update);
 
 /* The whole layer: route -> permute -> expert FFN -> combine (-> stats, bias

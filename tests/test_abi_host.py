@@ -115,3 +115,14 @@ def test_ffn_kernel_choice_by_shape(lib):
     bad = abi.Dims(0, 4096, 14336, 8, 2)
     with pytest.raises(abi.MoEError):
         abi.moe_ffn_kernel(bad)
+
+
+def test_layer_launch_counts(lib):
+    # decode: fused router, one-launch dispatch + gather, both GEMMs, combine (+ statistics tail)
+    assert abi.moe_layer_launch_count(abi.Dims(256, 4096, 14336, 8, 2), True, False) == 4
+    # statistics and the bias update add no launch
+    assert abi.moe_layer_launch_count(abi.Dims(256, 4096, 14336, 8, 2), True, True) == 4
+    # prefill: fused router, hist / scan / rank + gather, GEMMs, combine
+    assert abi.moe_layer_launch_count(abi.Dims(16384, 4096, 14336, 8, 2), True, False) == 7
+    # E > 32: transpose + logits GEMM + top-K router; DeepSeek-like T = 4096 > 1024
+    assert abi.moe_layer_launch_count(abi.Dims(4096, 7168, 2048, 256, 8), True, True) == 9
