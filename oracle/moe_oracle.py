@@ -141,6 +141,40 @@ def load_stats(counts: np.ndarray, probs: np.ndarray, T: int, K: int):
     return f, P, aux
 
 
+def router_z_loss(logits: np.ndarray) -> float:
+    """z_loss = (1/T) sum_t (log sum_j exp(s_tj))^2, in fp64.
+
+    [P2] section 3.2 (router z-loss: it keeps the router logits small by
+    penalising the square of their log-sum-exp, averaged over the tokens).
+    READING: s are the unbiased router logits x W_r, the same ones P_i uses;
+    the aux-free bias is a routing adjustment, not router output.
+    """
+    s = np.asarray(logits, dtype=np.float64)
+    m = s.max(axis=1)
+    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    return float(np.mean(lse * lse))
+
+
+def topk_load_stats(counts: np.ndarray, idx: np.ndarray, w: np.ndarray, T: int, K: int):
+    """(P_topk, aux_topk): the cheaper form of the balance loss that counts
+    only the probabilities of the selected experts.
+
+    [P2] section 3.2 (an approximate aux loss that sums only the top-K
+    selected probabilities instead of the soft assignment over all experts).
+    READING: P~_i = (1/T) * sum over (t, k) with idx[t, k] = i of w[t, k],
+    the renormalised top-K weights the router emits; aux_topk =
+    N * sum_i f_i P~_i with f_i as in load_stats.
+    """
+    E = counts.shape[0]
+    f = np.asarray(counts, dtype=np.float64) / float(T * K)
+    Pt = np.zeros(E)
+    for t in range(idx.shape[0]):
+        for k in range(idx.shape[1]):
+            Pt[int(idx[t, k])] += float(w[t, k])
+    Pt /= float(T)
+    return Pt, float(E) * float(np.sum(f * Pt))
+
+
 # ---------------------------------------------------------------------------
 # a4. Dispatch with capacity
 # ---------------------------------------------------------------------------
@@ -301,7 +335,8 @@ def moe_layer(x, Wr, W1, W3, W2, K, capacity_factor=0.0, bias32=None, alpha=0.0,
     ``tokens`` restricts the FFN/combine to those token ids (routing, counts
     and capacity still use all T tokens); y rows of other tokens are NaN.
 
-    Returns a dict with logits (fp64), idx, w, counts, f, P, aux, dispatch
+    Returns a dict with logits (fp64), idx, w, counts, f, P, aux, P_topk,
+    aux_topk, z_loss, dispatch
     fields, y_perm (expert-grouped FFN rows), y [T,d] fp64 and the updated
     bias.
     """
@@ -314,6 +349,8 @@ def moe_layer(x, Wr, W1, W3, W2, K, capacity_factor=0.0, bias32=None, alpha=0.0,
     probs = softmax_rows(l64)                               # a3 (unbiased)
     cnt = expert_counts(idx, E)
     f, P, aux = load_stats(cnt, probs, T, K)
+    P_topk, aux_topk = topk_load_stats(cnt, idx, w, T, K)
+    z_loss = router_z_loss(l64)
     C = capacity(T, K, E, capacity_factor)                  # a4
     disp = dispatch(idx, E, C)
     want = np.ones(T, dtype=bool)
@@ -331,7 +368,8 @@ def moe_layer(x, Wr, W1, W3, W2, K, capacity_factor=0.0, bias32=None, alpha=0.0,
     new_bias = None
     if bias32 is not None:
         new_bias = bias_update(bias32, cnt, T, K, alpha)    # a7
-    out = dict(logits=l64, logits32=l32, idx=idx, w=w, counts=cnt, f=f, P=P, aux=aux,
+    out = dict(logits=l64, logits32=l32, idx=idx, w=w, counts=cnt, f=f, P=P, aux=aux, P_topk=P_topk,
+               aux_topk=aux_topk, z_loss=z_loss,
                capacity=C, y=y, y_perm=Yp, bias=new_bias)
     out.update({k: v for k, v in disp.items() if k != "counts"})
     return out

@@ -149,6 +149,51 @@ def test_aux_loss_uniform_cases():
     assert abs(O.load_stats(cnt, probs, T, K)[2] - E) < 1e-15
 
 
+def test_router_z_loss_closed_forms():
+    T, E = 5, 6
+    # all logits 0: log-sum-exp = log E for every token
+    assert abs(O.router_z_loss(np.zeros((T, E))) - math.log(E) ** 2) < 1e-15
+    # all logits c: log-sum-exp = c + log E
+    for c in (-3.5, 0.25, 7.0):
+        assert abs(O.router_z_loss(np.full((T, E), c)) - (c + math.log(E)) ** 2) < 1e-12
+    # two experts: log(e^a + e^b) = max + log1p(e^-|a-b|), token by token
+    ab = np.array([[1.0, -2.0], [0.5, 0.5], [-4.0, 3.0]])
+    want = np.mean([(max(a, b) + math.log1p(math.exp(-abs(a - b)))) ** 2 for a, b in ab])
+    assert abs(O.router_z_loss(ab) - want) < 1e-14
+    # one dominant logit (others 60 below it): log-sum-exp -> that logit
+    s = np.zeros((3, 4)); s[:, 1] = 60.0
+    assert abs(O.router_z_loss(s) - 3600.0) < 1e-9
+    # large logits do not overflow (shifted by the row max)
+    s = np.array([[800.0, 799.0, 0.0]])
+    assert abs(O.router_z_loss(s) - (800.0 + math.log1p(math.exp(-1.0))) ** 2) < 1e-9
+
+
+def test_topk_aux_loss_cases():
+    r = _rng(8)
+    T, E = 40, 6
+    logits = r.standard_normal((T, E))
+    # K = 1: the single weight is 1, so P~ = f and aux_topk = E * sum f^2
+    idx, w, _ = O.route_from_logits_f32(logits.astype(np.float32), 1)
+    cnt = O.expert_counts(idx, E)
+    Pt, at = O.topk_load_stats(cnt, idx, w, T, 1)
+    f = cnt / float(T)
+    assert np.allclose(Pt, f, atol=1e-15) and abs(at - E * np.sum(f * f)) < 1e-13
+    # K = E without bias: the renormalised weights are the full softmax, so
+    # P~ equals the full-softmax P_i and aux_topk equals aux
+    idx, w, _ = O.route_from_logits_f32(logits.astype(np.float32), E)
+    cnt = O.expert_counts(idx, E)
+    Pt, at = O.topk_load_stats(cnt, idx, w, T, E)
+    f, P, aux = O.load_stats(cnt, O.softmax_rows(logits.astype(np.float32).astype(np.float64)), T, E)
+    assert np.allclose(Pt, P, atol=1e-7) and abs(at - aux) < 1e-7
+    # any K: the weights of a token sum to 1, so sum_i P~_i = 1; uniform f gives 1
+    for K in (2, 3):
+        idx, w, _ = O.route_from_logits_f32(logits.astype(np.float32), K)
+        cnt = O.expert_counts(idx, E)
+        Pt, _ = O.topk_load_stats(cnt, idx, w, T, K)
+        assert abs(Pt.sum() - 1.0) < 1e-12
+        assert abs(float(E) * np.sum(np.full(E, 1.0 / E) * Pt) - 1.0) < 1e-12
+
+
 # ------------------------------------------------------------- a4 dispatch
 
 def test_capacity_values():
