@@ -246,6 +246,15 @@ typedef struct moe_layer_outputs {
      * update (these run in one extra CTA of the combine launch, so [4] and
      * [5] mark the same point).  For per-stage timing. */
     void* const* stage_events; /* [MOE_NUM_STAGE_EVENTS] */
+    /* Further router statistics ([P2] section 3.2), computed with P_i:
+     * P_topk[i] = (1/T) * sum of the renormalised top-K weights w[t,k] of
+     * the slots that chose expert i (the cheaper balance statistic that
+     * counts only the selected experts' probabilities); aux_topk =
+     * E * sum_i f_i P_topk[i]; z_loss = (1/T) * sum_t (log sum_e
+     * exp(logits[t,e]))^2 over the unbiased logits (router z-loss). */
+    float* P_topk;      /* [E] */
+    float* aux_topk;    /* [1] */
+    float* z_loss;      /* [1] */
 } moe_layer_outputs;
 
 #define MOE_NUM_STAGE_EVENTS 6

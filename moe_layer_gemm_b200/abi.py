@@ -50,7 +50,7 @@ class moe_dims(ctypes.Structure):
 class moe_layer_outputs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("topk_idx", "topk_w", "logits", "counts", "kept", "offsets", "inv", "n_dropped", "f", "P", "aux",
-                 "stage_events")]
+                 "stage_events", "P_topk", "aux_topk", "z_loss")]
 
 
 _lib = None

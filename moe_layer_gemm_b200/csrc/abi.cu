@@ -115,7 +115,7 @@ Layout layout_of(const moe_dims* d) {
     L.kept = take(E * 4);
     L.offsets = take((E + 1) * 4);
     L.ndrop = take(4);
-    L.prob_part = take(static_cast<size_t>(L.route_nb) * E * 4);
+    L.prob_part = take(static_cast<size_t>(L.route_nb) * (2 * E + 1) * 4);  // router statistics rows
     L.prob_mean = take(E * 4);
     L.f = take(E * 4);
     L.aux = take(4);
@@ -454,7 +454,7 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
     int32_t* offsets = o.offsets ? o.offsets : at<int32_t>(ws, L.offsets);
     int32_t* inv = o.inv ? o.inv : at<int32_t>(ws, L.inv);
     int32_t* ndrop = o.n_dropped ? o.n_dropped : at<int32_t>(ws, L.ndrop);
-    const bool want_stats = o.P || o.aux || o.f;
+    const bool want_stats = o.P || o.aux || o.f || o.P_topk || o.aux_topk || o.z_loss;
     float* P = o.P ? o.P : at<float>(ws, L.prob_mean);
     const bf16* xb = reinterpret_cast<const bf16*>(x);
 
@@ -492,6 +492,9 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
             tail.P = P;
             tail.f = o.f;
             tail.aux = o.aux;
+            tail.P_topk = o.P_topk;
+            tail.aux_topk = o.aux_topk;
+            tail.z_loss = o.z_loss;
         }
         if (bias && alpha != 0.0f) {
             tail.bias = bias;

@@ -33,23 +33,32 @@ __device__ __forceinline__ float warp_sum_fixed(float x) {
 
 // The statistics tail (one CTA of any multiple of 32 threads): warp w
 // reduces experts w, w + nw, ...: lane l adds router blocks l, l + 32, ...
-// in order, then a fixed butterfly; P_i = sum / T, f_i = counts_i / (T K);
-// aux = E * sum_i f_i P_i summed per warp in expert order, then over warps
-// in warp order.  Then the bias update, one expert per thread.  Every sum
+// in order, then a fixed butterfly; P_i = sum / T, f_i = counts_i / (T K),
+// P~_i (top-K weights) likewise; aux = E * sum_i f_i P_i and aux_topk =
+// E * sum_i f_i P~_i summed per warp in expert order, then over warps in
+// warp order; z_loss = (sum of the blocks' squared log-sum-exp sums: lane l
+// adds blocks l, l + 32, ..., then the fixed butterfly) / T.  Then the bias update, one expert per thread.  Every sum
 // has a fixed order, so results are reproducible.
+// Column `col` of the router statistics rows summed over the blocks: lane l
+// adds blocks l, l + 32, ... in order, then the fixed butterfly.
+__device__ __forceinline__ float sum_column(const float* part, int64_t row, int col, int nblocks, int lane) {
+    float v = 0.f;
+    for (int b = lane; b < nblocks; b += 32) v += part[b * row + col];
+    return warp_sum_fixed(v);
+}
+
 __device__ void stats_tail(const StatsTail& s, int64_t T, int K) {
-    __shared__ float red[32];
+    __shared__ float red[2][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int E = s.E;
+    const int64_t row = 2 * static_cast<int64_t>(E) + 1;
     if (s.part) {
         const float invT = 1.0f / static_cast<float>(T);
         const float invA = 1.0f / static_cast<float>(T * K);
+        // P_i, f_i and their products (one pass), then P~_i (a second pass)
         float acc = 0.f;
         for (int e = warp; e < E; e += nw) {
-            float sum = 0.f;
-            for (int b = lane; b < s.nblocks; b += 32) sum += s.part[static_cast<int64_t>(b) * E + e];
-            sum = warp_sum_fixed(sum);
-            const float pe = sum * invT;
+            const float pe = sum_column(s.part, row, e, s.nblocks, lane) * invT;
             const float fe = static_cast<float>(s.counts[e]) * invA;
             if (lane == 0) {
                 s.P[e] = pe;
@@ -57,12 +66,32 @@ __device__ void stats_tail(const StatsTail& s, int64_t T, int K) {
                 acc += fe * pe;
             }
         }
-        if (lane == 0) red[warp] = acc;
+        float acc_t = 0.f;
+        if (s.P_topk || s.aux_topk)
+            for (int e = warp; e < E; e += nw) {
+                const float pte = sum_column(s.part, row, E + e, s.nblocks, lane) * invT;
+                if (lane == 0) {
+                    if (s.P_topk) s.P_topk[e] = pte;
+                    acc_t += static_cast<float>(s.counts[e]) * invA * pte;
+                }
+            }
+        if (lane == 0) {
+            red[0][warp] = acc;
+            red[1][warp] = acc_t;
+        }
         __syncthreads();
-        if (threadIdx.x == 0 && s.aux) {
-            float a = 0.f;
-            for (int i = 0; i < nw; ++i) a += red[i];
-            *s.aux = static_cast<float>(E) * a;
+        if (warp == 0) {
+            const float z = s.z_loss ? sum_column(s.part, row, 2 * E, s.nblocks, lane) : 0.f;
+            if (lane == 0) {
+                float a = 0.f, at = 0.f;
+                for (int i = 0; i < nw; ++i) {
+                    a += red[0][i];
+                    at += red[1][i];
+                }
+                if (s.aux) *s.aux = static_cast<float>(E) * a;
+                if (s.aux_topk) *s.aux_topk = static_cast<float>(E) * at;
+                if (s.z_loss) *s.z_loss = z * invT;
+            }
         }
     }
     if (s.bias && s.alpha != 0.0f) {

@@ -115,12 +115,16 @@ int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, i
 // update.  Both need only routing results, which are complete when the
 // combine starts.
 struct StatsTail {
-    const float* part;      // router per-block probability sums [nblocks, E]; nullptr: no statistics
+    const float* part;      // router per-block rows [nblocks, 2 E + 1]: probability sums, top-K weight
+                            // sums, squared log-sum-exp sum; nullptr: no statistics
     int nblocks;
     const int32_t* counts;  // nullptr: no tail CTA at all
     float* P;               // required with part
     float* f;               // may be nullptr
     float* aux;             // may be nullptr
+    float* P_topk;          // may be nullptr
+    float* aux_topk;        // may be nullptr
+    float* z_loss;          // may be nullptr
     float* bias;            // updated in place when non-null and alpha != 0
     float alpha;
     int E;

@@ -92,12 +92,15 @@ __device__ __forceinline__ float warp_max(float x) {
     return x;
 }
 
-// Selection, weights and probability accumulation for one token whose
-// unbiased logits are l[j] (expert lane + 32 j).
+// Selection, weights and statistics for one token whose unbiased logits are
+// l[j] (expert lane + 32 j).  With want_prob, psum[j] accumulates the full
+// softmax probability of expert lane + 32 j, tsum[j] its renormalised top-K
+// weight when selected, and lane 0's zsum the squared log-sum-exp of the
+// unbiased logits (the router z-loss term).
 template <int J>
 __device__ __forceinline__ void finish_token(const float (&l)[J], const bool (&valid)[J], const float* bias,
                                              int64_t t, int K, int lane, int32_t* idx, float* w,
-                                             float (&psum)[J], bool want_prob) {
+                                             float (&psum)[J], float (&tsum)[J], float& zsum, bool want_prob) {
     if (want_prob) {
         float m = -FLT_MAX;
 #pragma unroll
@@ -115,6 +118,10 @@ __device__ __forceinline__ void finish_token(const float (&l)[J], const bool (&v
         const float inv = 1.0f / s;
 #pragma unroll
         for (int j = 0; j < J; ++j) psum[j] += p[j] * inv;
+        if (lane == 0) {
+            const float lse = m + logf(s);
+            zsum += lse * lse;
+        }
     }
     float lb[J];
 #pragma unroll
@@ -125,23 +132,51 @@ __device__ __forceinline__ void finish_token(const float (&l)[J], const bool (&v
     const float vmax = __shfl_sync(0xffffffffu, sv, 0);
     const float ex = (lane < K) ? expf(sv - vmax) : 0.f;
     const float den = warp_sum(ex);
+    const float wk = ex / den;
     if (lane < K) {
         idx[t * K + lane] = se;
-        w[t * K + lane] = ex / den;
+        w[t * K + lane] = wk;
     }
+    if (want_prob)
+        for (int r = 0; r < K; ++r) {  // slot r's weight goes to the lane that owns its expert
+            const int er = __shfl_sync(0xffffffffu, se, r);
+            const float wr = __shfl_sync(0xffffffffu, wk, r);
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+                if (er == lane + 32 * j) tsum[j] += wr;
+        }
 }
 
+// One row of 2 E + 1 floats per CTA: [probability sums | top-K weight sums |
+// squared log-sum-exp sum], each summed over the CTA's warps in warp order.
 template <int J>
-__device__ __forceinline__ void write_prob_partials(const float (&psum)[J], int E, float* prob_part) {
+__device__ __forceinline__ void write_prob_partials(const float (&psum)[J], const float (&tsum)[J], float zsum,
+                                                    int E, float* prob_part) {
     __shared__ float sp[kRouteWarps][J * 32];
+    __shared__ float st[kRouteWarps][J * 32];
+    __shared__ float sz[kRouteWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-    for (int j = 0; j < J; ++j) sp[warp][lane + 32 * j] = psum[j];
+    for (int j = 0; j < J; ++j) {
+        sp[warp][lane + 32 * j] = psum[j];
+        st[warp][lane + 32 * j] = tsum[j];
+    }
+    if (lane == 0) sz[warp] = zsum;
     __syncthreads();
+    float* row = prob_part + static_cast<int64_t>(blockIdx.x) * (2 * E + 1);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        float s = 0.f;
-        for (int wi = 0; wi < kRouteWarps; ++wi) s += sp[wi][e];
-        prob_part[static_cast<int64_t>(blockIdx.x) * E + e] = s;
+        float s = 0.f, u = 0.f;
+        for (int wi = 0; wi < kRouteWarps; ++wi) {
+            s += sp[wi][e];
+            u += st[wi][e];
+        }
+        row[e] = s;
+        row[E + e] = u;
+    }
+    if (threadIdx.x == 0) {
+        float z = 0.f;
+        for (int wi = 0; wi < kRouteWarps; ++wi) z += sz[wi];
+        row[2 * E] = z;
     }
 }
 
@@ -183,7 +218,7 @@ route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kRouteWarps;
-    float psum[1] = {0.f};
+    float psum[1] = {0.f}, tsum[1] = {0.f}, zsum = 0.f;
     const bool want_prob = prob_part != nullptr;
     const int nvec = d / 8;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps + warp; t < T; t += nwarps) {
@@ -233,9 +268,9 @@ route_fused_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
             if (e == lane) l[0] = acc[e];
         bool valid[1] = {lane < E};
         if (logits != nullptr && valid[0]) logits[t * E + lane] = l[0];
-        finish_token<1>(l, valid, bias, t, K, lane, idx, w, psum, want_prob);
+        finish_token<1>(l, valid, bias, t, K, lane, idx, w, psum, tsum, zsum, want_prob);
     }
-    if (want_prob) write_prob_partials<1>(psum, E, prob_part);
+    if (want_prob) write_prob_partials<1>(psum, tsum, zsum, E, prob_part);
 }
 
 // Small batches (decode): one CTA per token, its hidden dimension split
@@ -351,8 +386,16 @@ route_split_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
             bool valid[1] = {lane < E};
             if (logits != nullptr && valid[0]) logits[t * E + lane] = l[0];
             float psum[1] = {0.f};
-            finish_token<1>(l, valid, bias, t, K, lane, idx, w, psum, prob_part != nullptr);
-            if (prob_part != nullptr && lane < E) prob_part[t * E + lane] = psum[0];
+            float tsum[1] = {0.f}, zsum = 0.f;
+            finish_token<1>(l, valid, bias, t, K, lane, idx, w, psum, tsum, zsum, prob_part != nullptr);
+            if (prob_part != nullptr) {  // one statistics row per token (see write_prob_partials)
+                float* row = prob_part + t * (2 * E + 1);
+                if (lane < E) {
+                    row[lane] = psum[0];
+                    row[E + lane] = tsum[0];
+                }
+                if (lane == 0) row[2 * E] = zsum;
+            }
         }
         __syncthreads();
     }
@@ -366,9 +409,9 @@ topk_from_logits_kernel(const float* __restrict__ logits, const float* __restric
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kRouteWarps;
-    float psum[J];
+    float psum[J], tsum[J], zsum = 0.f;
 #pragma unroll
-    for (int j = 0; j < J; ++j) psum[j] = 0.f;
+    for (int j = 0; j < J; ++j) psum[j] = tsum[j] = 0.f;
     const bool want_prob = prob_part != nullptr;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps + warp; t < T; t += nwarps) {
         float l[J];
@@ -379,13 +422,14 @@ topk_from_logits_kernel(const float* __restrict__ logits, const float* __restric
             valid[j] = e < E;
             l[j] = valid[j] ? logits[t * E + e] : -FLT_MAX;
         }
-        finish_token<J>(l, valid, bias, t, K, lane, idx, w, psum, want_prob);
+        finish_token<J>(l, valid, bias, t, K, lane, idx, w, psum, tsum, zsum, want_prob);
     }
-    if (want_prob) write_prob_partials<J>(psum, E, prob_part);
+    if (want_prob) write_prob_partials<J>(psum, tsum, zsum, E, prob_part);
 }
 
 // P_i: warp w reduces experts w, w+32, ...: lane l adds router blocks l,
-// l+32, ... in order, then a fixed butterfly (reproducible).
+// l+32, ... in order, then a fixed butterfly (reproducible).  Block rows are
+// 2 E + 1 floats wide (write_prob_partials); P's sums are the first E.
 __global__ void __launch_bounds__(1024)
 prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float invT, float* __restrict__ out) {
     pdl_trigger();
@@ -393,7 +437,7 @@ prob_finalize_kernel(const float* __restrict__ part, int nblocks, int E, float i
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int e = warp; e < E; e += nw) {
         float s = 0.f;
-        for (int b = lane; b < nblocks; b += 32) s += part[static_cast<int64_t>(b) * E + e];
+        for (int b = lane; b < nblocks; b += 32) s += part[static_cast<int64_t>(b) * (2 * E + 1) + e];
         s = warp_sum(s);
         if (lane == 0) out[e] = s * invT;
     }

@@ -126,3 +126,11 @@ def test_layer_launch_counts(lib):
     assert abi.moe_layer_launch_count(abi.Dims(16384, 4096, 14336, 8, 2), True, False) == 7
     # E > 32: transpose + logits GEMM + top-K router; DeepSeek-like T = 4096 > 1024
     assert abi.moe_layer_launch_count(abi.Dims(4096, 7168, 2048, 256, 8), True, True) == 9
+
+
+def test_layer_outputs_struct_matches_header():
+    src = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    body = src[src.index("typedef struct moe_layer_outputs {"):src.index("} moe_layer_outputs;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\*\s*(\w+)\s*;", body)
+    assert names == [n for n, _ in abi.moe_layer_outputs._fields_]

@@ -20,7 +20,10 @@ def _forward(inp: LayerInputs, bias=None, alpha=0.0):
                 logits=torch.empty(T, E, dtype=torch.float32, device=d), counts=torch.empty(E, **i32),
                 kept=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32), inv=torch.empty(T, K, **i32),
                 n_dropped=torch.empty(1, **i32), f=torch.empty(E, dtype=torch.float32, device=d),
-                P=torch.empty(E, dtype=torch.float32, device=d), aux=torch.empty(1, dtype=torch.float32, device=d))
+                P=torch.empty(E, dtype=torch.float32, device=d), aux=torch.empty(1, dtype=torch.float32, device=d),
+                P_topk=torch.empty(E, dtype=torch.float32, device=d),
+                aux_topk=torch.empty(1, dtype=torch.float32, device=d),
+                z_loss=torch.empty(1, dtype=torch.float32, device=d))
     y = torch.full((T, inp.wl.d_model), float("nan"), dtype=torch.float32, device=d)
     abi.moe_reset_device_status(inp.ws)
     abi.moe_layer_forward(inp.dims, inp.x, inp.Wr, bias, alpha, inp.W13p, inp.W2p, y, inp.ws, outs)
@@ -60,6 +63,18 @@ def _check(inp, y, outs, ref, bias32=None, tokens=None, mirror=None):
     assert np.max(np.abs(f64(outs["P"]) - ref["P"])) <= 1e-5 + 2 * float(bound.max())
     aux_ref = E * float(np.sum(f_ref * ref["P"]))
     assert abs(float(outs["aux"].item()) - aux_ref) <= 1e-4 * max(1.0, aux_ref)
+    # top-K-only balance statistic: a token routed differently moves P~ by at most 2/T
+    Pt = f64(outs["P_topk"])
+    assert abs(Pt.sum() - 1.0) <= 1e-5
+    assert np.max(np.abs(Pt - ref["P_topk"])) <= 1e-5 + 2.0 * unc.sum() / inp.T
+    at_ref = E * float(np.sum(f_ref * Pt))
+    assert abs(float(outs["aux_topk"].item()) - at_ref) <= 1e-5 * max(1.0, at_ref)
+    # router z-loss: each log-sum-exp moves by at most the largest logit error
+    l64m = l64.max(axis=1)
+    lse = l64m + np.log(np.exp(l64 - l64m[:, None]).sum(axis=1))
+    delta = float(bound.max()) + 2e-6 * float(np.abs(lse).max())
+    tol = 2.0 * float(np.abs(lse).max()) * delta + delta * delta + 1e-5 * ref["z_loss"]
+    assert abs(float(outs["z_loss"].item()) - ref["z_loss"]) <= tol
     return rows
 
 
