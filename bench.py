@@ -47,7 +47,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--workload", default="mixtral_decode", choices=sorted(synth.workloads().keys()))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--e2e-steps", type=int, default=200)
+    p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: as many as --steps)")
     p.add_argument("--cpu-sample-tokens", type=int, default=32)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--tokens", type=int, default=0,
@@ -383,7 +383,7 @@ def run_ours(args):
     for b in range(2):
         ev_done[b].record(s)
         ev_out[b].record(s)
-    E2E = max(1, args.e2e_steps)
+    E2E = max(1, args.e2e_steps if args.e2e_steps > 0 else K)
 
     def e2e_step(i):
         b = i % 2
