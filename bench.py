@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: as many as --steps)")
     p.add_argument("--cpu-sample-tokens", type=int, default=32)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--chunk-tokens", type=int, default=0,
+                   help="run the chunked layer (moe_layer_forward_chunked) in chunks of this many tokens")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's T (smaller cases for profiling); recorded in config")
     return p.parse_args()
@@ -290,7 +292,8 @@ def run_ours(args):
         host_w = [t.to("cpu", torch.float32) for t in (x, Wr, W1, W3, W2)]
     del W1, W3, W2
     torch.cuda.empty_cache()
-    ws = abi.alloc_workspace(dims, dev)
+    chunk = args.chunk_tokens
+    ws = abi.alloc_chunked_workspace(dims, chunk, dev) if chunk > 0 else abi.alloc_workspace(dims, dev)
     y = torch.empty(wl.T, wl.d_model, dtype=torch.float32, device=dev)
     E = wl.E
     i32 = dict(dtype=torch.int32, device=dev)
@@ -300,8 +303,14 @@ def run_ours(args):
     bias = torch.zeros(E, dtype=torch.float32, device=dev) if wl.use_bias else None
     alpha = float(wl.alpha) if wl.use_bias else 0.0
 
+    def layer(x_in, y_out, evs=None):
+        if chunk > 0:   # per-stage events are not recorded by the chunked layer
+            abi.moe_layer_forward_chunked(dims, chunk, x_in, Wr, bias, alpha, W13p, W2p, y_out, ws, outs)
+        else:
+            abi.moe_layer_forward(dims, x_in, Wr, bias, alpha, W13p, W2p, y_out, ws, outs, stage_events=evs)
+
     def step(evs=None):
-        abi.moe_layer_forward(dims, x, Wr, bias, alpha, W13p, W2p, y, ws, outs, stage_events=evs)
+        layer(x, y, evs)
 
     abi.moe_reset_device_status(ws)
     for _ in range(args.warmup):
@@ -316,28 +325,33 @@ def run_ours(args):
     # from starting early, so the other steps run without them)
     K = args.steps
     nev = abi.NUM_STAGE_EVENTS
-    sampled = list(range(0, K, STAGE_EVERY))
+    sampled = list(range(0, K, STAGE_EVERY)) if chunk == 0 else []
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(K)]
     s = torch.cuda.current_stream()
     for row in evs:      # create the underlying events before the timed region
         for e in row:
             e.record(s)
+    sampled_set = set(sampled)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.reset_peak_memory_stats(dev)
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
     start.record(s)
     for i in range(K):
-        step(evs[i] if i % STAGE_EVERY == 0 else None)
+        step(evs[i] if i in sampled_set else None)
     end.record(s)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     ms_total = max_over_ranks(start.elapsed_time(end), dev)
     ms_step = ms_total / K
-    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in sampled])
-    stage_ms = stage.mean(axis=0)
+    peak_bytes = int(torch.cuda.max_memory_allocated(dev))
+    stage_ms = None
+    if sampled:
+        stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in sampled])
+        stage_ms = stage.mean(axis=0)
     st, detail = abi.moe_get_device_status(ws)
     if st != 0:
         raise RuntimeError(f"device-side wait ran out in the timed region (code {detail})")
@@ -346,26 +360,32 @@ def run_ours(args):
     kept = outs["kept"].cpu().numpy()
     alg = layer_algorithmic(wl, counts, kept)
     peaks, peak_src = load_peaks()
-    gemm_ms = float(stage_ms[2])
+    gemm_ms = float(stage_ms[2]) if stage_ms is not None else ms_step
     sustained = ms_total > 1000.0
     tensor_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     bw = peaks["hbm_gbs"]
     t_bytes = alg["layer_bytes"] / (bw * 1e9)
     t_flops = alg["layer_flops"] / (tensor_peak * 1e12)
     layer_bound = "hbm" if t_bytes >= t_flops else "tensor"
-    g_bytes_t = alg["gemm_bytes"] / (bw * 1e9)
-    g_flops_t = alg["gemm_flops"] / (tensor_peak * 1e12)
+    # the expert GEMMs' own work and time; the chunked layer records no
+    # per-stage events, so there the whole layer's work over its time
+    w_bytes = alg["gemm_bytes"] if stage_ms is not None else alg["layer_bytes"]
+    w_flops = alg["gemm_flops"] if stage_ms is not None else alg["layer_flops"]
+    g_bytes_t = w_bytes / (bw * 1e9)
+    g_flops_t = w_flops / (tensor_peak * 1e12)
     if g_bytes_t >= g_flops_t:
-        achieved = alg["gemm_bytes"] / (gemm_ms * 1e-3) / 1e9
+        achieved = w_bytes / (gemm_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": bw, "unit": "GB/s", "frac": achieved / bw}
     else:
-        achieved = alg["gemm_flops"] / (gemm_ms * 1e-3) / 1e12
+        achieved = w_flops / (gemm_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
                 "frac": achieved / tensor_peak}
     kernel = abi.moe_ffn_kernel(dims)
-    traffic = profile_traffic(kernel, wl.name)
-    roof.update({"traffic": traffic, "kernel": f"{kernel} (gate/up and down in one launch)",
-                 "algorithmic_per_step": alg["gemm_bytes"] if roof["bound"] == "hbm" else alg["gemm_flops"],
+    traffic = profile_traffic(kernel, wl.name) if chunk == 0 else None
+    what = (f"{kernel} (gate/up and down in one launch)" if chunk == 0 else
+            f"whole chunked layer (no per-stage events; {kernel} once per chunk)")
+    roof.update({"traffic": traffic, "kernel": what,
+                 "algorithmic_per_step": w_bytes if roof["bound"] == "hbm" else w_flops,
                  "ms_per_step": gemm_ms, "peak_source": f"{peak_src}" + (" sustained" if sustained and roof["bound"] == "tensor" else "")})
 
     # ---- end to end through the public API with host buffers: every step
@@ -393,7 +413,7 @@ def run_ours(args):
         ev_in[b].record(s_in)
         s.wait_event(ev_in[b])
         s.wait_event(ev_out[b])               # y_dev[b] copied out by step i - 2
-        abi.moe_layer_forward(dims, x_dev[b], Wr, bias, alpha, W13p, W2p, y_dev[b], ws, outs)
+        layer(x_dev[b], y_dev[b])
         ev_done[b].record(s)
         s_out.wait_event(ev_done[b])
         with torch.cuda.stream(s_out):
@@ -416,7 +436,10 @@ def run_ours(args):
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / E2E, dev)
 
-    launches = abi.moe_layer_launch_count(dims, True, bias is not None and alpha != 0.0) * K
+    if chunk > 0:
+        launches = abi.moe_layer_chunked_launch_count(dims, chunk, True, bias is not None and alpha != 0.0) * K
+    else:
+        launches = abi.moe_layer_launch_count(dims, True, bias is not None and alpha != 0.0) * K
 
     cpu = None
     if host_w is not None:
@@ -440,12 +463,16 @@ def run_ours(args):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
                    "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (expert weights %.2f GB)" % (wl.E * 3 * wl.d_model * wl.d_ff * 2 / 1e9)},
+                   "l2": "inputs larger than L2 (expert weights %.2f GB)" % (wl.E * 3 * wl.d_model * wl.d_ff * 2 / 1e9),
+                   "workspace_bytes": int(ws.numel()), "peak_device_bytes": peak_bytes,
+                   **({"chunk_tokens": chunk,
+                       "workspace_bytes_whole_batch": abi.moe_workspace_size(dims)} if chunk > 0 else {})},
         "roofline": roof,
         "layer_roofline": {"bound": layer_bound, "t_roof_ms": max(t_bytes, t_flops) * 1e3, "t_meas_ms": ms_step,
                            "frac": max(t_bytes, t_flops) * 1e3 / ms_step, "bytes": alg["layer_bytes"],
                            "flops": alg["layer_flops"]},
-        "stage_ms": {"route": stage_ms[0], "dispatch": stage_ms[1], "expert_gemms": stage_ms[2],
+        "stage_ms": None if stage_ms is None else
+                    {"route": stage_ms[0], "dispatch": stage_ms[1], "expert_gemms": stage_ms[2],
                      "combine": stage_ms[3], "stats_bias": stage_ms[4]},
         "routing": {"n_kept": alg["n_kept"], "experts_touched": alg["touched"],
                     "max_over_mean_load": float(counts.max() / (wl.T * wl.K / wl.E)),

@@ -285,6 +285,31 @@ MOE_API int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe
                       float alpha, const moe_bf16* W13p, const moe_bf16* W2p, float* y,
                       const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Chunked MoE ([P2] section 4.3: prefill tokens go through the MoE step in
+ * chunks, so the expert stage never holds the whole batch and the memory
+ * peak drops).  The same layer as moe_layer_forward for dims without a
+ * capacity (a capacity is defined over the whole batch: capacity_factor > 0
+ * returns MOE_EUNSUPPORTED):
+ *   1. routing, statistics rows and top-K of all T tokens (small state);
+ *   2. for each chunk of at most chunk_tokens consecutive tokens: dispatch,
+ *      both expert GEMMs and the combine into y's rows of that chunk, in one
+ *      chunk-sized workspace region;
+ *   3. the whole batch's counts, f_i, P_i, aux, P_topk, aux_topk, z_loss and
+ *      the bias update (with alpha != 0), from the whole batch's routing.
+ * Routing, statistics and the bias update equal moe_layer_forward's; y rows
+ * agree within floating-point reordering (the GEMM tiling follows the chunk's
+ * groups).  out->offsets and out->inv are not written (rows are chunk-local);
+ * out->kept receives the counts and out->n_dropped 0.  stage_events are
+ * ignored.  ws: moe_chunked_workspace_size bytes (host query); d_model % 8 == 0. */
+MOE_API int moe_chunked_workspace_size(const moe_dims* dims, int64_t chunk_tokens, size_t* bytes);
+/* Kernel launches one moe_layer_forward_chunked call enqueues (host only;
+ * < 0 on bad arguments). */
+MOE_API int moe_layer_chunked_launch_count(const moe_dims* dims, int64_t chunk_tokens, int stats, int bias_update);
+MOE_API int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const moe_bf16* x,
+                                      const moe_bf16* Wr, float* bias, float alpha, const moe_bf16* W13p,
+                                      const moe_bf16* W2p, float* y, const moe_layer_outputs* out, void* ws,
+                                      size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,6 +32,7 @@ EXPORTED = [
     "moe_get_device_status", "moe_pack_weights", "moe_route", "moe_route_from_logits", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
     "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc", "moe_ffn_kernel",
+    "moe_chunked_workspace_size", "moe_layer_forward_chunked", "moe_layer_chunked_launch_count",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -86,6 +87,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_packed_weight_bytes": (I, [dims_p, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
         "moe_permute_noalloc": (I, [dims_p, P, P, P, P, P, P, P, P, P, P]),
         "moe_ffn_kernel": (I, [dims_p]),
+        "moe_chunked_workspace_size": (I, [dims_p, ctypes.c_int64, ctypes.POINTER(SZ)]),
+        "moe_layer_chunked_launch_count": (I, [dims_p, ctypes.c_int64, I, I]),
+        "moe_layer_forward_chunked": (I, [dims_p, ctypes.c_int64, P, P, P, F, P, P, P,
+                                          ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -165,6 +170,18 @@ def moe_workspace_size(dims) -> int:
     n = ctypes.c_size_t(0)
     _check("moe_workspace_size", load().moe_workspace_size(ctypes.byref(_dims(dims)), ctypes.byref(n)))
     return int(n.value)
+
+
+def moe_chunked_workspace_size(dims, chunk_tokens: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_chunked_workspace_size", load().moe_chunked_workspace_size(
+        ctypes.byref(_dims(dims)), ctypes.c_int64(chunk_tokens), ctypes.byref(n)))
+    return int(n.value)
+
+
+def alloc_chunked_workspace(dims, chunk_tokens: int, device="cuda") -> torch.Tensor:
+    """Caller-owned workspace for moe_layer_forward_chunked."""
+    return torch.zeros(moe_chunked_workspace_size(dims, chunk_tokens), dtype=torch.uint8, device=device)
 
 
 def alloc_workspace(dims, device="cuda") -> torch.Tensor:
@@ -265,6 +282,29 @@ def moe_layer_forward(dims, x, Wr, bias, alpha: float, W13p, W2p, y, ws, outputs
         ctypes.byref(_dims(dims)), _ptr(x, BF16, "x"), _ptr(Wr, BF16, "Wr"), _ptr(bias, F32, "bias"),
         ctypes.c_float(alpha), _ptr(W13p, BF16, "W13p"), _ptr(W2p, BF16, "W2p"), _ptr(y, F32, "y"),
         ctypes.byref(o) if o is not None else None, _ptr(ws, None, "ws"), ws.numel(), _stream(stream)))
+
+
+def moe_layer_forward_chunked(dims, chunk_tokens: int, x, Wr, bias, alpha: float, W13p, W2p, y, ws,
+                              outputs: Optional[dict] = None, stream=None):
+    """The layer in chunks of at most ``chunk_tokens`` tokens (see the header)."""
+    o = None
+    if outputs:
+        o = moe_layer_outputs()
+        for k, t in outputs.items():
+            setattr(o, k, _ptr(t, None, k))
+    _check("moe_layer_forward_chunked", load().moe_layer_forward_chunked(
+        ctypes.byref(_dims(dims)), ctypes.c_int64(chunk_tokens), _ptr(x, BF16, "x"), _ptr(Wr, BF16, "Wr"),
+        _ptr(bias, F32, "bias"), ctypes.c_float(alpha), _ptr(W13p, BF16, "W13p"), _ptr(W2p, BF16, "W2p"),
+        _ptr(y, F32, "y"), ctypes.byref(o) if o is not None else None, _ptr(ws, None, "ws"), ws.numel(),
+        _stream(stream)))
+
+
+def moe_layer_chunked_launch_count(dims, chunk_tokens: int, stats: bool, bias_update: bool) -> int:
+    n = load().moe_layer_chunked_launch_count(ctypes.byref(_dims(dims)), ctypes.c_int64(chunk_tokens), int(stats),
+                                              int(bias_update))
+    if n < 0:
+        raise MoEError("moe_layer_chunked_launch_count", n, "invalid arguments")
+    return n
 
 
 def moe_layer_launch_count(dims, stats: bool, bias_update: bool) -> int:

@@ -141,6 +141,48 @@ int map_launch(int r) {
     return MOE_ECUDA;
 }
 
+// Workspace of the chunked layer: one chunk's layer workspace at offset 0
+// (large enough for a full chunk and for the last, shorter one; its status
+// word is the workspace's), then the whole batch's routing state.
+struct ChunkLayout {
+    size_t chunk_bytes;  // the per-chunk region
+    Layout whole;        // whole-batch router sizes, offsets rebased past the chunk region
+    size_t counts_total, total;
+};
+
+ChunkLayout chunk_layout_of(const moe_dims* d, int64_t chunk) {
+    ChunkLayout C{};
+    moe_dims dc = *d;
+    dc.T = chunk < d->T ? chunk : d->T;
+    C.chunk_bytes = layout_of(&dc).total;
+    const int64_t rem = d->T % dc.T;
+    if (rem > 0) {
+        dc.T = rem;
+        const size_t r = layout_of(&dc).total;
+        C.chunk_bytes = r > C.chunk_bytes ? r : C.chunk_bytes;
+    }
+    C.whole = layout_of(d);
+    const int64_t T = d->T, E = d->E, K = d->K;
+    size_t o = C.chunk_bytes;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align256(o + bytes);
+        return at;
+    };
+    Layout& W = C.whole;
+    W.status = 0;  // shared with the chunk region
+    W.sched_router = take(gemm_sched_bytes(1));
+    W.idx = take(static_cast<size_t>(T * K) * 4);
+    W.w = take(static_cast<size_t>(T * K) * 4);
+    W.logits = W.fused_router ? 0 : take(static_cast<size_t>(T * E) * 4);
+    W.prob_part = take(static_cast<size_t>(W.route_nb) * (2 * E + 1) * 4);
+    W.prob_mean = take(E * 4);
+    W.wrt = W.fused_router ? 0 : take(static_cast<size_t>((W.E_pad + 127) / 128) * 128 * ((d->d_model + 63) / 64) * 64 * 2);
+    C.counts_total = take(E * 4);
+    C.total = o;
+    return C;
+}
+
 int check_ws(const moe_dims* d, void* ws, size_t ws_bytes) {
     if (!ws || !aligned16(ws)) return MOE_EINVAL;
     if (ws_bytes < layout_of(d).total) return MOE_EWORKSPACE;
@@ -506,6 +548,116 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
     mark(4);
     mark(5);
     return MOE_OK;
+}
+
+int moe_chunked_workspace_size(const moe_dims* dims, int64_t chunk_tokens, size_t* bytes) {
+    MOE_TRY(check_dims(dims));
+    if (!bytes || chunk_tokens < 1) return MOE_EINVAL;
+    *bytes = chunk_layout_of(dims, chunk_tokens).total;
+    return MOE_OK;
+}
+
+int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const moe_bf16* x, const moe_bf16* Wr,
+                              float* bias, float alpha, const moe_bf16* W13p, const moe_bf16* W2p, float* y,
+                              const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (chunk_tokens < 1) return MOE_EINVAL;
+    if (!x || !Wr || !W13p || !W2p || !y) return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(Wr) || !aligned16(W13p) || !aligned16(W2p) || !aligned16(y))
+        return MOE_EUNSUPPORTED;
+    if (!std::isfinite(alpha)) return MOE_EINVAL;
+    if (capacity_of(dims) >= 0) return MOE_EUNSUPPORTED;  // a capacity is defined over the whole batch
+    if (dims->d_model % 8 != 0) return MOE_EUNSUPPORTED;    // chunk offsets into x, y stay 16-byte aligned
+    const ChunkLayout CL = chunk_layout_of(dims, chunk_tokens);
+    if (!ws || !aligned16(ws)) return MOE_EINVAL;
+    if (ws_bytes < CL.total) return MOE_EWORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    moe_layer_outputs o{};
+    if (out) o = *out;
+    const int64_t T = dims->T, K = dims->K, D = dims->d_model;
+    const Layout& W = CL.whole;
+    int32_t* idx = o.topk_idx ? o.topk_idx : at<int32_t>(ws, W.idx);
+    float* w = o.topk_w ? o.topk_w : at<float>(ws, W.w);
+    int32_t* counts = o.counts ? o.counts : at<int32_t>(ws, CL.counts_total);
+    const bool want_stats = o.P || o.aux || o.f || o.P_topk || o.aux_topk || o.z_loss;
+    float* P = o.P ? o.P : at<float>(ws, W.prob_mean);
+    const bf16* xb = reinterpret_cast<const bf16*>(x);
+
+    // 1. routing of the whole batch (its state is small: [T, K] and per-block rows)
+    MOE_TRY(do_route(dims, W, xb, reinterpret_cast<const bf16*>(Wr), bias, o.logits, idx, w,
+                     want_stats ? P : nullptr, ws, st, /*finalize=*/false));
+    // 2. dispatch, expert GEMMs and combine chunk by chunk in one chunk-sized workspace
+    for (int64_t t0 = 0; t0 < T; t0 += chunk_tokens) {
+        moe_dims dc = *dims;
+        dc.T = T - t0 < chunk_tokens ? T - t0 : chunk_tokens;
+        const Layout Lc = layout_of(&dc);
+        const int32_t* idx_c = idx + t0 * K;
+        const bf16* x_c = xb + t0 * D;
+        int32_t* cnt_c = at<int32_t>(ws, Lc.counts);
+        int32_t* inv_c = at<int32_t>(ws, Lc.inv);
+        if (dispatch_gather_fused_supported(dc.T, dc.E, dc.K))
+            MOE_TRY(map_launch(launch_dispatch_gather_small(
+                idx_c, x_c, dc.T, dc.d_model, dc.E, dc.K, -1, cnt_c, at<int32_t>(ws, Lc.kept),
+                at<int32_t>(ws, Lc.offsets), inv_c, at<int32_t>(ws, Lc.src), at<bf16>(ws, Lc.xperm),
+                at<int32_t>(ws, Lc.ndrop), at<int32_t>(ws, Lc.sched_ffn),
+                static_cast<int>(gemm_sched_bytes(dc.E) / 4), st)));
+        else
+            MOE_TRY(map_launch(launch_permute(idx_c, x_c, dc.T, dc.d_model, dc.E, dc.K, -1,
+                                              at<int32_t>(ws, Lc.block_hist), cnt_c, at<int32_t>(ws, Lc.kept),
+                                              at<int32_t>(ws, Lc.offsets), inv_c, at<int32_t>(ws, Lc.src),
+                                              at<bf16>(ws, Lc.xperm), at<int32_t>(ws, Lc.ndrop),
+                                              at<int32_t>(ws, Lc.sched_ffn),
+                                              static_cast<int>(gemm_sched_bytes(dc.E) / 4), st)));
+        float* yp = at<float>(ws, Lc.yperm);
+        MOE_TRY(do_ffn(&dc, Lc, at<bf16>(ws, Lc.xperm), at<int32_t>(ws, Lc.offsets),
+                       reinterpret_cast<const bf16*>(W13p), reinterpret_cast<const bf16*>(W2p),
+                       at<bf16>(ws, Lc.h), yp, Lc.nsplit, ws, st));
+        MOE_TRY(map_launch(launch_combine(yp, Lc.nsplit, dc.T * dc.K * dc.d_model, inv_c, w + t0 * K, dc.T,
+                                          dc.d_model, dc.K, y + t0 * D, st)));
+        MOE_TRY(map_launch(launch_accumulate_counts(counts, cnt_c, dims->E, t0 == 0, st)));
+    }
+    // 3. the whole batch's statistics and bias update (one statistics CTA, no tokens)
+    if (o.kept)
+        if (cudaMemcpyAsync(o.kept, counts, dims->E * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return MOE_ECUDA;
+    if (o.n_dropped)
+        if (cudaMemsetAsync(o.n_dropped, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ECUDA;
+    if (want_stats || (bias && alpha != 0.0f)) {
+        StatsTail tail{};
+        tail.counts = counts;
+        tail.E = dims->E;
+        tail.T = T;
+        if (want_stats) {
+            tail.part = at<float>(ws, W.prob_part);
+            tail.nblocks = W.route_nb;
+            tail.P = P;
+            tail.f = o.f;
+            tail.aux = o.aux;
+            tail.P_topk = o.P_topk;
+            tail.aux_topk = o.aux_topk;
+            tail.z_loss = o.z_loss;
+        }
+        if (bias && alpha != 0.0f) {
+            tail.bias = bias;
+            tail.alpha = alpha;
+        }
+        MOE_TRY(map_launch(launch_combine(nullptr, 1, 0, nullptr, nullptr, 0, dims->d_model, dims->K, nullptr, st,
+                                          &tail)));
+    }
+    return MOE_OK;
+}
+
+int moe_layer_chunked_launch_count(const moe_dims* dims, int64_t chunk_tokens, int stats, int bias_update) {
+    if (check_dims(dims) != MOE_OK || chunk_tokens < 1) return -1;
+    const Layout L = layout_of(dims);
+    int n = L.fused_router ? 1 : 3;  // routing of the whole batch
+    for (int64_t t0 = 0; t0 < dims->T; t0 += chunk_tokens) {
+        const int64_t Tc = dims->T - t0 < chunk_tokens ? dims->T - t0 : chunk_tokens;
+        n += dispatch_gather_fused_supported(Tc, dims->E, dims->K) ? 1 : launch_count(Tc) + 1;
+        n += 3;  // expert GEMMs, combine, counts accumulation
+    }
+    if (stats || bias_update) n += 1;  // the statistics CTA
+    return n;
 }
 
 int moe_ffn_kernel(const moe_dims* dims) {

@@ -120,7 +120,7 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
     // with a statistics tail the last CTA does only that
     const int ntok_blocks = static_cast<int>(gridDim.x) - (tail.counts ? 1 : 0);
     if (tail.counts && static_cast<int>(blockIdx.x) == ntok_blocks) {
-        stats_tail(tail, T, K);
+        stats_tail(tail, tail.T > 0 ? tail.T : T, K);
         return;
     }
     const int nvec = d / 4;
@@ -230,6 +230,14 @@ __global__ void bias_update_kernel(const int32_t* __restrict__ counts, int64_t T
     bias[e] = b;
 }
 
+__global__ void accumulate_counts_kernel(int32_t* __restrict__ dst, const int32_t* __restrict__ src, int E,
+                                         int first) {
+    pdl_trigger();
+    pdl_wait();
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < E) dst[e] = (first ? 0 : dst[e]) + src[e];
+}
+
 // W13p[e][32b + j][k] = (j < 16 ? W1 : W3)[e][k][16b + (j & 15)];  W2p[e][n][k] = W2[e][k][n].
 // Both are [rows][cols] <- transpose of a [cols][rows]-shaped source, by
 // 32 x 32 tiles through shared memory.
@@ -317,6 +325,11 @@ int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
+
+int launch_accumulate_counts(int32_t* dst, const int32_t* src, int E, bool first, cudaStream_t st) {
+    (void)launch_pdl(accumulate_counts_kernel, dim3((E + 255) / 256), dim3(256), 0, st, dst, src, E, first ? 1 : 0);
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
 
 int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias, cudaStream_t st) {
     (void)launch_pdl(bias_update_kernel, dim3((E + 255) / 256), dim3(256), 0, st, counts, T * K, E, alpha, bias);

@@ -128,11 +128,14 @@ struct StatsTail {
     float* bias;            // updated in place when non-null and alpha != 0
     float alpha;
     int E;
+    int64_t T;              // tokens the statistics cover (0: the combine's own T)
 };
 
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv,
                    const float* w, int64_t T, int d, int K, float* y, cudaStream_t st,
                    const StatsTail* tail = nullptr);
+// dst[e] = (first ? 0 : dst[e]) + src[e] for e < E (a batch's counts from its chunks').
+int launch_accumulate_counts(int32_t* dst, const int32_t* src, int E, bool first, cudaStream_t st);
 int launch_reduce_splits(const float* part, int nsplit, int64_t split_stride, const int32_t* offsets,
                          int E, int d, float* y_perm, cudaStream_t st);
 int launch_stats(const int32_t* counts, const float* prob_mean, int64_t T, int E, int K,

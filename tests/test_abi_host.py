@@ -134,3 +134,45 @@ def test_layer_outputs_struct_matches_header():
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     names = re.findall(r"\*\s*(\w+)\s*;", body)
     assert names == [n for n, _ in abi.moe_layer_outputs._fields_]
+
+
+def test_chunked_workspace_and_host_checks(lib):
+    big = abi.Dims(16384, 4096, 14336, 8, 2)
+    full = abi.moe_workspace_size(big)
+    chunked = abi.moe_chunked_workspace_size(big, 2048)
+    # the expert stage buffers (x_perm, H, Y_perm) shrink with the chunk
+    A_c = 2048 * 2
+    assert chunked < full / 4
+    assert chunked >= A_c * 4096 * 2 + A_c * 14336 * 2 + A_c * 4096 * 4
+    # one chunk covering the batch needs about the unchunked workspace
+    assert abi.moe_chunked_workspace_size(big, 16384) >= full
+    # the last, shorter chunk may need more per-token room (a reduction split): it is covered
+    odd = abi.Dims(4096 + 100, 1024, 2048, 8, 2)
+    assert abi.moe_chunked_workspace_size(odd, 4096) >= abi.moe_workspace_size(abi.Dims(100, 1024, 2048, 8, 2))
+    with pytest.raises(abi.MoEError):
+        abi.moe_chunked_workspace_size(big, 0)
+    # a capacity is defined over the whole batch: rejected before any launch
+    d = abi.Dims(1000, 128, 256, 8, 2, 1.0).c()
+    fake = ctypes.c_void_p(0x10000)   # never dereferenced
+    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 256, fake, fake, None, 0.0, fake, fake, fake, None,
+                                       fake, 1 << 30, None)
+    assert st == abi.MOE_EUNSUPPORTED
+    d = abi.Dims(1000, 128, 256, 8, 2).c()
+    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 0, fake, fake, None, 0.0, fake, fake, fake, None,
+                                       fake, 1 << 30, None)
+    assert st == abi.MOE_EINVAL
+    n = abi.moe_chunked_workspace_size(abi.Dims(1000, 128, 256, 8, 2), 256)
+    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 256, fake, fake, None, 0.0, fake, fake, fake, None,
+                                       fake, n - 1, None)
+    assert st == abi.MOE_EWORKSPACE
+
+
+def test_chunked_launch_counts(lib):
+    # Mixtral prefill in 4 chunks of 4096: fused router + 4 x (hist/scan/rank + gather, GEMMs, combine,
+    # counts) + the statistics CTA
+    d = abi.Dims(16384, 4096, 14336, 8, 2)
+    assert abi.moe_layer_chunked_launch_count(d, 4096, True, False) == 1 + 4 * (4 + 3) + 1
+    # chunks of 1024 take the one-launch dispatch
+    assert abi.moe_layer_chunked_launch_count(d, 1024, True, False) == 1 + 16 * (1 + 3) + 1
+    # no statistics, no bias: no statistics CTA
+    assert abi.moe_layer_chunked_launch_count(d, 16384, False, False) == 1 + (4 + 3)
