@@ -7,7 +7,10 @@
  *            stable token-order ranks, capacity drop, row gather)
  *   expert   per expert: H = silu(X W1) * (X W3); Y = H W2  (tcgen05 GEMMs)
  *   combine  y[t] = sum_k w[t,k] * Y[row(t,k)]  (deterministic gather)
- *   stats    counts, f_i, P_i, aux = E * sum f_i P_i; aux-free bias update
+ *   stats    counts, f_i, P_i, aux = E * sum f_i P_i, the top-K-only balance
+ *            statistic and the router z-loss; aux-free bias update
+ * moe_layer_forward runs all five on one stream; moe_layer_forward_chunked
+ * runs the same layer over token chunks in a chunk-sized workspace.
  *
  * Sources (web pages; cited by title and section):
  *   [P1] "MoE serving essay", dpshk.com/news/3211971

@@ -12,7 +12,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kVersion = 100;
+constexpr int kVersion = 101;  // 1.01: layer outputs gained P_topk, aux_topk, z_loss; chunked layer
 constexpr int64_t kMaxT = int64_t(1) << 24;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
