@@ -119,6 +119,17 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3])}
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
+def l2_note(wl) -> str:
+    """How the timed steps relate to the 126 MB L2 (no flush between steps)."""
+    wbytes = wl.E * 3 * wl.d_model * wl.d_ff * 2
+    if wbytes > L2_BYTES:
+        return "inputs larger than L2 (expert weights %.2f GB)" % (wbytes / 1e9)
+    return "inputs fit in L2 (expert weights %.1f MB), not flushed between steps: a parity-size case" % (wbytes / 1e6)
+
+
 def layer_algorithmic(wl, counts: np.ndarray, kept: np.ndarray):
     """Algorithmic bytes / FLOPs of one layer step and of its expert GEMMs.
 
@@ -246,7 +257,7 @@ def run_reference(args):
         "steps": steps, "warmup": warm, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
-                   "capacity_factor": wl.capacity_factor},
+                   "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{args.gpus}", "l2": l2_note(wl)},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{S} of {wl.T} tokens per step (routing, counts and capacity over all "
                                    f"{wl.T}); {steps} steps after {warm} warm-up (of {args.steps}/{args.warmup} "
@@ -463,10 +474,9 @@ def run_ours(args):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
                    "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (expert weights %.2f GB)" % (wl.E * 3 * wl.d_model * wl.d_ff * 2 / 1e9),
-                   "workspace_bytes": int(ws.numel()), "peak_device_bytes": peak_bytes,
-                   **({"chunk_tokens": chunk,
-                       "workspace_bytes_whole_batch": abi.moe_workspace_size(dims)} if chunk > 0 else {})},
+                   "l2": l2_note(wl), **({"chunk_tokens": chunk} if chunk > 0 else {})},
+        "memory": {"workspace_bytes": int(ws.numel()), "peak_device_bytes": peak_bytes,
+                   **({"workspace_bytes_whole_batch": abi.moe_workspace_size(dims)} if chunk > 0 else {})},
         "roofline": roof,
         "layer_roofline": {"bound": layer_bound, "t_roof_ms": max(t_bytes, t_flops) * 1e3, "t_meas_ms": ms_step,
                            "frac": max(t_bytes, t_flops) * 1e3 / ms_step, "bytes": alg["layer_bytes"],
