@@ -75,6 +75,8 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (600, 256, 256, 16, 4, 1.2),      # CTA pairs, weight- and token-major groups in one launch
     (512, 256, 2560, 64, 4, 0.0),     # CTA pairs, gate/up tiles of two 256-row weight sub-tiles, 8-way split
     (1024, 1024, 1024, 256, 8, 1.1),  # CTA pairs, two weight sub-tiles in both phases, skewed small groups
+    (2000, 256, 256, 1, 1, 0.0),      # one expert (dense FFN) on CTA-pair token-major tiles, ragged tail
+    (1, 256, 512, 8, 2, 0.0),         # a single token: two one-row groups on CTA-pair weight-major tiles
 ])
 def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
     # weight scale shrinks with the width so |y| stays O(1), the scale the
