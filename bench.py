@@ -48,7 +48,7 @@ def parse():
     p.add_argument("--workload", default="mixtral_decode", choices=sorted(synth.workloads().keys()))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: as many as --steps)")
-    p.add_argument("--cpu-sample-tokens", type=int, default=32)
+    p.add_argument("--cpu-sample-tokens", type=int, default=96)  # ~5-7 s of oracle work per run at decode
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--chunk-tokens", type=int, default=0,
                    help="run the chunked layer (moe_layer_forward_chunked) in chunks of this many tokens")
