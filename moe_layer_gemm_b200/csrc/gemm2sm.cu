@@ -302,6 +302,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             uint32_t s = 0, ph = 0, r = 0, rph = 0;
             bool ok = true;
             bool sent_end = false;
+            uint32_t issued_mask = 0, issued_ph = 0;  // stages armed by the leader, and their phase
             int next = leader ? atomicAdd(&a.sched[0], 1) : 0;
             const uint32_t peer_ring = mapa_shared(smem_u32(ring), 1);
             const uint32_t peer_rfull = mapa_shared(smem_u32(rfull), 1);
@@ -378,6 +379,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                             tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + j * 2048, bar, kb * kBK,
                                           static_cast<int32_t>(trow + 16 * j), pol_last);
                     }
+                    issued_mask |= 1u << s;
+                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
             }
@@ -390,6 +393,14 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 mbar_arrive(&rfull[r]);
                 remote_arrive(peer_rfull + 8u * r);
             }
+            // Drain (leader): every stage's copies, the peer's included (they
+            // complete on the leader's barrier), have landed before the pair
+            // may pass its final cluster barrier and exit.  Bounded.
+            if (leader)
+                for (int i = 0; i < S; ++i)
+                    if (issued_mask & (1u << i))
+                        for (uint32_t it = 0; it < kWaitLimit; ++it)
+                            if (mbar_try_wait(&full[i], (issued_ph >> i) & 1u)) break;
         }
     } else if (warp == 1) {
         if (leader && lane == 0) {
