@@ -11,6 +11,13 @@ than L2, so no flush is needed between steps.  With N > 1 (torchrun), every
 rank runs an independent replica of the layer (the path has no exchange
 step), timing is the max over ranks and ``value`` counts all ranks' tokens.
 
+The headline is the Mixtral-shaped decode layer (T = 256).  The same JSON
+line also carries a second-long ``sustained`` run of it (the power cap has
+settled) and, on one GPU, a ``workloads`` entry for each other layer shape of
+the metric: Mixtral prefill (T = 16384, tensor-bound), the Qwen-like layer
+with capacity, and the DeepSeek-like layer whose steps update the bias in
+place and draw fresh tokens (step j takes the tokens of seed step j mod 10).
+
 ``--impl reference`` times the CPU oracle (the plain fp64 implementation the
 tests check against) on the host cores on a bounded token sample per step;
 under torchrun only rank 0 runs it.
@@ -48,10 +55,14 @@ def parse():
     p.add_argument("--workload", default="mixtral_decode", choices=sorted(synth.workloads().keys()))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: as many as --steps)")
-    p.add_argument("--cpu-sample-tokens", type=int, default=96)  # ~5-7 s of oracle work per run at decode
+    p.add_argument("--cpu-sample-tokens", type=int, default=96,
+                   help="tokens per oracle run of the CPU baseline (a bounded sample of the batch)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--chunk-tokens", type=int, default=0,
                    help="run the chunked layer (moe_layer_forward_chunked) in chunks of this many tokens")
+    p.add_argument("--no-extra", action="store_true",
+                   help="time only the headline workload (not prefill, capacity and bias-loop entries)")
+    p.add_argument("--no-sustained", action="store_true", help="skip the second-long sustained run")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's T (smaller cases for profiling); recorded in config")
     return p.parse_args()
@@ -135,9 +146,10 @@ def layer_algorithmic(wl, counts: np.ndarray, kept: np.ndarray):
 
     Layer: weights of every expert with >= 1 kept row (3 d f bf16) + x (bf16)
     + y (fp32) + W_r (bf16); FLOPs 2 T d E (router) + 6 d f N_kept.
-    Expert GEMMs (gate/up + down, one kernel): the touched weights plus the
-    activations they must move: x_perm in (bf16), H out and back in (bf16),
-    y_perm out (fp32); FLOPs 6 d f N_kept.
+    Expert GEMMs (gate/up + down, one kernel): the touched weights; FLOPs
+    6 d f N_kept.  The activations the GEMM kernel moves by design (x_perm
+    in, H out and back in, y_perm out) are reported apart, as
+    gemm_design_bytes, and are not counted as algorithmic work.
     """
     T, d, f, E = wl.T, wl.d_model, wl.d_ff, wl.E
     n_kept = int(kept.sum())
@@ -145,10 +157,10 @@ def layer_algorithmic(wl, counts: np.ndarray, kept: np.ndarray):
     wbytes = touched * 3 * d * f * 2
     layer_bytes = wbytes + T * d * 2 + T * d * 4 + d * E * 2
     layer_flops = 2 * T * d * E + 6 * d * f * n_kept
-    gemm_bytes = wbytes + n_kept * (d * 2 + 2 * f * 2 + d * 4)
     gemm_flops = 6 * d * f * n_kept
+    design = n_kept * (d * 2 + 2 * f * 2 + d * 4)
     return dict(n_kept=n_kept, touched=touched, layer_bytes=layer_bytes, layer_flops=layer_flops,
-                gemm_bytes=gemm_bytes, gemm_flops=gemm_flops)
+                gemm_bytes=wbytes, gemm_design_bytes=design, gemm_flops=gemm_flops)
 
 
 def profile_traffic(kernel: str, workload: str):
@@ -268,6 +280,164 @@ def run_reference(args):
     return 0
 
 
+class Layer:
+    """One workload's inputs, packed weights, workspace and outputs on the
+    device, and the call that runs one step of the layer."""
+
+    def __init__(self, wl, dev, chunk: int = 0, keep_host: bool = False):
+        from moe_layer_gemm_b200 import abi
+        self.abi = abi
+        self.wl = wl
+        self.dev = dev
+        self.chunk = chunk
+        self.dims = abi.Dims(wl.T, wl.d_model, wl.d_ff, wl.E, wl.K, wl.capacity_factor)
+        # workloads with per-step tokens (the bias loop) draw fresh x each
+        # step: step j uses the tokens of seed step j (cycled over wl.steps)
+        nx = wl.steps if wl.steps > 1 else 1
+        self.xs = [synth.make_x(wl, j, device=dev)[: wl.T].contiguous() for j in range(nx)]
+        self.Wr = synth.make_router(wl, device=dev)
+        W1, W3, W2 = synth.make_expert_weights(wl, device=dev)
+        self.W13p, self.W2p = abi.pack_weights(self.dims, W1, W3, W2)
+        torch.cuda.synchronize()
+        self.host = None
+        if keep_host:
+            self.host = [t.to("cpu", torch.float32) for t in (self.xs[0], self.Wr, W1, W3, W2)]
+        del W1, W3, W2
+        torch.cuda.empty_cache()
+        self.ws = abi.alloc_chunked_workspace(self.dims, chunk, dev) if chunk > 0 else abi.alloc_workspace(self.dims, dev)
+        self.y = torch.empty(wl.T, wl.d_model, dtype=torch.float32, device=dev)
+        E = wl.E
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.outs = dict(counts=torch.zeros(E, **i32), kept=torch.zeros(E, **i32), n_dropped=torch.zeros(1, **i32),
+                         f=torch.zeros(E, **f32), P=torch.zeros(E, **f32), aux=torch.zeros(1, **f32))
+        self.bias = torch.zeros(E, **f32) if wl.use_bias else None
+        self.alpha = float(wl.alpha) if wl.use_bias else 0.0
+
+    def run(self, x_in, y_out, evs=None):
+        abi = self.abi
+        if self.chunk > 0:   # per-stage events are not recorded by the chunked layer
+            abi.moe_layer_forward_chunked(self.dims, self.chunk, x_in, self.Wr, self.bias, self.alpha, self.W13p,
+                                          self.W2p, y_out, self.ws, self.outs)
+        else:
+            abi.moe_layer_forward(self.dims, x_in, self.Wr, self.bias, self.alpha, self.W13p, self.W2p, y_out,
+                                  self.ws, self.outs, stage_events=evs)
+
+    def step(self, i, evs=None):
+        self.run(self.xs[i % len(self.xs)], self.y, evs)
+
+    def launches(self) -> int:
+        stats, upd = True, self.bias is not None and self.alpha != 0.0
+        if self.chunk > 0:
+            return self.abi.moe_layer_chunked_launch_count(self.dims, self.chunk, stats, upd)
+        return self.abi.moe_layer_launch_count(self.dims, stats, upd)
+
+    def check_status(self, where: str):
+        st, detail = self.abi.moe_get_device_status(self.ws)
+        if st != 0:
+            raise RuntimeError(f"device-side status {st} ({detail}) {where}")
+
+
+# per-stage events: [0] before routing, [1] after routing, [2] after
+# dispatch, [3] after the expert GEMMs, [4] after the combine (whose extra
+# CTA also computes the statistics and the bias update; event [5] marks the
+# same point and is not reported)
+STAGES = ("route", "dispatch", "expert_gemms", "combine_stats")
+
+
+def time_steps(layer: Layer, K: int, barrier, clock_index: int, stage_every: int = STAGE_EVERY, start_step: int = 0):
+    """Time K layer steps with CUDA events on the launching stream (barrier
+    and device synchronisation on both sides); per-stage events ride on every
+    stage_every-th step (an event between two kernels keeps the second from
+    starting early, so the other steps run without them).  Clocks are
+    sampled during the region."""
+    from moe_layer_gemm_b200 import abi
+    nev = abi.NUM_STAGE_EVENTS
+    sampled = list(range(0, K, stage_every)) if layer.chunk == 0 and stage_every > 0 else []
+    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(nev)] for i in sampled}
+    s = torch.cuda.current_stream()
+    for row in evs.values():   # create the underlying events before the timed region
+        for e in row:
+            e.record(s)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.reset_peak_memory_stats(layer.dev)
+    clocks = ClockSampler(clock_index)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    start.record(s)
+    for i in range(K):
+        layer.step(start_step + i, evs.get(i))
+    end.record(s)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(start.elapsed_time(end), layer.dev)
+    stage_ms = None
+    if sampled:
+        st = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(STAGES))] for i in sampled])
+        stage_ms = st.mean(axis=0)
+    layer.check_status("in the timed region")
+    return dict(ms_total=ms_total, ms_step=ms_total / K, stage_ms=stage_ms, clocks=clk,
+                peak_bytes=int(torch.cuda.max_memory_allocated(layer.dev)))
+
+
+def roofline_of(layer: Layer, res: dict, peaks: dict, peak_src: str):
+    """The expert-GEMM roofline (touched weight bytes or FLOPs over the
+    kernel's event-timed duration) and the layer roofline of one timed run."""
+    from moe_layer_gemm_b200 import abi
+    wl = layer.wl
+    counts = layer.outs["counts"].cpu().numpy()
+    kept = layer.outs["kept"].cpu().numpy()
+    alg = layer_algorithmic(wl, counts, kept)
+    ms_step, stage_ms = res["ms_step"], res["stage_ms"]
+    sustained = res["ms_total"] > 1000.0
+    tensor_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    tensor_src = peak_src + (" sustained" if sustained else " burst")
+    bw = peaks["hbm_gbs"]
+    t_bytes = alg["layer_bytes"] / (bw * 1e9)
+    t_flops = alg["layer_flops"] / (tensor_peak * 1e12)
+    layer_roof = {"bound": "hbm" if t_bytes >= t_flops else "tensor", "t_roof_ms": max(t_bytes, t_flops) * 1e3,
+                  "t_meas_ms": ms_step, "frac": max(t_bytes, t_flops) * 1e3 / ms_step, "bytes": alg["layer_bytes"],
+                  "flops": alg["layer_flops"]}
+    # the expert GEMMs' own work and time; the chunked layer records no
+    # per-stage events, so there the whole layer's work over its time
+    per_stage = stage_ms is not None
+    gemm_ms = float(stage_ms[2]) if per_stage else ms_step
+    w_bytes = alg["gemm_bytes"] if per_stage else alg["layer_bytes"]
+    w_flops = alg["gemm_flops"] if per_stage else alg["layer_flops"]
+    if w_bytes / (bw * 1e9) >= w_flops / (tensor_peak * 1e12):
+        achieved = w_bytes / (gemm_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": bw, "unit": "GB/s", "frac": achieved / bw,
+                "peak_source": f"{peak_src} copy bandwidth"}
+    else:
+        achieved = w_flops / (gemm_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak, "peak_source": f"{tensor_src} bf16 GEMM"}
+    kernel = abi.moe_ffn_kernel(layer.dims)
+    traffic = profile_traffic(kernel, wl.name) if layer.chunk == 0 and wl.T == synth.get_workload(wl.name).T else None
+    roof.update({
+        "traffic": traffic,
+        "kernel": (f"{kernel} (gate/up and down in one launch)" if per_stage else
+                   f"whole chunked layer (no per-stage events; {kernel} once per chunk)"),
+        "algorithmic_per_step": w_bytes if roof["bound"] == "hbm" else w_flops,
+        "algorithmic_what": ("touched expert weights (bytes)" if roof["bound"] == "hbm" else
+                             "6 d_model d_ff N_kept (FLOPs)") if per_stage else "whole layer",
+        "design_activation_bytes": alg["gemm_design_bytes"] if per_stage else None,
+        "ms_per_step": gemm_ms})
+    routing = {"n_kept": alg["n_kept"], "experts_touched": alg["touched"],
+               "max_over_mean_load": float(counts.max() / (wl.T * wl.K / wl.E)),
+               "count_cv": float(counts.std() / counts.mean()), "n_dropped": int(layer.outs["n_dropped"].item())}
+    return roof, layer_roof, routing
+
+
+def stage_dict(stage_ms):
+    return None if stage_ms is None else {k: float(v) for k, v in zip(STAGES, stage_ms)}
+
+
+EXTRA_WORKLOADS = ("mixtral_prefill", "qwen_capacity", "deepseek_bias")
+
+
 def run_ours(args):
     from moe_layer_gemm_b200 import abi
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -289,124 +459,48 @@ def run_ours(args):
         if pg:
             torch.distributed.barrier()
 
+    peaks, peak_src = load_peaks()
     wl = synth.get_workload(args.workload)
     if args.tokens > 0:
         wl.T = args.tokens
-    dims = abi.Dims(wl.T, wl.d_model, wl.d_ff, wl.E, wl.K, wl.capacity_factor)
-    x = synth.make_x(wl, device=dev)[: wl.T].contiguous()
-    Wr = synth.make_router(wl, device=dev)
-    W1, W3, W2 = synth.make_expert_weights(wl, device=dev)
-    W13p, W2p = abi.pack_weights(dims, W1, W3, W2)
-    torch.cuda.synchronize()
-    host_w = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.tokens == 0:
-        host_w = [t.to("cpu", torch.float32) for t in (x, Wr, W1, W3, W2)]
-    del W1, W3, W2
-    torch.cuda.empty_cache()
     chunk = args.chunk_tokens
-    ws = abi.alloc_chunked_workspace(dims, chunk, dev) if chunk > 0 else abi.alloc_workspace(dims, dev)
-    y = torch.empty(wl.T, wl.d_model, dtype=torch.float32, device=dev)
-    E = wl.E
-    i32 = dict(dtype=torch.int32, device=dev)
-    outs = dict(counts=torch.zeros(E, **i32), kept=torch.zeros(E, **i32), n_dropped=torch.zeros(1, **i32),
-                f=torch.zeros(E, dtype=torch.float32, device=dev), P=torch.zeros(E, dtype=torch.float32, device=dev),
-                aux=torch.zeros(1, dtype=torch.float32, device=dev))
-    bias = torch.zeros(E, dtype=torch.float32, device=dev) if wl.use_bias else None
-    alpha = float(wl.alpha) if wl.use_bias else 0.0
-
-    def layer(x_in, y_out, evs=None):
-        if chunk > 0:   # per-stage events are not recorded by the chunked layer
-            abi.moe_layer_forward_chunked(dims, chunk, x_in, Wr, bias, alpha, W13p, W2p, y_out, ws, outs)
-        else:
-            abi.moe_layer_forward(dims, x_in, Wr, bias, alpha, W13p, W2p, y_out, ws, outs, stage_events=evs)
-
-    def step(evs=None):
-        layer(x, y, evs)
-
-    abi.moe_reset_device_status(ws)
-    for _ in range(args.warmup):
-        step()
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and args.tokens == 0
+    layer = Layer(wl, dev, chunk, keep_host=want_cpu)
+    abi.moe_reset_device_status(layer.ws)
+    for i in range(args.warmup):
+        layer.step(i)
     torch.cuda.synchronize()
-    st, detail = abi.moe_get_device_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device-side wait ran out during warm-up (code {detail})")
+    layer.check_status("during warm-up")
 
-    # ---- timed region: K steps; per-stage events recorded live on every
-    # STAGE_EVERY-th step (an event between two kernels keeps the second
-    # from starting early, so the other steps run without them)
+    # ---- timed region: K steps of the headline workload
     K = args.steps
-    nev = abi.NUM_STAGE_EVENTS
-    sampled = list(range(0, K, STAGE_EVERY)) if chunk == 0 else []
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(K)]
-    s = torch.cuda.current_stream()
-    for row in evs:      # create the underlying events before the timed region
-        for e in row:
-            e.record(s)
-    sampled_set = set(sampled)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.reset_peak_memory_stats(dev)
-    clocks = ClockSampler(local)
-    clocks.start()
-    barrier()
-    torch.cuda.synchronize()
-    start.record(s)
-    for i in range(K):
-        step(evs[i] if i in sampled_set else None)
-    end.record(s)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    ms_total = max_over_ranks(start.elapsed_time(end), dev)
-    ms_step = ms_total / K
-    peak_bytes = int(torch.cuda.max_memory_allocated(dev))
-    stage_ms = None
-    if sampled:
-        stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in sampled])
-        stage_ms = stage.mean(axis=0)
-    st, detail = abi.moe_get_device_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device-side wait ran out in the timed region (code {detail})")
+    res = time_steps(layer, K, barrier, local, start_step=args.warmup)
+    roof, layer_roof, routing = roofline_of(layer, res, peaks, peak_src)
+    ms_step = res["ms_step"]
 
-    counts = outs["counts"].cpu().numpy()
-    kept = outs["kept"].cpu().numpy()
-    alg = layer_algorithmic(wl, counts, kept)
-    peaks, peak_src = load_peaks()
-    gemm_ms = float(stage_ms[2]) if stage_ms is not None else ms_step
-    sustained = ms_total > 1000.0
-    tensor_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    bw = peaks["hbm_gbs"]
-    t_bytes = alg["layer_bytes"] / (bw * 1e9)
-    t_flops = alg["layer_flops"] / (tensor_peak * 1e12)
-    layer_bound = "hbm" if t_bytes >= t_flops else "tensor"
-    # the expert GEMMs' own work and time; the chunked layer records no
-    # per-stage events, so there the whole layer's work over its time
-    w_bytes = alg["gemm_bytes"] if stage_ms is not None else alg["layer_bytes"]
-    w_flops = alg["gemm_flops"] if stage_ms is not None else alg["layer_flops"]
-    g_bytes_t = w_bytes / (bw * 1e9)
-    g_flops_t = w_flops / (tensor_peak * 1e12)
-    if g_bytes_t >= g_flops_t:
-        achieved = w_bytes / (gemm_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": bw, "unit": "GB/s", "frac": achieved / bw}
-    else:
-        achieved = w_flops / (gemm_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": achieved / tensor_peak}
-    kernel = abi.moe_ffn_kernel(dims)
-    traffic = profile_traffic(kernel, wl.name) if chunk == 0 else None
-    what = (f"{kernel} (gate/up and down in one launch)" if chunk == 0 else
-            f"whole chunked layer (no per-stage events; {kernel} once per chunk)")
-    roof.update({"traffic": traffic, "kernel": what,
-                 "algorithmic_per_step": w_bytes if roof["bound"] == "hbm" else w_flops,
-                 "ms_per_step": gemm_ms, "peak_source": f"{peak_src}" + (" sustained" if sustained and roof["bound"] == "tensor" else "")})
+    # ---- the same workload over at least a second of steps (the power cap
+    # settles in): its own timed region and clock record
+    sustained = None
+    if not args.no_sustained and chunk == 0:
+        n_sus = max(K, int(np.ceil(1100.0 / max(ms_step, 1e-3))))
+        rs = time_steps(layer, n_sus, barrier, local, start_step=args.warmup + K)
+        r2, l2, _ = roofline_of(layer, rs, peaks, peak_src)
+        sustained = {"steps": n_sus, "ms_per_step": rs["ms_step"],
+                     "value": job_tokens_per_s(wl.T, world, rs["ms_step"]), "timed_ms": rs["ms_total"],
+                     "roofline_frac": r2["frac"], "roofline_bound": r2["bound"], "gemm_ms": r2["ms_per_step"],
+                     "layer_roofline_frac": l2["frac"], "stage_ms": stage_dict(rs["stage_ms"]),
+                     "clocks": rs["clocks"]}
 
     # ---- end to end through the public API with host buffers: every step
     # copies its input in from pinned host memory and its result y back out.
     # Two buffer sets and two copy streams pipeline the copies of one step
     # with the layer of another, as a serving loop would.
-    x_host = x.cpu().pin_memory()
+    s = torch.cuda.current_stream()
+    x0 = layer.xs[0]
+    x_host = [xx.cpu().pin_memory() for xx in layer.xs]
     y_host = [torch.empty(wl.T, wl.d_model, dtype=torch.float32).pin_memory() for _ in range(2)]
-    x_dev = [torch.empty_like(x) for _ in range(2)]
-    y_dev = [torch.empty_like(y) for _ in range(2)]
+    x_dev = [torch.empty_like(x0) for _ in range(2)]
+    y_dev = [torch.empty_like(layer.y) for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -420,11 +514,11 @@ def run_ours(args):
         b = i % 2
         s_in.wait_event(ev_done[b])          # x_dev[b] no longer read by step i - 2
         with torch.cuda.stream(s_in):
-            x_dev[b].copy_(x_host, non_blocking=True)
+            x_dev[b].copy_(x_host[i % len(x_host)], non_blocking=True)
         ev_in[b].record(s_in)
         s.wait_event(ev_in[b])
         s.wait_event(ev_out[b])               # y_dev[b] copied out by step i - 2
-        layer(x_dev[b], y_dev[b])
+        layer.run(x_dev[b], y_dev[b])
         ev_done[b].record(s)
         s_out.wait_event(ev_done[b])
         with torch.cuda.stream(s_out):
@@ -446,22 +540,51 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / E2E, dev)
-
-    if chunk > 0:
-        launches = abi.moe_layer_chunked_launch_count(dims, chunk, True, bias is not None and alpha != 0.0) * K
-    else:
-        launches = abi.moe_layer_launch_count(dims, True, bias is not None and alpha != 0.0) * K
+    layer.check_status("in the end-to-end steps")
+    launches = layer.launches() * K
 
     cpu = None
-    if host_w is not None:
+    if layer.host is not None:
         S = min(args.cpu_sample_tokens, wl.T)
         tokens = np.linspace(0, wl.T - 1, S).astype(int).tolist()
-        b32 = np.zeros(E, np.float32) if wl.use_bias else None
-        times = time_oracle(wl, *host_w, tokens, b32, steps=2)
+        b32 = np.zeros(wl.E, np.float32) if wl.use_bias else None
+        times = time_oracle(wl, *layer.host, tokens, b32, steps=2)
         sec = min(times)
         cpu = {"value": S / sec, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{S} of {wl.T} tokens (routing over all {wl.T}), best of 2 runs of {sec:.1f}-"
-                         f"{max(times):.1f} s"}
+                         f"{max(times):.1f} s; numpy fp64 with the BLAS threads given in cores"}
+    line_cfg = {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
+                "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{world}",
+                "l2": l2_note(wl), **({"chunk_tokens": chunk} if chunk > 0 else {})}
+    memory = {"workspace_bytes": int(layer.ws.numel()), "peak_device_bytes": res["peak_bytes"],
+              **({"workspace_bytes_whole_batch": abi.moe_workspace_size(layer.dims)} if chunk > 0 else {})}
+    del layer, x_host, y_host, x_dev, y_dev
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads of the metric (prefill, capacity, bias loop):
+    # same step, same timing, one entry each; 1-GPU runs only
+    extras = {}
+    if (world == 1 and not args.no_extra and args.workload == "mixtral_decode" and args.tokens == 0
+            and chunk == 0):
+        for name in EXTRA_WORKLOADS:
+            wx = synth.get_workload(name)
+            lx = Layer(wx, dev)
+            abi.moe_reset_device_status(lx.ws)
+            for i in range(args.warmup):
+                lx.step(i)
+            torch.cuda.synchronize()
+            lx.check_status(f"during warm-up ({name})")
+            rx = time_steps(lx, K, barrier, local, start_step=args.warmup)
+            rf, lr, rt = roofline_of(lx, rx, peaks, peak_src)
+            extras[name] = {"value": job_tokens_per_s(wx.T, world, rx["ms_step"]), "unit": "tokens/s",
+                            "ms_per_step": rx["ms_step"], "steps": K, "warmup": args.warmup,
+                            "config": {"T": wx.T, "d_model": wx.d_model, "d_ff": wx.d_ff, "E": wx.E, "K": wx.K,
+                                       "capacity_factor": wx.capacity_factor, "bias_update": wx.use_bias,
+                                       "fresh_tokens_per_step": len(lx.xs) > 1, "l2": l2_note(wx)},
+                            "roofline": rf, "layer_roofline": lr, "stage_ms": stage_dict(rx["stage_ms"]),
+                            "routing": rt, "clocks": rx["clocks"], "gpu_launches_per_step": lx.launches()}
+            del lx
+            torch.cuda.empty_cache()
 
     if pg:
         torch.distributed.destroy_process_group()
@@ -472,26 +595,19 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
-                   "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{world}",
-                   "l2": l2_note(wl), **({"chunk_tokens": chunk} if chunk > 0 else {})},
-        "memory": {"workspace_bytes": int(ws.numel()), "peak_device_bytes": peak_bytes,
-                   **({"workspace_bytes_whole_batch": abi.moe_workspace_size(dims)} if chunk > 0 else {})},
+        "config": line_cfg,
+        "memory": memory,
         "roofline": roof,
-        "layer_roofline": {"bound": layer_bound, "t_roof_ms": max(t_bytes, t_flops) * 1e3, "t_meas_ms": ms_step,
-                           "frac": max(t_bytes, t_flops) * 1e3 / ms_step, "bytes": alg["layer_bytes"],
-                           "flops": alg["layer_flops"]},
-        "stage_ms": None if stage_ms is None else
-                    {"route": stage_ms[0], "dispatch": stage_ms[1], "expert_gemms": stage_ms[2],
-                     "combine": stage_ms[3], "stats_bias": stage_ms[4]},
-        "routing": {"n_kept": alg["n_kept"], "experts_touched": alg["touched"],
-                    "max_over_mean_load": float(counts.max() / (wl.T * wl.K / wl.E)),
-                    "count_cv": float(counts.std() / counts.mean()), "n_dropped": int(outs["n_dropped"].item())},
+        "layer_roofline": layer_roof,
+        "stage_ms": stage_dict(res["stage_ms"]),
+        "routing": routing,
+        "sustained": sustained,
         "cpu_baseline": cpu,
         "e2e": {"value": job_tokens_per_s(wl.T, world, ms_e2e), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
+                "h2d_bytes_per_step": int(x0.numel() * 2), "d2h_bytes_per_step": int(wl.T * wl.d_model * 4)},
         "gpu_launches": launches,
-        "clocks": clk,
+        "clocks": res["clocks"],
+        "workloads": extras or None,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -81,6 +81,7 @@ enum {
     MOE_EWORKSPACE = -4,   /* workspace too small */
     MOE_ETIMEOUT = -5,     /* a device-side bounded wait ran out (from moe_get_device_status) */
     MOE_ESCRATCH = -6,     /* batch too large for the static scratch of moe_permute_noalloc */
+    MOE_EINDEX = -7,       /* a dispatch input named an expert outside [0, E) (from moe_get_device_status) */
 };
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -88,6 +89,20 @@ MOE_API const char* moe_status_str(int status);
 
 /* Library ABI version (major * 100 + minor). */
 MOE_API int moe_version(void);
+
+/* Testing the device-side timeouts (no counterpart on the source pages).
+ * Sets, for the expert-GEMM launches enqueued afterwards by this process,
+ * the poll limit of every bounded wait (wait_polls) and of the down
+ * projection's readiness wait (dependency_polls); a value <= 0 restores the
+ * default (2^26 polls, seconds), other values are clamped to [1024, 2^31].
+ * With dependency_never_ready != 0 the readiness target of every
+ * down-projection tile is made unreachable, so those waits run out: the
+ * launch ends early, with MOE_ETIMEOUT and detail 6 in the workspace status
+ * flag, after its abort and drain paths have run; its outputs are undefined.
+ * Lets a test exercise those paths without faulting or hanging anything.
+ * Process-wide and not synchronised with launches in flight on other
+ * threads: call it only between launches. */
+MOE_API int moe_test_set_wait_limits(int64_t wait_polls, int64_t dependency_polls, int dependency_never_ready);
 
 /* Capacity C of [P2] section 3.1 for these dims: -1 when there is no limit,
  * else ceil(capacity_factor * T * K / E) >= 1.  Returns < -1 on bad dims. */
@@ -101,8 +116,10 @@ MOE_API int moe_workspace_size(const moe_dims* dims, size_t* bytes);
 MOE_API int moe_reset_device_status(void* ws, void* stream);
 
 /* Read the workspace's device status flag: synchronises `stream`, then
- * *status = MOE_OK, or MOE_ETIMEOUT with *detail naming the wait that ran
- * out (a small integer; 0 if none). */
+ * *status = MOE_OK; MOE_ETIMEOUT with *detail naming the wait that ran out
+ * (a small integer, 1..6); or MOE_EINDEX (*detail = 7) when a dispatch input
+ * named an expert outside [0, E).  The first failure recorded wins; the
+ * flag stays set until moe_reset_device_status. */
 MOE_API int moe_get_device_status(const void* ws, void* stream, int* status, int* detail);
 
 /* Bytes of the packed expert weights moe_pack_weights writes for these dims:
@@ -155,7 +172,13 @@ MOE_API int moe_route_from_logits(const moe_dims* dims, const float* logits, con
 
 /* Step 3: dispatch ([P2] section 2.1: group by expert via sort and cumsum;
  * section 3.1: capacity drop).
- *   topk_idx  [T, K] int32 in
+ *   topk_idx  [T, K] int32 in: entries should lie in [0, E).  An entry
+ *             outside that range is never used as an address: its slot is
+ *             skipped (not counted, inv = -1, no row) and the workspace
+ *             status flag records MOE_EINDEX (moe_get_device_status).  The
+ *             router writes K distinct experts per token; a token that lists
+ *             an expert twice is treated as two assignments, ranked in slot
+ *             order.
  *   x         [T, d_model] bf16 in, or NULL to skip the row gather
  *   counts    [E] int32 out: selections per expert before drops
  *   kept      [E] int32 out: min(counts, C)
@@ -164,8 +187,10 @@ MOE_API int moe_route_from_logits(const moe_dims* dims, const float* logits, con
  *   src       [T*K] int32 out: token of each row (rows >= N_kept untouched)
  *   x_perm    [T*K, d_model] bf16 out (rows >= N_kept untouched), or NULL
  *   n_dropped [1] int32 out or NULL
- * The rank of (t, k) within its expert is the number of tokens t' < t that
- * chose the same expert; rows are expert-major, token-ascending. */
+ * The rank of (t, k) within its expert is the number of assignments
+ * (t', k') before it in token-major order that chose the same expert (for
+ * distinct experts per token: the tokens t' < t that chose it); rows are
+ * expert-major, token-ascending. */
 MOE_API int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x,
                 int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
                 moe_bf16* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream);
@@ -191,6 +216,13 @@ MOE_API int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe
  * the last call's contents; every value a call reads is written earlier in
  * the same call, so no clearing is needed, but calls whose work overlaps on
  * the same GPU (for example on two streams) race on it: serialise them.
+ * The looked-up address is kept for the life of the process, so do not use
+ * this entry point across a cudaDeviceReset (or any other teardown of the
+ * device's primary context) in the same process.
+ *
+ * An out-of-range expert index is skipped as in moe_permute, but with no
+ * workspace there is no status flag to record it: validate topk_idx first
+ * where it does not come from moe_route.
  *
  * There is no counterpart of this entry point on the source pages; it
  * exists for the callers described above. */

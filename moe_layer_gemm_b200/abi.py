@@ -26,6 +26,7 @@ MOE_ECUDA = -3
 MOE_EWORKSPACE = -4
 MOE_ETIMEOUT = -5
 MOE_ESCRATCH = -6
+MOE_EINDEX = -7
 
 EXPORTED = [
     "moe_status_str", "moe_version", "moe_capacity", "moe_workspace_size", "moe_reset_device_status",
@@ -33,6 +34,7 @@ EXPORTED = [
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
     "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc", "moe_ffn_kernel",
     "moe_chunked_workspace_size", "moe_layer_forward_chunked", "moe_layer_chunked_launch_count",
+    "moe_test_set_wait_limits",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -91,6 +93,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_layer_chunked_launch_count": (I, [dims_p, ctypes.c_int64, I, I]),
         "moe_layer_forward_chunked": (I, [dims_p, ctypes.c_int64, P, P, P, F, P, P, P,
                                           ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
+        "moe_test_set_wait_limits": (I, [ctypes.c_int64, ctypes.c_int64, I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -160,6 +163,13 @@ def moe_status_str(status: int) -> str:
 
 def moe_version() -> int:
     return load().moe_version()
+
+
+def moe_test_set_wait_limits(wait_polls: int = 0, dependency_polls: int = 0, dependency_never_ready: bool = False):
+    """Test-only: poll limits of the expert GEMMs' bounded waits (0 = default)
+    and an unreachable down-projection readiness target (see the header)."""
+    _check("moe_test_set_wait_limits", load().moe_test_set_wait_limits(
+        ctypes.c_int64(wait_polls), ctypes.c_int64(dependency_polls), int(bool(dependency_never_ready))))
 
 
 def moe_capacity(dims) -> int:

@@ -5,14 +5,32 @@
 #include <cstring>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "../../include/moe_b200.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 using namespace moe;
 
+namespace moe {
+
+namespace {
+std::atomic<uint32_t> g_wait_limit{0};
+std::atomic<uint32_t> g_dep_wait_limit{0};
+std::atomic<int> g_dep_never_ready{0};
+}  // namespace
+
+WaitSettings wait_settings() {
+    return WaitSettings{g_wait_limit.load(std::memory_order_relaxed), g_dep_wait_limit.load(std::memory_order_relaxed),
+                        g_dep_never_ready.load(std::memory_order_relaxed)};
+}
+
+}  // namespace moe
+
 namespace {
 
-constexpr int kVersion = 101;  // 1.01: layer outputs gained P_topk, aux_topk, z_loss; chunked layer
+constexpr int kVersion = 102;  // 1.02: MOE_EINDEX, moe_test_set_wait_limits; 1.01: P_topk, aux_topk, z_loss; chunked layer
 constexpr int64_t kMaxT = int64_t(1) << 24;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -280,6 +298,10 @@ GemmLaunch ffn_launch(const moe_dims* d, const Layout& L, const bf16* xperm, con
     p1.split_stride = A * d->d_model;
     g.status = ws ? at<int>(ws, L.status) : nullptr;
     g.sched = ws ? at<int>(ws, L.sched_ffn) : nullptr;
+    const WaitSettings wt = wait_settings();
+    g.wait_limit = wt.wait_limit;
+    g.dep_wait_limit = wt.dep_wait_limit;
+    g.dep_extra = wt.dep_never_ready ? (1 << 30) : 0;
     return g;
 }
 
@@ -314,11 +336,25 @@ const char* moe_status_str(int s) {
         case MOE_EWORKSPACE: return "MOE_EWORKSPACE: workspace too small";
         case MOE_ETIMEOUT: return "MOE_ETIMEOUT: a device-side wait ran out";
         case MOE_ESCRATCH: return "MOE_ESCRATCH: batch too large for the library's static scratch";
+        case MOE_EINDEX: return "MOE_EINDEX: a dispatch input named an expert outside [0, E); the slot was skipped";
         default: return "unknown status";
     }
 }
 
 int moe_version(void) { return kVersion; }
+
+int moe_test_set_wait_limits(int64_t wait_polls, int64_t dependency_polls, int dependency_never_ready) {
+    auto clamp = [](int64_t v) -> uint32_t {
+        if (v <= 0) return 0u;  // the default
+        if (v < 1024) return 1024u;
+        if (v > (int64_t(1) << 31)) return 1u << 31;
+        return static_cast<uint32_t>(v);
+    };
+    g_wait_limit.store(clamp(wait_polls), std::memory_order_relaxed);
+    g_dep_wait_limit.store(clamp(dependency_polls), std::memory_order_relaxed);
+    g_dep_never_ready.store(dependency_never_ready ? 1 : 0, std::memory_order_relaxed);
+    return MOE_OK;
+}
 
 int64_t moe_capacity(const moe_dims* dims) {
     if (check_dims(dims) != MOE_OK) return -2;
@@ -344,7 +380,7 @@ int moe_get_device_status(const void* ws, void* stream, int* status, int* detail
             cudaSuccess ||
         cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return MOE_ECUDA;
-    *status = host == 0 ? MOE_OK : MOE_ETIMEOUT;
+    *status = host == 0 ? MOE_OK : (host == DEV_BAD_INDEX ? MOE_EINDEX : MOE_ETIMEOUT);
     if (detail) *detail = host;
     return MOE_OK;
 }
@@ -407,12 +443,12 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x
         return map_launch(launch_dispatch_gather_small(
             topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
             counts, kept, offsets, inv, src, reinterpret_cast<bf16*>(x_perm), n_dropped, at<int32_t>(ws, L.sched_ffn),
-            static_cast<int>(gemm_sched_bytes(dims->E) / 4), static_cast<cudaStream_t>(stream)));
+            static_cast<int>(gemm_sched_bytes(dims->E) / 4), at<int>(ws, L.status), static_cast<cudaStream_t>(stream)));
     return map_launch(launch_permute(topk_idx, reinterpret_cast<const bf16*>(x), dims->T, dims->d_model, dims->E,
                                      dims->K, capacity_of(dims), at<int32_t>(ws, L.block_hist), counts, kept,
                                      offsets, inv, src, reinterpret_cast<bf16*>(x_perm), n_dropped,
                                      at<int32_t>(ws, L.sched_ffn), static_cast<int>(gemm_sched_bytes(dims->E) / 4),
-                                     static_cast<cudaStream_t>(stream)));
+                                     at<int>(ws, L.status), static_cast<cudaStream_t>(stream)));
 }
 
 int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets, const moe_bf16* W13p,
@@ -511,13 +547,14 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
         MOE_TRY(map_launch(launch_dispatch_gather_small(
             idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims), counts, kept, offsets, inv,
             at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop, at<int32_t>(ws, L.sched_ffn),
-            static_cast<int>(gemm_sched_bytes(dims->E) / 4), st)));
+            static_cast<int>(gemm_sched_bytes(dims->E) / 4), at<int>(ws, L.status), st)));
     else
         MOE_TRY(map_launch(launch_permute(idx, xb, dims->T, dims->d_model, dims->E, dims->K, capacity_of(dims),
                                           at<int32_t>(ws, L.block_hist), counts, kept, offsets, inv,
                                           at<int32_t>(ws, L.src), at<bf16>(ws, L.xperm), ndrop,
                                           at<int32_t>(ws, L.sched_ffn),
-                                          static_cast<int>(gemm_sched_bytes(dims->E) / 4), st)));
+                                          static_cast<int>(gemm_sched_bytes(dims->E) / 4), at<int>(ws, L.status),
+                                          st)));
     mark(2);
     float* yp = at<float>(ws, L.yperm);
     MOE_TRY(do_ffn(dims, L, at<bf16>(ws, L.xperm), offsets, reinterpret_cast<const bf16*>(W13p),
@@ -600,14 +637,15 @@ int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const 
                 idx_c, x_c, dc.T, dc.d_model, dc.E, dc.K, -1, cnt_c, at<int32_t>(ws, Lc.kept),
                 at<int32_t>(ws, Lc.offsets), inv_c, at<int32_t>(ws, Lc.src), at<bf16>(ws, Lc.xperm),
                 at<int32_t>(ws, Lc.ndrop), at<int32_t>(ws, Lc.sched_ffn),
-                static_cast<int>(gemm_sched_bytes(dc.E) / 4), st)));
+                static_cast<int>(gemm_sched_bytes(dc.E) / 4), at<int>(ws, Lc.status), st)));
         else
             MOE_TRY(map_launch(launch_permute(idx_c, x_c, dc.T, dc.d_model, dc.E, dc.K, -1,
                                               at<int32_t>(ws, Lc.block_hist), cnt_c, at<int32_t>(ws, Lc.kept),
                                               at<int32_t>(ws, Lc.offsets), inv_c, at<int32_t>(ws, Lc.src),
                                               at<bf16>(ws, Lc.xperm), at<int32_t>(ws, Lc.ndrop),
                                               at<int32_t>(ws, Lc.sched_ffn),
-                                              static_cast<int>(gemm_sched_bytes(dc.E) / 4), st)));
+                                              static_cast<int>(gemm_sched_bytes(dc.E) / 4), at<int>(ws, Lc.status),
+                                              st)));
         float* yp = at<float>(ws, Lc.yperm);
         MOE_TRY(do_ffn(&dc, Lc, at<bf16>(ws, Lc.xperm), at<int32_t>(ws, Lc.offsets),
                        reinterpret_cast<const bf16*>(W13p), reinterpret_cast<const bf16*>(W2p),

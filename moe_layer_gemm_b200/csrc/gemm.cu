@@ -76,6 +76,9 @@ struct DevArgs {
     uint32_t wslot, xslot;      // bytes per weight / token slot
     int* status;
     int* sched;         // [0] tile counter, [1..G] phase-0 tiles done per group (x4 warps)
+    uint32_t wait_limit;      // polls of a bounded mbarrier or drain wait
+    uint32_t dep_wait_limit;  // polls of the phase-1 readiness wait
+    int dep_extra;            // added to the phase-1 readiness target (0; a test makes it unreachable)
 };
 
 struct Maps {
@@ -273,35 +276,35 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             // ------------------------------------------- scheduler + producer
             const uint64_t pol_first = policy_evict_first();
             const uint64_t pol_last = policy_evict_last();
-                    uint32_t s = 0, ph = 0, r = 0, rph = 0;
+            uint32_t s = 0, ph = 0, r = 0, rph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool ok = true;
-            bool sent_end = false;
             // claims run one tile ahead so the atomic's round trip overlaps
             // the loads of the current tile
             int next = atomicAdd(&a.sched[0], 1);
             while (ok) {
                 const int tile = next < total ? next : -1;
                 if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
-                if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, a.wait_limit)) {
                     ok = false;
                     break;
                 }
                 ring[r] = tile;
                 mbar_arrive(&rfull[r]);
                 if (++r == kRing) { r = 0; rph ^= 1u; }
-                if (tile < 0) {
-                    sent_end = true;
-                    break;
-                }
+                if (tile < 0) break;  // the end marker
                 const Tile t = decode_tile(a, tile, tstart, off);
                 const PhaseArgs& pa = a.ph[t.phase];
                 if (t.phase == 1 && a.dep) {
                     // all phase-0 tiles of this group must have stored their rows
-                    const int need = 4 * (tstart[t.g + 1] - tstart[t.g]);
+                    const int need = 4 * (tstart[t.g + 1] - tstart[t.g]) + a.dep_extra;
                     uint32_t i = 0;
                     while (ld_acquire(&a.sched[1 + t.g]) < need) {
-                        if (++i > kWaitLimit || *abort_flag) {
+                        if (*abort_flag) {
+                            ok = false;
+                            break;
+                        }
+                        if (++i > a.dep_wait_limit) {
                             atomicCAS(a.status, 0, DEV_TIMEOUT_DEPENDENCY);
                             *abort_flag = 1;
                             ok = false;
@@ -316,7 +319,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 const uint32_t wbytes = t.swap ? 16384u : static_cast<uint32_t>(pa.BN) * 128u;
                 const uint32_t xbytes = t.swap ? static_cast<uint32_t>(nb) * 4096u : kTileABytes;
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -348,18 +351,13 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
             }
-            if (!sent_end) {
-                // a failed wait: hand the consumers the end marker (bounded)
-                for (uint32_t i = 0; i < kWaitLimit; ++i)
-                    if (mbar_try_wait(&rempty[r], rph ^ 1u)) break;
-                ring[r] = -1;
-                mbar_arrive(&rfull[r]);
-            }
-            // Drain: every issued copy has landed before the CTA may exit.
+            // Leaving without the end marker means a wait failed and raised the
+            // abort flag, which every consumer's wait watches, so none needs it.
+            // Drain: every issued copy has landed before the CTA may exit.  A
+            // stage is armed and its copies issued together, so each armed
+            // stage's last phase completes once those copies land.
             for (int i = 0; i < S; ++i)
-                if (issued_mask & (1u << i))
-                    for (uint32_t it = 0; it < kWaitLimit; ++it)
-                        if (mbar_try_wait(&full[i], (issued_ph >> i) & 1u)) break;
+                if (issued_mask & (1u << i)) mbar_drain(&full[i], (issued_ph >> i) & 1u, a.status, DEV_TIMEOUT_DRAIN, a.wait_limit);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -368,7 +366,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             int it = 0;
             bool ok = true;
             while (ok) {
-                if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) break;
+                if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag, a.wait_limit)) break;
                 const int tile = ring[r];
                 mbar_arrive(&rempty[r]);
                 if (++r == kRing) { r = 0; rph ^= 1u; }
@@ -377,14 +375,15 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 const int buf = it & 1;
                 const uint32_t use = static_cast<uint32_t>(it >> 1);
                 ++it;
-                if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) break;
+                if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag, a.wait_limit))
+                    break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
                 const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 31) / 32) * 32u
                                               : static_cast<uint32_t>(a.ph[t.phase].BN);
                 const uint32_t idesc = umma_idesc_bf16(128, n_mma);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
+                    if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -404,8 +403,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             }
             // All issued MMAs complete before TMEM is released.
             umma_commit(drain);
-            for (uint32_t i = 0; i < kWaitLimit; ++i)
-                if (mbar_try_wait(drain, 0)) break;
+            mbar_drain(drain, 0, a.status, DEV_TIMEOUT_DRAIN, a.wait_limit);
         }
     } else {
         // ---------------------------------------------------- epilogue
@@ -413,7 +411,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         uint32_t r = 0, rph = 0;
         int it = 0;
         for (;;) {
-            if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag, a.wait_limit)) break;
             const int tile = ring[r];
             __syncwarp();
             if (lane == 0) mbar_arrive(&rempty[r]);
@@ -424,7 +422,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             const int buf = it & 1;
             const uint32_t use = static_cast<uint32_t>(it >> 1);
             ++it;
-            if (!mbar_wait(&tfull[buf], use & 1u, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            if (!mbar_wait(&tfull[buf], use & 1u, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag, a.wait_limit)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf) * 256u +
                                    (static_cast<uint32_t>(q * 32) << 16);
@@ -568,6 +566,9 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
     a.dep = (L.nphase == 2) ? 1 : 0;
     a.status = L.status;
     a.sched = L.sched;
+    a.wait_limit = L.wait_limit ? L.wait_limit : kWaitLimit;
+    a.dep_wait_limit = L.dep_wait_limit ? L.dep_wait_limit : kWaitLimit;
+    a.dep_extra = L.dep_extra;
     const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
     a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
     {

@@ -36,6 +36,19 @@
 //   ring       the leader claims tiles and writes them into both CTAs' rings;
 //              the pair's 10 consumers free a slot on the leader's rempty
 // Every wait is bounded.  No TMA multicast is used.
+//
+// Failure handling.  A wait that runs out records its code in the status
+// word and raises the abort flag of BOTH CTAs (the peer's by a store into
+// its shared memory), so every role of the pair stops within one poll
+// interval.  Before the pair passes its final cluster barrier, every copy
+// either CTA issued must have landed.  The peer's copies complete on the
+// leader's full[] barriers, which the leader alone arms, so the leader
+// reconciles with the peer: once its producer stops, the peer reports how
+// many stage uses it issued and their byte counts; the leader arms the uses
+// the peer issued beyond its own (expecting the peer's bytes only),
+// completes by hand the peer's half of the uses it armed that the peer never
+// issued, and then waits for every stage's last phase.  The MMA issuer waits
+// for its last MMAs before TMEM is freed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -78,6 +91,19 @@ struct Args2 {
     uint32_t xoff;         // weight-major tiles: offset of the token rows in a stage
     int* status;
     int* sched;
+    uint32_t wait_limit;      // polls of a bounded mbarrier or drain wait
+    uint32_t dep_wait_limit;  // polls of the phase-1 readiness wait
+    int dep_extra;            // added to the phase-1 readiness target (0; a test makes it unreachable)
+};
+
+constexpr int kMaxStages = 16;
+// The peer's report to the leader at the end of its producer loop (in the
+// leader's shared memory): stage uses issued, done flag, and the bytes of
+// its last use of each stage.
+struct PeerReport {
+    uint32_t uses;
+    uint32_t done;
+    uint32_t bytes[kMaxStages];
 };
 
 struct Maps2 {
@@ -115,6 +141,12 @@ __device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
 __device__ __forceinline__ void remote_store(uint32_t cluster_addr, int v) {
     asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t ld_acquire_cluster(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 // TMA tile load into this CTA's shared memory, completing on the leader's barrier.
 __device__ __forceinline__ void tma_load_pair(const CUtensorMap* map, void* smem_dst, uint32_t leader_bar, int32_t x,
                                               int32_t y, uint64_t policy) {
@@ -138,6 +170,16 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
                  ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3))
                  : "memory");
+}
+
+// A bounded wait whose failure (its own, or an abort seen) also raises the
+// other CTA's abort flag.
+__device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, const Args2& a, int code,
+                                      volatile int* abort_flag, uint32_t peer_abort) {
+    if (mbar_wait(bar, parity, a.status, code, abort_flag, a.wait_limit)) return true;
+    *abort_flag = 1;
+    remote_store(peer_abort, 1);
+    return false;
 }
 
 __device__ __forceinline__ bool swaps2(const Args2& a, int64_t rows) { return rows <= a.swap_max_rows; }
@@ -220,6 +262,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int64_t* off = reinterpret_cast<int64_t*>(tmem_slot + 2);
     int* tstart = reinterpret_cast<int*>(off + a.G + 1);
+    PeerReport* report = reinterpret_cast<PeerReport*>(tstart + 2 * (a.G + 1));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -242,6 +285,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
+        report->uses = 0;
+        report->done = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0)
@@ -293,6 +338,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     const uint32_t leader_rempty0 = mapa_shared(smem_u32(rempty), 0);
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(tempty), 0);
     const uint32_t leader_full0 = mapa_shared(smem_u32(full), 0);
+    const uint32_t peer_abort = mapa_shared(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -301,8 +347,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             const uint64_t pol_last = policy_evict_last();
             uint32_t s = 0, ph = 0, r = 0, rph = 0;
             bool ok = true;
-            bool sent_end = false;
-            uint32_t issued_mask = 0, issued_ph = 0;  // stages armed by the leader, and their phase
+            uint32_t uses = 0;                 // stage uses this CTA issued (armed, on the leader)
+            uint32_t use_bytes[kMaxStages];    // bytes of the pair's (leader) or own (peer) last use per stage
             int next = leader ? atomicAdd(&a.sched[0], 1) : 0;
             const uint32_t peer_ring = mapa_shared(smem_u32(ring), 1);
             const uint32_t peer_rfull = mapa_shared(smem_u32(rfull), 1);
@@ -311,7 +357,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 if (leader) {
                     tile = next < total ? next : -1;
                     if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
-                    if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                    if (!pwait(&rempty[r], rph ^ 1u, a, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, peer_abort)) {
                         ok = false;
                         break;
                     }
@@ -320,7 +366,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     mbar_arrive(&rfull[r]);
                     remote_arrive(peer_rfull + 8u * r);
                 } else {
-                    if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
+                    if (!pwait(&rfull[r], rph, a, DEV_TIMEOUT_MMA_FULL, abort_flag, peer_abort)) {
                         ok = false;
                         break;
                     }
@@ -328,19 +374,21 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     remote_arrive(leader_rempty0 + 8u * r);
                 }
                 if (++r == kRing) { r = 0; rph ^= 1u; }
-                if (tile < 0) {
-                    sent_end = true;
-                    break;
-                }
+                if (tile < 0) break;  // the end marker
                 const Tile2 t = decode2(a, tile, tstart, off);
                 const Phase2& pa = a.ph[t.phase];
                 if (t.phase == 1 && a.dep) {
-                    const int need = 8 * (tstart[t.g + 1] - tstart[t.g]);
+                    const int need = 8 * (tstart[t.g + 1] - tstart[t.g]) + a.dep_extra;
                     uint32_t i = 0;
                     while (ld_acquire2(&a.sched[1 + t.g]) < need) {
-                        if (++i > kWaitLimit || *abort_flag) {
+                        if (*abort_flag) {
+                            ok = false;
+                            break;
+                        }
+                        if (++i > a.dep_wait_limit) {
                             atomicCAS(a.status, 0, DEV_TIMEOUT_DEPENDENCY);
                             *abort_flag = 1;
+                            remote_store(peer_abort, 1);
                             ok = false;
                             break;
                         }
@@ -355,10 +403,11 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 // this CTA holds N / 2 of them (a multiple of 8), loaded in 16-row boxes
                 const int half = t.swap ? ((t.rows + 15) / 16) * 8 : 0;
                 const int nb16 = (half + 15) / 16;
+                // each CTA loads exactly half of the pair's bytes
                 const uint32_t pair_bytes =
                     t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(nb16) * 2048u) : 4u * kHalf;
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag)) {
+                    if (!pwait(&empty[s], ph ^ 1u, a, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, peer_abort)) {
                         ok = false;
                         break;
                     }
@@ -379,28 +428,64 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                             tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + j * 2048, bar, kb * kBK,
                                           static_cast<int32_t>(trow + 16 * j), pol_last);
                     }
-                    issued_mask |= 1u << s;
-                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+                    use_bytes[s] = leader ? pair_bytes : pair_bytes / 2u;
+                    ++uses;
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
             }
-            if (leader && !sent_end) {
-                // a failed wait: hand every consumer the end marker (bounded)
-                for (uint32_t i = 0; i < kWaitLimit; ++i)
-                    if (mbar_try_wait(&rempty[r], rph ^ 1u)) break;
-                ring[r] = -1;
-                remote_store(peer_ring + 4u * r, -1);
-                mbar_arrive(&rfull[r]);
-                remote_arrive(peer_rfull + 8u * r);
-            }
-            // Drain (leader): every stage's copies, the peer's included (they
-            // complete on the leader's barrier), have landed before the pair
-            // may pass its final cluster barrier and exit.  Bounded.
-            if (leader)
+            if (!leader) {
+                // report to the leader: this CTA issues no more copies
+                const uint32_t rep = mapa_shared(smem_u32(report), 0);
+                remote_store(rep, static_cast<int>(uses));
                 for (int i = 0; i < S; ++i)
-                    if (issued_mask & (1u << i))
-                        for (uint32_t it = 0; it < kWaitLimit; ++it)
-                            if (mbar_try_wait(&full[i], (issued_ph >> i) & 1u)) break;
+                    remote_store(rep + 8u + 4u * i, static_cast<int>(use_bytes[i]));
+                fence_cluster();
+                remote_store(rep + 4u, 1);
+            } else {
+                // Drain (leader): reconcile with the peer's report, then wait
+                // for every stage's last phase, so that no copy of either CTA
+                // is in flight when the pair passes its final cluster barrier.
+                bool have = false;
+                for (uint32_t i = 0; i < a.wait_limit; ++i) {
+                    if (ld_acquire_cluster(&report->done) != 0u) {
+                        have = true;
+                        break;
+                    }
+                    if (i > 64) __nanosleep(128);
+                }
+                fence_cluster();
+                uint32_t last = uses;  // stage uses whose phases are armed
+                if (!have) {
+                    atomicCAS(a.status, 0, DEV_TIMEOUT_DRAIN);
+                    *abort_flag = 1;
+                    remote_store(peer_abort, 1);
+                } else {
+                    const uint32_t np = report->uses;
+                    if (np > uses && np - uses <= static_cast<uint32_t>(S)) {
+                        // uses the peer issued and the leader never armed: arm them
+                        // for the peer's bytes alone
+                        for (uint32_t u = uses; u < np; ++u) {
+                            const uint32_t st = u % static_cast<uint32_t>(S);
+                            mbar_arrive_expect_tx(&full[st], report->bytes[st]);
+                        }
+                        last = np;
+                    } else if (np < uses && uses - np <= static_cast<uint32_t>(S)) {
+                        // uses the leader armed that the peer never issued: the
+                        // peer's half will not arrive, complete it by hand
+                        for (uint32_t u = np; u < uses; ++u) {
+                            const uint32_t st = u % static_cast<uint32_t>(S);
+                            mbar_complete_tx(&full[st], use_bytes[st] / 2u);
+                        }
+                    } else if (np != uses) {
+                        atomicCAS(a.status, 0, DEV_TIMEOUT_DRAIN);  // inconsistent report: drain what is known
+                    }
+                }
+                // the last armed phase of every stage (use u of stage u % S has parity (u / S) & 1)
+                const uint32_t first = last > static_cast<uint32_t>(S) ? last - static_cast<uint32_t>(S) : 0u;
+                for (uint32_t u = first; u < last; ++u)
+                    mbar_drain(&full[u % static_cast<uint32_t>(S)], (u / static_cast<uint32_t>(S)) & 1u, a.status,
+                               DEV_TIMEOUT_DRAIN, a.wait_limit);
+            }
         }
     } else if (warp == 1) {
         if (leader && lane == 0) {
@@ -409,7 +494,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             int it = 0;
             bool ok = true;
             while (ok) {
-                if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) break;
+                if (!pwait(&rfull[r], rph, a, DEV_TIMEOUT_MMA_FULL, abort_flag, peer_abort)) break;
                 const int tile = ring[r];
                 mbar_arrive(&rempty[r]);
                 if (++r == kRing) { r = 0; rph ^= 1u; }
@@ -418,13 +503,13 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 const int buf = it & 1;
                 const uint32_t use = static_cast<uint32_t>(it >> 1);
                 ++it;
-                if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, a.status, DEV_TIMEOUT_MMA_TEMPTY, abort_flag)) break;
+                if (!pwait(&tempty[buf], (use & 1u) ^ 1u, a, DEV_TIMEOUT_MMA_TEMPTY, abort_flag, peer_abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
                 const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 15) / 16) * 16u : 256u;
                 const uint32_t idesc = umma_idesc_bf16(256, n_mma);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!mbar_wait(&full[s], ph, a.status, DEV_TIMEOUT_MMA_FULL, abort_flag)) {
+                    if (!pwait(&full[s], ph, a, DEV_TIMEOUT_MMA_FULL, abort_flag, peer_abort)) {
                         ok = false;
                         break;
                     }
@@ -450,10 +535,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 }
                 if (ok) umma_commit_pair(&tfull[buf]);
             }
+            // all issued MMAs (into both CTAs' TMEM) complete before TMEM is freed
             asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          ::"r"(smem_u32(drain)) : "memory");
-            for (uint32_t i = 0; i < kWaitLimit; ++i)
-                if (mbar_try_wait(drain, 0)) break;
+            mbar_drain(drain, 0, a.status, DEV_TIMEOUT_DRAIN, a.wait_limit);
         }
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
@@ -461,7 +546,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
         uint32_t r = 0, rph = 0;
         int it = 0;
         for (;;) {
-            if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            if (!pwait(&rfull[r], rph, a, DEV_TIMEOUT_EPI_TFULL, abort_flag, peer_abort)) break;
             const int tile = ring[r];
             __syncwarp();
             if (lane == 0) remote_arrive(leader_rempty0 + 8u * r);
@@ -472,7 +557,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             const int buf = it & 1;
             const uint32_t use = static_cast<uint32_t>(it >> 1);
             ++it;
-            if (!mbar_wait(&tfull[buf], use & 1u, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag)) break;
+            if (!pwait(&tfull[buf], use & 1u, a, DEV_TIMEOUT_EPI_TFULL, abort_flag, peer_abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(buf) * 256u + (static_cast<uint32_t>(q * 32) << 16);
             float v[32];
@@ -598,6 +683,9 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     a.dep = L.nphase == 2 ? 1 : 0;
     a.status = L.status;
     a.sched = L.sched;
+    a.wait_limit = L.wait_limit ? L.wait_limit : kWaitLimit;
+    a.dep_wait_limit = L.dep_wait_limit ? L.dep_wait_limit : kWaitLimit;
+    a.dep_extra = L.dep_extra;
     const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
     a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
     {
@@ -640,8 +728,8 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         const uint64_t wrows = static_cast<uint64_t>(L.G) * ph.nb * ph.k_blocks * 128;
         if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
     }
-    const size_t fixed = 1024 + static_cast<size_t>(2 * 16 + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
-                         static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + 64;
+    const size_t fixed = 1024 + static_cast<size_t>(2 * kMaxStages + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
+                         static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + sizeof(PeerReport) + 64;
     // stage: token-major tiles need 2 x 16 KB; weight-major tiles wt x 16 KB
     // of weights and BNs / 2 token rows
     int wt_max = 1;
@@ -654,7 +742,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     }
     a.stage_bytes = stage_bytes;
     int stages = static_cast<int>((227 * 1024 - fixed) / stage_bytes);
-    if (stages > 16) stages = 16;
+    if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return -2;
     a.stages = stages;
     const size_t smem = fixed + static_cast<size_t>(stages) * stage_bytes;

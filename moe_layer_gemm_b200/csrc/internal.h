@@ -79,7 +79,21 @@ struct GemmLaunch {
     GemmPhase ph[2];
     int* status;             // device status word
     int* sched;              // gemm_sched_bytes(G) bytes, zero at launch
+    // Bounded waits (0 = the default limit of ptx.cuh), and a value added to
+    // the phase-1 readiness target (0 in production; a test of the timeout
+    // paths makes the target unreachable).
+    uint32_t wait_limit = 0;
+    uint32_t dep_wait_limit = 0;
+    int dep_extra = 0;
 };
+
+// Test-only settings of the expert-GEMM launches (see moe_test_set_wait_limits
+// in the header); all zero in production.
+struct WaitSettings {
+    uint32_t wait_limit, dep_wait_limit;
+    int dep_never_ready;
+};
+WaitSettings wait_settings();
 
 size_t gemm_sched_bytes(int G);
 // CTA-pair (cta_group::2) kernel: 256-wide tiles, so both phases' widths
@@ -107,7 +121,7 @@ int permute_blocks(int64_t T);
 int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                    int32_t* block_hist, int32_t* counts, int32_t* kept, int32_t* offsets,
                    int32_t* inv, int32_t* src, bf16* x_perm, int32_t* n_dropped, int32_t* zero_out,
-                   int zero_count, cudaStream_t st);
+                   int zero_count, int* status, cudaStream_t st);
 
 // ------------------------------------------------------------ combine / stats
 // Work folded into the combine launch as one extra CTA: the load statistics
@@ -147,7 +161,7 @@ bool dispatch_gather_fused_supported(int64_t T, int E, int K);
 int launch_dispatch_gather_small(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                                  int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
                                  bf16* x_perm, int32_t* n_dropped, int32_t* zero_out, int zero_count,
-                                 cudaStream_t st);
+                                 int* status, cudaStream_t st);
 int64_t permute_static_max_hist();
 int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                           int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,

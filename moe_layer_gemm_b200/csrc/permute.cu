@@ -6,12 +6,20 @@
 // offsets; section 3.1: an expert keeps at most C = CF * T * K / E
 // assignments and the overflow is dropped.
 //
-// The rank of (t, k) on expert e is the number of earlier tokens that chose
-// e.  It is assembled from three exact integer counts, never from the order
-// in which atomics happen to land:
+// The rank of (t, k) on expert e is the number of assignments (t', k')
+// before it in token-major order that chose e: the earlier tokens that chose
+// e, plus the earlier slots of the same token if it lists e more than once
+// (the router never does; such a token is treated as separate assignments).
+// It is assembled from exact integer counts, never from the order in which
+// atomics happen to land:
 //   base of the block (earlier blocks)  + earlier warps of the block
-//   + earlier lanes of the warp (one __match_any_sync per slot).
+//   + earlier lanes of the warp (one __match_any_sync per slot)
+//   + earlier slots of the same token.
 // Kept iff rank < C; row = offsets[e] + rank.
+//
+// An index outside [0, E) is never used as an address: the slot is skipped
+// (not counted, inv = -1) and DEV_BAD_INDEX is recorded in the status word
+// when the caller passed one.
 //
 // Batches of at most kSmallT tokens take one fused single-CTA kernel
 // (count, scan, rank); larger ones take hist -> scan -> rank over many CTAs.
@@ -42,10 +50,24 @@ struct WarpTable {
     int* tag;        // [E]
 };
 
+// Expert of slot (t, k), or -1 (and the status recorded) when the caller's
+// index lies outside [0, E).
+__device__ __forceinline__ int checked_expert(const int32_t* idx, int64_t i, int E, int* status) {
+    const int e = idx[i];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) return e;
+    if (status) atomicCAS(status, 0, DEV_BAD_INDEX);
+    return -1;
+}
+
+// pre[k] = slots of earlier lanes of the warp, and earlier slots of this
+// lane, that chose my[k] (slots with my[k] < 0 are ignored).
 __device__ __forceinline__ void warp_prefix(const int (&my)[kMaxK], int K, int lane, WarpTable tab, int gen,
                                             int (&pre)[kMaxK]) {
     const unsigned lt = (1u << lane) - 1u;
-    for (int k = 0; k < K; ++k) pre[k] = 0;
+    for (int k = 0; k < K; ++k) {
+        pre[k] = 0;
+        for (int k2 = 0; k2 < k; ++k2) pre[k] += (my[k2] == my[k]) ? 1 : 0;
+    }
     for (int k2 = 0; k2 < K; ++k2) {
         const int v = my[k2];
         const unsigned m = __match_any_sync(0xffffffffu, v);
@@ -63,13 +85,17 @@ __device__ __forceinline__ void warp_prefix(const int (&my)[kMaxK], int K, int l
 }
 
 __global__ void __launch_bounds__(kTokPerBlock)
-hist_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int32_t* __restrict__ block_hist) {
+hist_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int32_t* __restrict__ block_hist,
+            int* __restrict__ status) {
     __shared__ int32_t h[kMaxE];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kTokPerBlock + threadIdx.x;
     if (t < T)
-        for (int k = 0; k < K; ++k) atomicAdd(&h[idx[t * K + k]], 1);  // integer counts: order-free
+        for (int k = 0; k < K; ++k) {
+            const int e = checked_expert(idx, t * K + k, E, status);
+            if (e >= 0) atomicAdd(&h[e], 1);  // integer counts: order-free
+        }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) block_hist[static_cast<int64_t>(blockIdx.x) * E + e] = h[e];
 }
@@ -125,7 +151,7 @@ scan_kernel(int32_t* __restrict__ block_hist, int nblocks, int E, int64_t C, int
 __global__ void __launch_bounds__(kTokPerBlock)
 rank_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int64_t C,
             const int32_t* __restrict__ block_base, const int32_t* __restrict__ offsets,
-            int32_t* __restrict__ inv, int32_t* __restrict__ src) {
+            int32_t* __restrict__ inv, int32_t* __restrict__ src, int* __restrict__ status) {
     constexpr int W = kTokPerBlock / 32;
     __shared__ int32_t wh[W][kMaxE];
     __shared__ unsigned tmask[W][kMaxE];
@@ -140,8 +166,8 @@ rank_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int64_t C,
     __syncthreads();
     int my[kMaxK];
     for (int k = 0; k < K; ++k) {
-        my[k] = live ? idx[t * K + k] : -1;
-        if (live) atomicAdd(&wh[warp][my[k]], 1);
+        my[k] = live ? checked_expert(idx, t * K + k, E, status) : -1;
+        if (my[k] >= 0) atomicAdd(&wh[warp][my[k]], 1);
     }
     int pre[kMaxK];
     warp_prefix(my, K, lane, WarpTable{tmask[warp], tag[warp]}, 1, pre);
@@ -149,6 +175,10 @@ rank_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int64_t C,
     if (!live) return;
     for (int k = 0; k < K; ++k) {
         const int e = my[k];
+        if (e < 0) {
+            inv[t * K + k] = -1;
+            continue;
+        }
         int32_t r = block_base[static_cast<int64_t>(blockIdx.x) * E + e] + pre[k];
         for (int w2 = 0; w2 < warp; ++w2) r += wh[w2][e];
         if (C < 0 || r < C) {
@@ -166,7 +196,7 @@ __global__ void __launch_bounds__(kSmallThreads)
 dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int E, int K, int64_t C,
                       int32_t* __restrict__ counts, int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
                       int32_t* __restrict__ inv, int32_t* __restrict__ src, int32_t* __restrict__ n_dropped,
-                      int32_t* __restrict__ zero_out, int zero_count) {
+                      int32_t* __restrict__ zero_out, int zero_count, int* __restrict__ status) {
     constexpr int W = kSmallThreads / 32;
     for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_out[i] = 0;  // next kernel's scheduler words
     extern __shared__ int32_t sm[];
@@ -184,8 +214,8 @@ dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int E, int K, int6
     __syncthreads();
     int my[kMaxK];
     for (int k = 0; k < K; ++k) {
-        my[k] = live ? idx[t * K + k] : -1;
-        if (live) atomicAdd(&wh[warp * E + my[k]], 1);
+        my[k] = live ? checked_expert(idx, static_cast<int64_t>(t) * K + k, E, status) : -1;
+        if (my[k] >= 0) atomicAdd(&wh[warp * E + my[k]], 1);
     }
     int pre[kMaxK];
     warp_prefix(my, K, lane, WarpTable{tmask + warp * E, tag + warp * E}, 1, pre);
@@ -231,6 +261,10 @@ dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int E, int K, int6
     if (!live) return;
     for (int k = 0; k < K; ++k) {
         const int e = my[k];
+        if (e < 0) {
+            inv[t * K + k] = -1;
+            continue;
+        }
         int r = pre[k];
         for (int w2 = 0; w2 < warp; ++w2) r += wh[w2 * E + e];
         if (C < 0 || r < C) {
@@ -297,7 +331,8 @@ dispatch_gather_small_kernel(const int32_t* __restrict__ idx, const __nv_bfloat1
                              int E, int K, int64_t C, int parts, int32_t* __restrict__ counts,
                              int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ inv,
                              int32_t* __restrict__ src, int32_t* __restrict__ n_dropped,
-                             __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ zero_out, int zero_count) {
+                             __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ zero_out, int zero_count,
+                             int* __restrict__ status) {
     pdl_trigger();
     pdl_wait();
     constexpr int W = kSmallThreads / 32;
@@ -320,8 +355,8 @@ dispatch_gather_small_kernel(const int32_t* __restrict__ idx, const __nv_bfloat1
     __syncthreads();
     int my[kMaxK];
     for (int k = 0; k < K; ++k) {
-        my[k] = live ? idx[t * K + k] : -1;
-        if (live) atomicAdd(&wh[warp * E + my[k]], 1);
+        my[k] = live ? checked_expert(idx, static_cast<int64_t>(t) * K + k, E, status) : -1;
+        if (my[k] >= 0) atomicAdd(&wh[warp * E + my[k]], 1);
     }
     int pre[kMaxK];
     warp_prefix(my, K, lane, WarpTable{tmask + warp * E, tag + warp * E}, 1, pre);
@@ -370,8 +405,9 @@ dispatch_gather_small_kernel(const int32_t* __restrict__ idx, const __nv_bfloat1
         for (int k = 0; k < K; ++k) {
             const int e = my[k];
             int r = pre[k];
-            for (int w2 = 0; w2 < warp; ++w2) r += wh[w2 * E + e];
-            const int row = (C < 0 || r < C) ? soff[e] + r : -1;
+            if (e >= 0)
+                for (int w2 = 0; w2 < warp; ++w2) r += wh[w2 * E + e];
+            const int row = (e >= 0 && (C < 0 || r < C)) ? soff[e] + r : -1;
             srow[t * K + k] = row;
             if (writer) {
                 inv[t * K + k] = row;
@@ -417,7 +453,7 @@ int permute_blocks(int64_t T) { return static_cast<int>((T + kTokPerBlock - 1) /
 int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                    int32_t* block_hist, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv,
                    int32_t* src, bf16* x_perm, int32_t* n_dropped, int32_t* zero_out, int zero_count,
-                   cudaStream_t st) {
+                   int* status, cudaStream_t st) {
     if (E > kMaxE || K > kMaxK) return -2;
     if (T <= kSmallT) {
         const size_t smem = static_cast<size_t>(3 * (kSmallThreads / 32) * E + E + 1) * 4;
@@ -426,13 +462,14 @@ int launch_permute(const int32_t* idx, const bf16* x, int64_t T, int d, int E, i
                            (3 * (kSmallThreads / 32) * kMaxE + kMaxE + 1) * 4, attr_done) != 0)
             return -3;
         dispatch_small_kernel<<<1, kSmallThreads, smem, st>>>(idx, static_cast<int>(T), E, K, C, counts, kept,
-                                                              offsets, inv, src, n_dropped, zero_out, zero_count);
+                                                              offsets, inv, src, n_dropped, zero_out, zero_count,
+                                                              status);
     } else {
         const int nb = permute_blocks(T);
-        hist_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, block_hist);
+        hist_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, block_hist, status);
         scan_kernel<<<1, 1024, 0, st>>>(block_hist, nb, E, C, counts, kept, offsets, n_dropped, zero_out,
                                         zero_count);
-        rank_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, C, block_hist, offsets, inv, src);
+        rank_kernel<<<nb, kTokPerBlock, 0, st>>>(idx, T, E, K, C, block_hist, offsets, inv, src, status);
     }
     if (x != nullptr && x_perm != nullptr) {
         const int sms = num_sms() > 0 ? num_sms() : 148;
@@ -454,7 +491,7 @@ bool dispatch_gather_fused_supported(int64_t T, int E, int K) { return T <= kSma
 int launch_dispatch_gather_small(const int32_t* idx, const bf16* x, int64_t T, int d, int E, int K, int64_t C,
                                  int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* inv, int32_t* src,
                                  bf16* x_perm, int32_t* n_dropped, int32_t* zero_out, int zero_count,
-                                 cudaStream_t st) {
+                                 int* status, cudaStream_t st) {
     if (!dispatch_gather_fused_supported(T, E, K) || !x || !x_perm || d % 8 != 0) return -2;
     const size_t smem = static_cast<size_t>(3 * (kSmallThreads / 32) * E + E + 1 + T * K) * 4;
     static std::atomic<unsigned long long> attr_done{0};
@@ -470,7 +507,7 @@ int launch_dispatch_gather_small(const int32_t* idx, const bf16* x, int64_t T, i
     const int grid = static_cast<int>(need < sms ? (need < 1 ? 1 : need) : sms);
     (void)launch_pdl(dispatch_gather_small_kernel, dim3(grid), dim3(kSmallThreads), smem, st, idx, x,
                      static_cast<int>(T), d, E, K, C, parts, counts, kept, offsets, inv, src, n_dropped, x_perm,
-                     zero_out, zero_count);
+                     zero_out, zero_count, status);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
@@ -519,7 +556,7 @@ int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, i
     int32_t* scratch = dispatch_scratch_address();
     if (scratch == nullptr) return -3;
     return launch_permute(idx, x, T, d, E, K, C, scratch, counts, kept, offsets, inv, src, x_perm, n_dropped,
-                          nullptr, 0, st);
+                          nullptr, 0, nullptr, st);
 }
 
 }  // namespace moe

@@ -18,9 +18,12 @@ enum : int {
     DEV_TIMEOUT_EPI_TFULL = 4,
     DEV_TIMEOUT_DRAIN = 5,
     DEV_TIMEOUT_DEPENDENCY = 6,
+    DEV_BAD_INDEX = 7,  // a dispatch input named an expert outside [0, E); the slot was skipped
 };
 
-// About a few seconds of polling on a B200 before a wait gives up.
+// Default poll limit of a bounded wait: about a few seconds on a B200
+// before it gives up.  Launches pass their limit to the kernels (a test can
+// ask for a much shorter one).
 constexpr uint32_t kWaitLimit = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -77,11 +80,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Gives up after
-// kWaitLimit polls: records `code` in *status (first writer wins) and returns
-// false.  `abort_flag` (shared) lets other roles stop early after a failure.
+// `limit` polls: records `code` in *status (first writer wins), raises
+// *abort_flag and returns false.  `abort_flag` (shared) lets other roles stop
+// early after a failure: once it is set the wait returns false without
+// recording anything.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int code,
-                                          volatile int* abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+                                          volatile int* abort_flag, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 1023u) == 1023u) {
             if (*abort_flag) return false;
@@ -91,6 +96,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     atomicCAS(status, 0, code);
     *abort_flag = 1;
     return false;
+}
+
+// Drain wait: the phase with the given parity must complete (copies or MMAs
+// in flight finish before the CTA exits), whatever the abort flag says.
+// Gives up after `limit` polls, recording `code`, and returns false.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, int code, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && i > 65536u) __nanosleep(64);
+    }
+    atomicCAS(status, 0, code);
+    return false;
+}
+
+// Complete `bytes` of the barrier's current phase's expected transaction
+// count without a copy (stands in for bytes that will never arrive).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- TMA

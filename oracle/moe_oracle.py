@@ -376,11 +376,15 @@ def moe_layer(x, Wr, W1, W3, W2, K, capacity_factor=0.0, bias32=None, alpha=0.0,
 
 
 def dot_error_bound(x: np.ndarray, Wr: np.ndarray) -> np.ndarray:
-    """Rigorous bound on |fp32-accumulated dot product - exact| per logit.
+    """Rigorous bound on |fp32-accumulated dot product - exact| per logit,
+    before the final result is stored.
 
-    gamma_n * sum_i |x_i W_ie| + u32 * |l|, gamma_n = n u / (1 - n u),
-    u = 2**-24, for any summation order with round-to-nearest (Higham,
-    Accuracy and Stability of Numerical Algorithms, section 3.1).
+    Returns gamma_n * sum_i |x_i W_ie| with gamma_n = n u / (1 - n u),
+    u = 2**-24: the accumulation error of an n-term sum of exact products in
+    fp32 with round-to-nearest, for any summation order (Higham, Accuracy and
+    Stability of Numerical Algorithms, section 3.1).  The term for rounding
+    the exact logit itself to fp32 (u * |l|) is not included; callers that
+    compare against an fp64 logit add it.
     """
     x = np.abs(np.asarray(x, dtype=np.float64))
     W = np.abs(np.asarray(Wr, dtype=np.float64))
@@ -391,7 +395,14 @@ def dot_error_bound(x: np.ndarray, Wr: np.ndarray) -> np.ndarray:
 
 
 def bf16_round(a: np.ndarray) -> np.ndarray:
-    """Round fp64 values to bf16 (round to nearest even) and back to fp64."""
+    """Round to bf16 through fp32, and widen back to fp64.
+
+    Two roundings, both to nearest with ties to even: fp64 -> fp32, then
+    fp32 -> bf16.  This is the path of a value the kernels hold in fp32 (an
+    fp32 accumulator stored as bf16).  It differs from a single fp64 -> bf16
+    rounding only when the fp64 value lies within half an fp32 ulp of a bf16
+    rounding midpoint (double rounding can then land on the even neighbour).
+    """
     f = np.asarray(a, dtype=np.float32)
     b = f.view(np.uint32).astype(np.uint64)
     lsb = (b >> 16) & 1

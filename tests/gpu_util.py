@@ -160,3 +160,51 @@ def oracle_layer(inp: LayerInputs, bias32=None, tokens=None, h_round=None, alpha
 
     return O.moe_layer(x64, Wr64, Lazy(inp.W1), Lazy(inp.W3), Lazy(inp.W2), inp.wl.K,
                        inp.wl.capacity_factor, bias32=bias32, alpha=alpha, tokens=tokens, h_round=h_round)
+
+
+def oracle_routing(inp: LayerInputs, bias32=None):
+    """The oracle's own routing of the whole batch (fp32 decisions on its
+    correctly rounded logits) plus the rigorous logit error bound; computed
+    from the inputs only."""
+    x64, Wr64 = inp.host()
+    K, E = inp.wl.K, inp.wl.E
+    l64 = O.router_logits(x64, Wr64)
+    idx, _, _ = O.route_from_logits_f32(l64.astype(np.float32), K, bias32)
+    C = O.capacity(inp.T, K, E, inp.wl.capacity_factor)
+    disp = O.dispatch(idx, E, C)
+    bound = 2.0 * O.dot_error_bound(x64, Wr64) + np.abs(l64) * 2.0 ** -23
+    return idx, disp, l64, bound
+
+
+def covering_sample(inp: LayerInputs, S: int, bias32=None, seed: int = 0, per_expert: int = 2):
+    """Sorted token ids, at least min(S, T) of them: for every expert with
+    kept rows under the oracle's routing, the `per_expert` earliest tokens
+    that keep a slot on it, unambiguous ones (top-K fixed under the logit
+    error bound) first, so that one token routed differently by the library
+    does not lose the expert (early tokens also keep their capacity ranks
+    when a later routing differs); the rest seeded uniform draws.  Also
+    returns the set of experts with kept rows."""
+    idx, disp, l64, bound = oracle_routing(inp, bias32)
+    T, K, E = inp.T, inp.wl.K, inp.wl.E
+    amb = ambiguous_tokens(l64, bound, K, bias32)
+    inv = disp["inv"]
+    need = {e for e in range(E) if disp["kept"][e] > 0}
+    cand = {e: [] for e in need}
+    for t in range(T):
+        for k in range(K):
+            if inv[t, k] >= 0:
+                cand[int(idx[t, k])].append(t)
+    chosen = set()
+    for e in need:
+        ts = sorted(cand[e], key=lambda t: (bool(amb[t]), t))
+        chosen.update(ts[:per_expert])
+    rng = np.random.default_rng(seed)
+    rest = [t for t in rng.permutation(T).tolist() if t not in chosen]
+    chosen.update(rest[: max(0, S - len(chosen))])
+    return sorted(chosen), need
+
+
+def experts_compared(rows, idx_ref: np.ndarray, inv_ref: np.ndarray) -> set:
+    """Experts that hold a kept slot of at least one compared token."""
+    return {int(idx_ref[t, k]) for t in rows for k in range(idx_ref.shape[1]) if inv_ref[t, k] >= 0}
+

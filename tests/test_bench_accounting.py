@@ -14,7 +14,8 @@ def test_decode_layer_bytes_and_flops():
     assert alg["touched"] == E and alg["n_kept"] == T * K
     assert alg["layer_bytes"] == weights + T * d * 2 + T * d * 4 + d * E * 2
     assert alg["layer_flops"] == 2 * T * d * E + 6 * d * f * T * K
-    assert alg["gemm_bytes"] == weights + T * K * (d * 2 + 2 * f * 2 + d * 4)
+    assert alg["gemm_bytes"] == weights           # touched expert weights only
+    assert alg["gemm_design_bytes"] == T * K * (d * 2 + 2 * f * 2 + d * 4)
     assert alg["gemm_flops"] == 6 * d * f * T * K
     # the decode layer is HBM-bound at the measured peaks: 2.8 GB vs 180 GFLOP
     assert alg["layer_bytes"] / 6541e9 > alg["layer_flops"] / 1627e12

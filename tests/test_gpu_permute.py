@@ -63,3 +63,81 @@ def test_permute_is_deterministic():
         outs.append([b.cpu() for b in bufs])
     for b in range(6):
         assert torch.equal(outs[0][b], outs[1][b]) and torch.equal(outs[0][b], outs[2][b])
+
+
+def _permute_all(dims, idx, x, T, E, K, dm):
+    d = dev()
+    ws = abi.alloc_workspace(dims)
+    i32 = dict(dtype=torch.int32, device=d)
+    b = dict(counts=torch.empty(E, **i32), kept=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+             inv=torch.empty(T, K, **i32), src=torch.full((T * K,), -7, **i32),
+             xp=None if x is None else torch.zeros(T * K, dm, dtype=torch.bfloat16, device=d),
+             nd=torch.empty(1, **i32))
+    abi.moe_reset_device_status(ws)
+    abi.moe_permute(dims, idx, x, b["counts"], b["kept"], b["offsets"], b["inv"], b["src"], b["xp"], b["nd"], ws)
+    torch.cuda.synchronize()
+    return b, abi.moe_get_device_status(ws)
+
+
+@pytest.mark.parametrize("T,E,K,cf,with_x", [(700, 8, 2, 0.0, True), (700, 16, 4, 1.0, False),
+                                             (3000, 60, 4, 1.0, True), (2100, 256, 8, 0.0, False)])
+def test_permute_repeated_expert_in_a_token(T, E, K, cf, with_x):
+    """A token that lists an expert twice is two assignments, ranked in slot
+    order: the oracle's scan over (t, k) pairs gives the expected result."""
+    d = dev()
+    idx_h = synth.distinct_choices(T, E, K, seed=T + 3 * E).numpy().copy()
+    idx_h[::5, K - 1] = idx_h[::5, 0]          # every 5th token repeats its first expert
+    idx_h[1::9, :] = idx_h[1::9, :1]            # every 9th token lists one expert K times
+    idx = torch.from_numpy(idx_h).to(d)
+    dm = 64
+    x = synth.normal_bf16((T, dm), seed=6, stream=synth.STREAM_X, device=d) if with_x else None
+    dims = abi.Dims(T, dm, 64, E, K, cf)
+    b, (st, _) = _permute_all(dims, idx, x, T, E, K, dm)
+    assert st == abi.MOE_OK
+    o = O.dispatch(idx_h, E, O.capacity(T, K, E, cf))
+    for key, ref in (("counts", "counts"), ("kept", "kept"), ("offsets", "offsets"), ("inv", "inv")):
+        assert np.array_equal(b[key].cpu().numpy(), o[ref]), key
+    n = int(o["offsets"][-1])
+    assert np.array_equal(b["src"].cpu().numpy()[:n], o["src"])
+    assert int(b["nd"].item()) == o["n_dropped"]
+    if with_x:
+        xs = x.view(torch.int16).cpu().numpy()
+        assert np.array_equal(b["xp"].view(torch.int16).cpu().numpy()[:n], xs[o["src"]])
+
+
+@pytest.mark.parametrize("T,E,K,cf,with_x", [(500, 8, 2, 0.0, True), (500, 60, 4, 1.0, False),
+                                             (5000, 60, 4, 1.0, True), (3000, 256, 8, 0.0, False)])
+def test_permute_skips_out_of_range_experts(T, E, K, cf, with_x):
+    """Entries outside [0, E) are skipped (not counted, inv = -1) and the
+    status flag reads MOE_EINDEX.  Expected values: the oracle's dispatch
+    with those entries sent to an extra last expert E, whose rows come after
+    every real expert's, with the capacity of the real E."""
+    d = dev()
+    idx_h = synth.distinct_choices(T, E, K, seed=2 * T + E).numpy().copy()
+    bad = np.zeros((T, K), bool)
+    bad[::11, 0] = True
+    bad[3::13, K - 1] = True
+    vals = np.array([E, -1, E + 1000, -2 ** 31, 2 ** 31 - 1], np.int64)
+    idx_h[bad] = vals[np.arange(bad.sum()) % len(vals)]
+    idx = torch.from_numpy(idx_h.astype(np.int32)).to(d)
+    dm = 64
+    x = synth.normal_bf16((T, dm), seed=8, stream=synth.STREAM_X, device=d) if with_x else None
+    dims = abi.Dims(T, dm, 64, E, K, cf)
+    b, (st, detail) = _permute_all(dims, idx, x, T, E, K, dm)
+    assert st == abi.MOE_EINDEX and detail == 7
+    sink = np.where(bad, E, idx_h)
+    C = O.capacity(T, K, E, cf)
+    o = O.dispatch(sink, E + 1, C)
+    assert np.array_equal(b["counts"].cpu().numpy(), o["counts"][:E])
+    assert np.array_equal(b["kept"].cpu().numpy(), o["kept"][:E])
+    assert np.array_equal(b["offsets"].cpu().numpy(), o["offsets"][:E + 1])
+    inv_ref = np.where(bad, -1, o["inv"])
+    assert np.array_equal(b["inv"].cpu().numpy(), inv_ref)
+    n = int(o["offsets"][E])
+    assert np.array_equal(b["src"].cpu().numpy()[:n], o["src"][:n])
+    assert np.all(b["src"].cpu().numpy()[n:] == -7)
+    drops = int(np.sum(np.maximum(0, o["counts"][:E] - (C if C is not None else 1 << 40))))
+    assert int(b["nd"].item()) == drops
+    if with_x:
+        xs = x.view(torch.int16).cpu().numpy()
+        assert np.array_equal(b["xp"].view(torch.int16).cpu().numpy()[:n], xs[o["src"][:n]])

@@ -408,6 +408,27 @@ def test_bf16_round_ties_to_even():
     assert got.tolist() == [1.0, 1.0, 1.0 + 4 * 2 ** -8, 1.0, -2.5]
 
 
+def test_bf16_round_goes_through_fp32():
+    """Separates the two readings of "round to bf16": 1 + 2^-8 + 2^-40 lies just
+    above the bf16 midpoint between 1 and 1 + 2^-7, so a direct fp64 -> bf16
+    rounding goes up; rounded to fp32 first it becomes the midpoint itself
+    (2^-40 is below half an fp32 ulp at 1), which ties to the even neighbour
+    1.0.  The oracle takes the fp32 path, like a kernel storing an fp32 value.
+    Likewise just below a midpoint with the fp32 step rounding up onto it."""
+    up = 1.0 + 2.0 ** -8 + 2.0 ** -40
+    assert O.bf16_round(np.array([up])).tolist() == [1.0]
+    # direct single rounding (exact rational arithmetic) would give 1 + 2^-7
+    from fractions import Fraction
+    q = Fraction(up) / Fraction(2) ** -7
+    assert q - int(q) > Fraction(1, 2)
+    # midpoint between 1 + 2^-7 and 1 + 2^-6 (odd lower neighbour), reached
+    # from below: fp32 rounds 1 + 3 * 2^-8 - 2^-40 up to the midpoint, which
+    # then ties to the even neighbour 1 + 2^-6 (single rounding: 1 + 2^-7)
+    down = 1.0 + 3 * 2.0 ** -8 - 2.0 ** -40
+    assert O.bf16_round(np.array([down])).tolist() == [1.0 + 2.0 ** -6]
+    assert O.bf16_round(np.array([-up])).tolist() == [-1.0]
+
+
 def test_capacity_uses_exact_value_of_the_double():
     # 0.8 is stored as 0.8000000000000000444..., so 0.8*30*2/3 is just above 16
     assert O.capacity(30, 2, 3, 0.8) == 17
