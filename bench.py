@@ -65,6 +65,9 @@ def parse():
     p.add_argument("--no-sustained", action="store_true", help="skip the second-long sustained run")
     p.add_argument("--tokens", type=int, default=0,
                    help="override the workload's T (smaller cases for profiling); recorded in config")
+    p.add_argument("--experts", type=int, default=0,
+                   help="profiling case: keep only the first N experts (T scaled to keep the mean group "
+                        "size unless --tokens is given); recorded in config")
     return p.parse_args()
 
 
@@ -415,7 +418,8 @@ def roofline_of(layer: Layer, res: dict, peaks: dict, peak_src: str):
         roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
                 "frac": achieved / tensor_peak, "peak_source": f"{tensor_src} bf16 GEMM"}
     kernel = abi.moe_ffn_kernel(layer.dims)
-    traffic = profile_traffic(kernel, wl.name) if layer.chunk == 0 and wl.T == synth.get_workload(wl.name).T else None
+    full = synth.get_workload(wl.name)
+    traffic = profile_traffic(kernel, wl.name) if layer.chunk == 0 and (wl.T, wl.E) == (full.T, full.E) else None
     roof.update({
         "traffic": traffic,
         "kernel": (f"{kernel} (gate/up and down in one launch)" if per_stage else
@@ -461,10 +465,16 @@ def run_ours(args):
 
     peaks, peak_src = load_peaks()
     wl = synth.get_workload(args.workload)
+    if args.experts > 0:
+        if args.experts < wl.K:
+            raise SystemExit("--experts must be at least the workload's K")
+        wl.T = max(1, wl.T * args.experts // wl.E)
+        wl.E = args.experts
     if args.tokens > 0:
         wl.T = args.tokens
+    reduced = args.tokens > 0 or args.experts > 0
     chunk = args.chunk_tokens
-    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and args.tokens == 0
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not reduced
     layer = Layer(wl, dev, chunk, keep_host=want_cpu)
     abi.moe_reset_device_status(layer.ws)
     for i in range(args.warmup):
@@ -555,7 +565,8 @@ def run_ours(args):
                          f"{max(times):.1f} s; numpy fp64 with the BLAS threads given in cores"}
     line_cfg = {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K,
                 "capacity_factor": wl.capacity_factor, "parallelism": f"replicas x{world}",
-                "l2": l2_note(wl), **({"chunk_tokens": chunk} if chunk > 0 else {})}
+                "l2": l2_note(wl), **({"chunk_tokens": chunk} if chunk > 0 else {}),
+                **({"reduced_for_profiling": True} if reduced else {})}
     memory = {"workspace_bytes": int(layer.ws.numel()), "peak_device_bytes": res["peak_bytes"],
               **({"workspace_bytes_whole_batch": abi.moe_workspace_size(layer.dims)} if chunk > 0 else {})}
     del layer, x_host, y_host, x_dev, y_dev
@@ -564,8 +575,7 @@ def run_ours(args):
     # ---- the other workloads of the metric (prefill, capacity, bias loop):
     # same step, same timing, one entry each; 1-GPU runs only
     extras = {}
-    if (world == 1 and not args.no_extra and args.workload == "mixtral_decode" and args.tokens == 0
-            and chunk == 0):
+    if world == 1 and not args.no_extra and args.workload == "mixtral_decode" and not reduced and chunk == 0:
         for name in EXTRA_WORKLOADS:
             wx = synth.get_workload(name)
             lx = Layer(wx, dev)

@@ -244,10 +244,14 @@ MOE_API int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const i
 /* Step 5: combine ([P2] section 2 step 4 and section 2.3: weighted sum back
  * in token order; section 2.2: unselected experts add nothing).
  *   y[t] = sum_{k=0..K-1, inv[t,k] >= 0} topk_w[t,k] * y_perm[inv[t,k]]
- * summed in k order in fp32; a dropped slot adds nothing and the remaining
- * weights are not renormalised.  y [T, d_model] fp32 out. */
+ * summed in k order in fp32 (fused multiply-adds); a dropped slot adds
+ * nothing and the remaining weights are not renormalised.
+ *   y           [T, d_model] out: fp32 when y_is_bf16 == 0; bf16 otherwise,
+ *               each value the round-to-nearest-even of the fp32 sum (the
+ *               activation type an inference engine passes on; the fp32 form
+ *               is the parity output). */
 MOE_API int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* inv,
-                const float* topk_w, float* y, void* stream);
+                const float* topk_w, void* y, int y_is_bf16, void* stream);
 
 /* Load statistics ([P2] section 1.2): f_i = counts_i / (T K),
  * P_i = prob_mean_i, aux = E * sum_i f_i P_i.  Any output may be NULL. */
@@ -312,12 +316,13 @@ MOE_API int moe_layer_launch_count(const moe_dims* dims, int stats, int bias_upd
  *   x [T, d_model] bf16, Wr [d_model, E] bf16, W13p/W2p from moe_pack_weights
  *   bias  [E] fp32 or NULL; if non-NULL and alpha != 0 it is updated in place
  *         after routing (so the routing of this call uses the old value)
- *   y     [T, d_model] fp32 out
+ *   y     [T, d_model] out: fp32, or bf16 with y_is_bf16 != 0 (RNE of the
+ *         fp32 result, as in moe_combine)
  *   out   optional extra outputs (NULL = none)
  * [P1] section 2 lists the same sequence: score, select, dispatch, expert
  * FFN, gather back. */
 MOE_API int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* Wr, float* bias,
-                      float alpha, const moe_bf16* W13p, const moe_bf16* W2p, float* y,
+                      float alpha, const moe_bf16* W13p, const moe_bf16* W2p, void* y, int y_is_bf16,
                       const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Chunked MoE ([P2] section 4.3: prefill tokens go through the MoE step in
@@ -342,8 +347,32 @@ MOE_API int moe_chunked_workspace_size(const moe_dims* dims, int64_t chunk_token
 MOE_API int moe_layer_chunked_launch_count(const moe_dims* dims, int64_t chunk_tokens, int stats, int bias_update);
 MOE_API int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const moe_bf16* x,
                                       const moe_bf16* Wr, float* bias, float alpha, const moe_bf16* W13p,
-                                      const moe_bf16* W2p, float* y, const moe_layer_outputs* out, void* ws,
-                                      size_t ws_bytes, void* stream);
+                                      const moe_bf16* W2p, void* y, int y_is_bf16, const moe_layer_outputs* out,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* Expert parallelism ([P2] section 4.2; [P3] section 2.2: experts spread over
+ * GPUs, token rows exchanged by all-to-all before and after the expert
+ * computation).  The exchanges themselves are the caller's (NCCL through
+ * torch.distributed in the Python layer); this call is the receiving rank's
+ * one local step that has no single-GPU counterpart: it regroups the
+ * received rows by local expert.
+ *   n_ranks, E_local  ranks and experts per rank (n_ranks * E_local <= 2048)
+ *   recv_counts  [n_ranks, E_local] int32 (device): rows received from each
+ *                source rank for each local expert
+ *   rows_in      [n_rows, d_model] bf16: the received rows, source-major (a
+ *                source's rows for local expert 0, 1, .., in the order sent);
+ *                n_rows = sum of recv_counts
+ *   rows_out     [n_rows, d_model] bf16 out: expert-major; within an expert,
+ *                by source rank, then in the order received
+ *   offsets      [E_local + 1] int32 out: exclusive prefix of the per-expert
+ *                row totals (the group offsets moe_expert_ffn takes)
+ *   row_of       [n_rows] int32 out: the output row of each received row (to
+ *                return results in the received order, e.g. moe_combine with
+ *                K = 1, inv = row_of and unit weights, an exact copy)
+ * d_model % 8 == 0; pointers 16-byte aligned. */
+MOE_API int moe_ep_regroup(int n_ranks, int E_local, const int32_t* recv_counts, int64_t n_rows, int d_model,
+                           const moe_bf16* rows_in, moe_bf16* rows_out, int32_t* offsets, int32_t* row_of,
+                           void* stream);
 
 #ifdef __cplusplus
 }

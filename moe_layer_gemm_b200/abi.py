@@ -34,7 +34,7 @@ EXPORTED = [
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
     "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc", "moe_ffn_kernel",
     "moe_chunked_workspace_size", "moe_layer_forward_chunked", "moe_layer_chunked_launch_count",
-    "moe_test_set_wait_limits",
+    "moe_test_set_wait_limits", "moe_ep_regroup",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -81,19 +81,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_route_from_logits": (I, [dims_p, P, P, P, P, P, P, SZ, P]),
         "moe_permute": (I, [dims_p, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "moe_expert_ffn": (I, [dims_p, P, P, P, P, P, P, P, SZ, P]),
-        "moe_combine": (I, [dims_p, P, P, P, P, P]),
+        "moe_combine": (I, [dims_p, P, P, P, P, I, P]),
         "moe_load_stats": (I, [dims_p, P, P, P, P, P]),
         "moe_bias_update": (I, [dims_p, P, F, P, P]),
-        "moe_layer_forward": (I, [dims_p, P, P, P, F, P, P, P, ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
+        "moe_layer_forward": (I, [dims_p, P, P, P, F, P, P, P, I, ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
         "moe_layer_launch_count": (I, [dims_p, I, I]),
         "moe_packed_weight_bytes": (I, [dims_p, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
         "moe_permute_noalloc": (I, [dims_p, P, P, P, P, P, P, P, P, P, P]),
         "moe_ffn_kernel": (I, [dims_p]),
         "moe_chunked_workspace_size": (I, [dims_p, ctypes.c_int64, ctypes.POINTER(SZ)]),
         "moe_layer_chunked_launch_count": (I, [dims_p, ctypes.c_int64, I, I]),
-        "moe_layer_forward_chunked": (I, [dims_p, ctypes.c_int64, P, P, P, F, P, P, P,
+        "moe_layer_forward_chunked": (I, [dims_p, ctypes.c_int64, P, P, P, F, P, P, P, I,
                                           ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
         "moe_test_set_wait_limits": (I, [ctypes.c_int64, ctypes.c_int64, I]),
+        "moe_ep_regroup": (I, [I, I, P, I64, I, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -254,10 +255,19 @@ def moe_expert_ffn(dims, x_perm, offsets, W13p, W2p, h, y_perm, ws, stream=None)
         _ptr(ws, None, "ws"), ws.numel(), _stream(stream)))
 
 
+def _y_arg(y):
+    """Pointer and y_is_bf16 flag of a layer output (fp32 or bf16 tensor)."""
+    if y is not None and y.dtype == BF16:
+        return _ptr(y, BF16, "y"), 1
+    return _ptr(y, F32, "y"), 0
+
+
 def moe_combine(dims, y_perm, inv, topk_w, y, stream=None):
+    """y may be fp32 or bf16 (the fp32 sum rounded to nearest even)."""
+    yp, yb = _y_arg(y)
     _check("moe_combine", load().moe_combine(
         ctypes.byref(_dims(dims)), _ptr(y_perm, F32, "y_perm"), _ptr(inv, I32, "inv"),
-        _ptr(topk_w, F32, "topk_w"), _ptr(y, F32, "y"), _stream(stream)))
+        _ptr(topk_w, F32, "topk_w"), yp, yb, _stream(stream)))
 
 
 def moe_load_stats(dims, counts, prob_mean, f, aux, stream=None):
@@ -274,9 +284,9 @@ def moe_bias_update(dims, counts, alpha: float, bias, stream=None):
 
 def moe_layer_forward(dims, x, Wr, bias, alpha: float, W13p, W2p, y, ws, outputs: Optional[dict] = None,
                       stream=None, stage_events=None):
-    """The whole layer.  ``outputs`` maps moe_layer_outputs field names to
-    tensors; ``stage_events`` is a sequence of NUM_STAGE_EVENTS recorded
-    torch.cuda.Event objects (or None)."""
+    """The whole layer.  ``y`` is fp32 or bf16; ``outputs`` maps
+    moe_layer_outputs field names to tensors; ``stage_events`` is a sequence
+    of NUM_STAGE_EVENTS recorded torch.cuda.Event objects (or None)."""
     o = None
     keep = None
     if outputs or stage_events is not None:
@@ -290,7 +300,7 @@ def moe_layer_forward(dims, x, Wr, bias, alpha: float, W13p, W2p, y, ws, outputs
             o.stage_events = ctypes.cast(keep, ctypes.c_void_p)
     _check("moe_layer_forward", load().moe_layer_forward(
         ctypes.byref(_dims(dims)), _ptr(x, BF16, "x"), _ptr(Wr, BF16, "Wr"), _ptr(bias, F32, "bias"),
-        ctypes.c_float(alpha), _ptr(W13p, BF16, "W13p"), _ptr(W2p, BF16, "W2p"), _ptr(y, F32, "y"),
+        ctypes.c_float(alpha), _ptr(W13p, BF16, "W13p"), _ptr(W2p, BF16, "W2p"), *_y_arg(y),
         ctypes.byref(o) if o is not None else None, _ptr(ws, None, "ws"), ws.numel(), _stream(stream)))
 
 
@@ -305,7 +315,7 @@ def moe_layer_forward_chunked(dims, chunk_tokens: int, x, Wr, bias, alpha: float
     _check("moe_layer_forward_chunked", load().moe_layer_forward_chunked(
         ctypes.byref(_dims(dims)), ctypes.c_int64(chunk_tokens), _ptr(x, BF16, "x"), _ptr(Wr, BF16, "Wr"),
         _ptr(bias, F32, "bias"), ctypes.c_float(alpha), _ptr(W13p, BF16, "W13p"), _ptr(W2p, BF16, "W2p"),
-        _ptr(y, F32, "y"), ctypes.byref(o) if o is not None else None, _ptr(ws, None, "ws"), ws.numel(),
+        *_y_arg(y), ctypes.byref(o) if o is not None else None, _ptr(ws, None, "ws"), ws.numel(),
         _stream(stream)))
 
 
@@ -333,6 +343,16 @@ def moe_ffn_kernel(dims) -> str:
     if k < 0:
         raise MoEError("moe_ffn_kernel", k, "invalid dims")
     return FFN_KERNELS[k]
+
+
+def moe_ep_regroup(n_ranks: int, E_local: int, recv_counts, rows_in, rows_out, offsets, row_of, stream=None):
+    """Regroup the rows a rank received (source-major) by local expert (see the header)."""
+    n = 0 if rows_in is None else int(rows_in.shape[0])
+    d = int(rows_out.shape[1]) if rows_out is not None and rows_out.dim() == 2 else 8
+    _check("moe_ep_regroup", load().moe_ep_regroup(
+        int(n_ranks), int(E_local), _ptr(recv_counts, I32, "recv_counts"), ctypes.c_int64(n), d,
+        _ptr(rows_in, BF16, "rows_in") if n else None, _ptr(rows_out, BF16, "rows_out") if n else None,
+        _ptr(offsets, I32, "offsets"), _ptr(row_of, I32, "row_of") if n else None, _stream(stream)))
 
 
 # ---------------------------------------------------------------- helpers

@@ -30,7 +30,8 @@ WaitSettings wait_settings() {
 
 namespace {
 
-constexpr int kVersion = 102;  // 1.02: MOE_EINDEX, moe_test_set_wait_limits; 1.01: P_topk, aux_topk, z_loss; chunked layer
+constexpr int kVersion = 200;  // 2.00: y_is_bf16 in moe_combine and both layer calls; MOE_EINDEX;
+                                // moe_test_set_wait_limits.  1.01: P_topk, aux_topk, z_loss; chunked layer
 constexpr int64_t kMaxT = int64_t(1) << 24;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -84,12 +85,21 @@ struct Layout {
 // padding and the weight stream dominates.
 constexpr int kSwapMaxRows = 128;
 
-// Weight-major tiles are enabled when groups of decode size are expected:
-// a mean group of at most 256 rows (skewed routing then also leaves many
-// small groups).
+// Tile policy by the mean group (T K / E assignments per expert):
+//   1  decode-sized (mean <= 256 rows; skewed routing then also leaves many
+//      small groups): groups of <= 128 rows take weight-major tiles
+//   2  mid-sized (mean <= 2048 rows, e.g. a capacity-limited layer): every
+//      group takes weight-major CTA-pair tiles of up to 256 tokens, so a
+//      group's ragged tail is padded to 16 tokens instead of a 128- or
+//      256-row token tile (only when the CTA-pair kernel takes the shape;
+//      otherwise no weight-major tiles)
+//   0  large groups: token-major tiles
 int choose_swap(const moe_dims* d) {
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
-    return (avg <= 256 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
+    if (d->d_model % 128 != 0 || (2 * d->d_ff) % 128 != 0) return 0;
+    if (avg <= 256) return 1;
+    if (avg <= 2048 && d->d_model % 256 == 0 && (2 * d->d_ff) % 256 == 0) return 2;
+    return 0;
 }
 
 // Reduction split of the down projection when groups are decode-sized:
@@ -98,7 +108,7 @@ int choose_swap(const moe_dims* d) {
 // and there are tiles enough for the CTA-pair kernel to give each weight-
 // major tile two weight sub-tiles (half the token reads).
 int choose_nsplit(const moe_dims* d, int swap) {
-    if (!swap) return 1;
+    if (swap != 1) return 1;
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
     if (avg > kSwapMaxRows) return 1;
     int ks = static_cast<int>((d->d_ff + d->d_model - 1) / d->d_model);
@@ -269,7 +279,8 @@ GemmLaunch ffn_launch(const moe_dims* d, const Layout& L, const bf16* xperm, con
     g.group_off = offsets;
     g.dense_rows = 0;
     g.max_group_rows = maxrows;
-    g.swap_max_rows = L.swap ? kSwapMaxRows : 0;
+    g.swap_max_rows = L.swap == 1 ? kSwapMaxRows : (L.swap == 2 ? (1 << 30) : 0);
+    g.swap_tokens_max = L.swap == 2 ? 256 : 128;
     g.small_groups = (d->T * d->K) < static_cast<int64_t>(d->E) * 128;
     g.nphase = 2;
     GemmPhase& p0 = g.ph[0];
@@ -306,8 +317,9 @@ GemmLaunch ffn_launch(const moe_dims* d, const Layout& L, const bf16* xperm, con
 }
 
 // CTA-pair tiles: token-major pairs are 256 token rows, worth it when groups
-// are large (ragged 256-row tails of mid-sized groups cost more than they
-// save); weight-major pairs halve the token traffic of decode-sized groups.
+// are large; weight-major pairs halve the token traffic of decode-sized
+// groups and, up to 256 tokens wide, cover mid-sized groups with tails
+// padded to 16 tokens.
 bool ffn_uses_pair(const moe_dims* d, const Layout& L, const GemmLaunch& g) {
     const bool large_groups = d->T * d->K >= static_cast<int64_t>(d->E) * 1024;
     return (large_groups || L.swap) && gemm_2sm_supported(g);
@@ -318,8 +330,9 @@ bool ffn_uses_pair(const moe_dims* d, const Layout& L, const GemmLaunch& g) {
 // entry point clears them with a memset).
 int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
            const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st) {
-    const GemmLaunch g = ffn_launch(d, L, xperm, offsets, W13p, W2p, h, yout, nsplit, ws);
+    GemmLaunch g = ffn_launch(d, L, xperm, offsets, W13p, W2p, h, yout, nsplit, ws);
     if (ffn_uses_pair(d, L, g)) return map_launch(launch_grouped_gemm_2sm(g, st));
+    if (L.swap == 2) g.swap_max_rows = 0;  // wide weight-major tiles are a CTA-pair form
     return map_launch(launch_grouped_gemm(g, st));
 }
 
@@ -486,12 +499,12 @@ int moe_permute_noalloc(const moe_dims* dims, const int32_t* topk_idx, const moe
     return map_launch(r);
 }
 
-int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* inv, const float* topk_w, float* y,
-                void* stream) {
+int moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* inv, const float* topk_w, void* y,
+                int y_is_bf16, void* stream) {
     MOE_TRY(check_dims(dims));
     if (!y_perm || !inv || !topk_w || !y) return MOE_EINVAL;
     if (!aligned16(y_perm) || !aligned16(y)) return MOE_EUNSUPPORTED;
-    return map_launch(launch_combine(y_perm, 1, 0, inv, topk_w, dims->T, dims->d_model, dims->K, y,
+    return map_launch(launch_combine(y_perm, 1, 0, inv, topk_w, dims->T, dims->d_model, dims->K, y, y_is_bf16 != 0,
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -513,8 +526,8 @@ int moe_bias_update(const moe_dims* dims, const int32_t* counts, float alpha, fl
 }
 
 int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* Wr, float* bias, float alpha,
-                      const moe_bf16* W13p, const moe_bf16* W2p, float* y, const moe_layer_outputs* out,
-                      void* ws, size_t ws_bytes, void* stream) {
+                      const moe_bf16* W13p, const moe_bf16* W2p, void* y, int y_is_bf16,
+                      const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream) {
     MOE_TRY(check_dims(dims));
     if (!x || !Wr || !W13p || !W2p || !y) return MOE_EINVAL;
     if (!aligned16(x) || !aligned16(Wr) || !aligned16(W13p) || !aligned16(W2p) || !aligned16(y))
@@ -581,10 +594,22 @@ int moe_layer_forward(const moe_dims* dims, const moe_bf16* x, const moe_bf16* W
         }
     }
     MOE_TRY(map_launch(launch_combine(yp, L.nsplit, dims->T * dims->K * dims->d_model, inv, w, dims->T,
-                                      dims->d_model, dims->K, y, st, &tail)));
+                                      dims->d_model, dims->K, y, y_is_bf16 != 0, st, &tail)));
     mark(4);
     mark(5);
     return MOE_OK;
+}
+
+int moe_ep_regroup(int n_ranks, int E_local, const int32_t* recv_counts, int64_t n_rows, int d_model,
+                   const moe_bf16* rows_in, moe_bf16* rows_out, int32_t* offsets, int32_t* row_of, void* stream) {
+    if (n_ranks < 1 || E_local < 1 || static_cast<int64_t>(n_ranks) * E_local > ep_regroup_max_blocks())
+        return MOE_EINVAL;
+    if (n_rows < 0 || n_rows > (int64_t(1) << 31) - 1 || d_model < 8 || d_model > (1 << 16)) return MOE_EINVAL;
+    if (!recv_counts || !offsets || (n_rows > 0 && (!rows_in || !rows_out || !row_of))) return MOE_EINVAL;
+    if (d_model % 8 != 0 || !aligned16(rows_in) || !aligned16(rows_out)) return MOE_EUNSUPPORTED;
+    return map_launch(launch_ep_regroup(recv_counts, n_ranks, E_local, n_rows, reinterpret_cast<const bf16*>(rows_in),
+                                        d_model, reinterpret_cast<bf16*>(rows_out), offsets, row_of,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 int moe_chunked_workspace_size(const moe_dims* dims, int64_t chunk_tokens, size_t* bytes) {
@@ -595,8 +620,9 @@ int moe_chunked_workspace_size(const moe_dims* dims, int64_t chunk_tokens, size_
 }
 
 int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const moe_bf16* x, const moe_bf16* Wr,
-                              float* bias, float alpha, const moe_bf16* W13p, const moe_bf16* W2p, float* y,
-                              const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream) {
+                              float* bias, float alpha, const moe_bf16* W13p, const moe_bf16* W2p, void* y,
+                              int y_is_bf16, const moe_layer_outputs* out, void* ws, size_t ws_bytes,
+                              void* stream) {
     MOE_TRY(check_dims(dims));
     if (chunk_tokens < 1) return MOE_EINVAL;
     if (!x || !Wr || !W13p || !W2p || !y) return MOE_EINVAL;
@@ -650,8 +676,10 @@ int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const 
         MOE_TRY(do_ffn(&dc, Lc, at<bf16>(ws, Lc.xperm), at<int32_t>(ws, Lc.offsets),
                        reinterpret_cast<const bf16*>(W13p), reinterpret_cast<const bf16*>(W2p),
                        at<bf16>(ws, Lc.h), yp, Lc.nsplit, ws, st));
+        void* y_c = y_is_bf16 ? static_cast<void*>(static_cast<bf16*>(y) + t0 * D)
+                              : static_cast<void*>(static_cast<float*>(y) + t0 * D);
         MOE_TRY(map_launch(launch_combine(yp, Lc.nsplit, dc.T * dc.K * dc.d_model, inv_c, w + t0 * K, dc.T,
-                                          dc.d_model, dc.K, y + t0 * D, st)));
+                                          dc.d_model, dc.K, y_c, y_is_bf16 != 0, st)));
         MOE_TRY(map_launch(launch_accumulate_counts(counts, cnt_c, dims->E, t0 == 0, st)));
     }
     // 3. the whole batch's statistics and bias update (one statistics CTA, no tokens)
@@ -679,8 +707,8 @@ int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens, const 
             tail.bias = bias;
             tail.alpha = alpha;
         }
-        MOE_TRY(map_launch(launch_combine(nullptr, 1, 0, nullptr, nullptr, 0, dims->d_model, dims->K, nullptr, st,
-                                          &tail)));
+        MOE_TRY(map_launch(launch_combine(nullptr, 1, 0, nullptr, nullptr, 0, dims->d_model, dims->K, nullptr, false,
+                                          st, &tail)));
     }
     return MOE_OK;
 }

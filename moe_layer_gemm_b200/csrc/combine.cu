@@ -13,6 +13,7 @@
 // (ybb.press/quantum-computing/18594), section 1.2: overloaded experts get
 // bias -= alpha, underloaded bias += alpha.
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -106,15 +107,26 @@ __device__ void stats_tail(const StatsTail& s, int64_t T, int K) {
     }
 }
 
+// Store 4 consecutive outputs: fp32, or each rounded to bf16 (nearest even)
+// from the same fp32 sum, so a bf16 output is exactly RNE of the fp32 one.
+__device__ __forceinline__ void store4(float* y, int64_t i4, float4 v) { reinterpret_cast<float4*>(y)[i4] = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* y, int64_t i4, float4 v) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(y)[i4] = u;
+}
+
 // S >= nsplit slots for partial slices (S == nsplit except the 8-slot
 // fallback, which reads only the nsplit slices that exist).  Slots are
 // handled in groups of G, whose G x S loads are all in flight at once; G
 // shrinks as slices grow so the registers, and with them the resident
 // CTAs, stay put (more loads per thread measured slower at K = 4).
-template <int S>
+template <int S, typename OutT>
 __global__ void __launch_bounds__(256, S == 1 ? 8 : (S >= 8 ? 2 : 4))  // one slice: 32 registers, 8 CTAs per SM
 combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, const int32_t* __restrict__ inv,
-               const float* __restrict__ w, int64_t T, int d, int K, float* __restrict__ y, const StatsTail tail) {
+               const float* __restrict__ w, int64_t T, int d, int K, OutT* __restrict__ y, const StatsTail tail) {
     pdl_trigger();
     pdl_wait();
     // with a statistics tail the last CTA does only that
@@ -169,7 +181,7 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
                     }
                 }
             }
-            reinterpret_cast<float4*>(y + t * d)[c] = acc;
+            store4(y + t * d, c, acc);
         }
         __syncthreads();  // rows / ws are rewritten for the next token
     }
@@ -288,8 +300,20 @@ __global__ void pack_w2_kernel(const __nv_bfloat16* __restrict__ W2, int d, int 
 
 }  // namespace
 
+template <typename OutT>
+void launch_combine_t(int g, int threads, cudaStream_t st, const float* y_perm, int nsplit, int64_t split_stride,
+                      const int32_t* inv, const float* w, int64_t T, int d, int K, OutT* y, const StatsTail& tail) {
+    switch (nsplit) {
+        case 1: (void)launch_pdl(combine_kernel<1, OutT>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        case 2: (void)launch_pdl(combine_kernel<2, OutT>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        case 3: (void)launch_pdl(combine_kernel<3, OutT>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        case 4: (void)launch_pdl(combine_kernel<4, OutT>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+        default: (void)launch_pdl(combine_kernel<8, OutT>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
+    }
+}
+
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv, const float* w,
-                   int64_t T, int d, int K, float* y, cudaStream_t st, const StatsTail* tail_in) {
+                   int64_t T, int d, int K, void* y, bool y_bf16, cudaStream_t st, const StatsTail* tail_in) {
     if (K > kMaxK || d % 4 != 0 || nsplit < 1 || nsplit > kMaxSplit) return -2;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     int64_t grid = T < static_cast<int64_t>(sms) * 16 ? T : static_cast<int64_t>(sms) * 16;
@@ -302,13 +326,11 @@ int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const 
         ++grid;  // one extra CTA for the tail
     }
     const int g = static_cast<int>(grid);
-    switch (nsplit) {
-        case 1: (void)launch_pdl(combine_kernel<1>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
-        case 2: (void)launch_pdl(combine_kernel<2>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
-        case 3: (void)launch_pdl(combine_kernel<3>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
-        case 4: (void)launch_pdl(combine_kernel<4>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
-        default: (void)launch_pdl(combine_kernel<8>, dim3(g), dim3(threads), 0, st, y_perm, nsplit, split_stride, inv, w, T, d, K, y, tail); break;
-    }
+    if (y_bf16)
+        launch_combine_t(g, threads, st, y_perm, nsplit, split_stride, inv, w, T, d, K, static_cast<__nv_bfloat16*>(y),
+                         tail);
+    else
+        launch_combine_t(g, threads, st, y_perm, nsplit, split_stride, inv, w, T, d, K, static_cast<float*>(y), tail);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

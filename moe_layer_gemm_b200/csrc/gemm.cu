@@ -234,9 +234,11 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         }
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
-    // group offsets, scheduler words and token rows come from earlier kernels;
-    // no early trigger: the next kernel launches as this one drains
+    // group offsets, scheduler words and token rows come from earlier kernels
     pdl_wait();
+    // the next kernel may launch now: its CTAs wait in their own pdl_wait
+    // until this grid completes, but no launch gap remains
+    pdl_trigger();
     for (int g = threadIdx.x; g <= G; g += blockDim.x)
         off[g] = a.group_off ? static_cast<int64_t>(a.group_off[g]) : (g == 0 ? 0 : a.dense_rows);
     __syncthreads();

@@ -69,6 +69,7 @@ constexpr int kMaxGroups = 256;
 constexpr int kRing = 8;
 
 struct Phase2 {
+    const bf16* w;  // packed weights (read only for the L2 prefetch; loads go through the tensor map)
     int N, k_blocks, epi;
     int64_t nb;  // 128-row weight blocks per group
     int ksplit, kb_per_split;  // reduction split (every tile of the phase)
@@ -84,7 +85,7 @@ struct Args2 {
     int nphase;
     int dep;
     int swap_max_rows;  // groups with at most this many rows take weight-major pair tiles
-    int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 128)
+    int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 256; <= 128 with two sub-tiles)
     Phase2 ph[2];
     int stages;
     uint32_t stage_bytes;  // per stage and CTA
@@ -94,6 +95,7 @@ struct Args2 {
     uint32_t wait_limit;      // polls of a bounded mbarrier or drain wait
     uint32_t dep_wait_limit;  // polls of the phase-1 readiness wait
     int dep_extra;            // added to the phase-1 readiness target (0; a test makes it unreachable)
+    int prefetch_kb;          // k-blocks of the first-round weight tiles pulled into L2 before the wait (0: none)
 };
 
 constexpr int kMaxStages = 16;
@@ -147,6 +149,10 @@ __device__ __forceinline__ uint32_t ld_acquire_cluster(const uint32_t* p) {
     return v;
 }
 __device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
 // TMA tile load into this CTA's shared memory, completing on the leader's barrier.
 __device__ __forceinline__ void tma_load_pair(const CUtensorMap* map, void* smem_dst, uint32_t leader_bar, int32_t x,
                                               int32_t y, uint64_t policy) {
@@ -300,9 +306,33 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
-    // group offsets, scheduler words and token rows come from earlier kernels;
-    // no early trigger: the next kernel launches as this one drains
+    // Weight tiles depend on no earlier kernel.  While the router and the
+    // dispatch finish, pull the first k-blocks of the first round of
+    // weight-major tiles into L2: cluster c takes tile c of the first phase,
+    // as if every group had one token chunk (the decode case); whichever
+    // cluster claims that tile later finds them in L2.  A hint only: no
+    // result depends on it, and every address lies inside the packed weights.
+    if (a.prefetch_kb > 0 && warp == 0 && lane == 0) {
+        const Phase2& p0 = a.ph[0];
+        const int tpg = (p0.N / (256 * p0.wt)) * p0.ksplit;  // tiles per group with one token chunk
+        const int tile = static_cast<int>(blockIdx.x >> 1);
+        const int g = tile / tpg;
+        if (g < G) {
+            const int local = tile - g * tpg;
+            const int kb0 = (local % p0.ksplit) * p0.kb_per_split;
+            const int kb1 = min(p0.k_blocks, min(kb0 + p0.kb_per_split, kb0 + a.prefetch_kb));
+            const int n0 = (local / p0.ksplit) * 256 * p0.wt;
+            const int64_t wblk0 = static_cast<int64_t>(g) * p0.nb + (n0 + 128 * static_cast<int>(rank)) / 128;
+            for (int j = 0; j < p0.wt; ++j)
+                for (int kb = kb0; kb < kb1; ++kb)
+                    prefetch_l2(p0.w + ((wblk0 + 2 * j) * p0.k_blocks + kb) * 8192, 16384u);
+        }
+    }
+    // group offsets, scheduler words and token rows come from earlier kernels
     pdl_wait();
+    // the next kernel (the combine) may launch now: its CTAs wait in their own
+    // pdl_wait until this grid completes, but no launch gap remains
+    pdl_trigger();
     for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
     __syncthreads();
     if (warp == 0) {
@@ -688,9 +718,13 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     a.dep_extra = L.dep_extra;
     const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
     a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
+    // weight-major tiles take up to 128 tokens, or 256 when the launch asks
+    // for wide ones (then each tile has one 256-row weight sub-tile: both
+    // fill the 256 TMEM columns of an accumulator buffer)
+    const int bns_cap = L.swap_tokens_max == 256 ? 256 : 128;
     {
         const int64_t lim = mx < a.swap_max_rows ? mx : a.swap_max_rows;
-        a.BNs = static_cast<int>(lim >= 128 ? 128 : ((lim + 31) / 32) * 32);
+        a.BNs = static_cast<int>(lim >= bns_cap ? bns_cap : ((lim + 31) / 32) * 32);
         if (a.BNs < 32) a.BNs = 32;
     }
     const bool token_major_possible = mx > a.swap_max_rows;
@@ -703,6 +737,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     for (int p = 0; p < L.nphase; ++p) {
         const GemmPhase& g = L.ph[p];
         Phase2& ph = a.ph[p];
+        ph.w = g.w;
         ph.N = g.N;
         ph.k_blocks = (g.Kdim + kBK - 1) / kBK;
         ph.epi = g.epi;
@@ -720,7 +755,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         // last, to shorten the final tiles, measured slower at the Mixtral
         // decode shape: their extra token reads cost more than the shorter
         // tail saved.)
-        ph.wt = (weight_major_possible && g.N % 512 == 0 &&
+        ph.wt = (weight_major_possible && a.BNs <= 128 && g.N % 512 == 0 &&
                  static_cast<int64_t>(L.G) * (g.N / 512) * ph.ksplit >= 3LL * clusters) ? 2 : 1;
         const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
         if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
@@ -735,6 +770,10 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     int wt_max = 1;
     for (int p = 0; p < L.nphase; ++p) wt_max = a.ph[p].wt > wt_max ? a.ph[p].wt : wt_max;
     a.xoff = static_cast<uint32_t>(wt_max) * kHalf;
+    // decode-sized launches (weight-major tiles for groups of <= 128 rows):
+    // prefetch up to 16 k-blocks of each first-round weight tile
+    a.prefetch_kb = (weight_major_possible && a.swap_max_rows <= 128 && a.BNs <= 128)
+                        ? (a.ph[0].k_blocks < 16 ? a.ph[0].k_blocks : 16) : 0;
     uint32_t stage_bytes = token_major_possible ? 2u * kHalf : 0u;
     if (weight_major_possible) {
         const uint32_t wm = a.xoff + static_cast<uint32_t>(a.BNs) * 64u;

@@ -73,6 +73,7 @@ struct GemmLaunch {
     int64_t dense_rows;
     int64_t max_group_rows;  // host-known upper bound on any group's rows
     int swap_max_rows;       // groups with at most this many rows use weight-major tiles
+    int swap_tokens_max = 128;  // CTA-pair kernel: tokens per weight-major tile, 128 or 256
     bool small_groups;       // mean group below 128 rows: keep token-major tiles narrow
     int bn_max;              // cap on token-major BN (0 = none)
     int nphase;              // 1, or 2: phase 1 of group g starts after phase 0 of g
@@ -145,8 +146,9 @@ struct StatsTail {
     int64_t T;              // tokens the statistics cover (0: the combine's own T)
 };
 
+// y [T, d]: fp32, or bf16 (each value RNE of the fp32 sum) when y_bf16.
 int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const int32_t* inv,
-                   const float* w, int64_t T, int d, int K, float* y, cudaStream_t st,
+                   const float* w, int64_t T, int d, int K, void* y, bool y_bf16, cudaStream_t st,
                    const StatsTail* tail = nullptr);
 // dst[e] = (first ? 0 : dst[e]) + src[e] for e < E (a batch's counts from its chunks').
 int launch_accumulate_counts(int32_t* dst, const int32_t* src, int E, bool first, cudaStream_t st);
@@ -168,6 +170,11 @@ int launch_permute_static(const int32_t* idx, const bf16* x, int64_t T, int d, i
                           bf16* x_perm, int32_t* n_dropped, cudaStream_t st);
 int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alpha, float* bias,
                        cudaStream_t st);
+
+// ------------------------------------------------------------ expert parallelism
+int ep_regroup_max_blocks();
+int launch_ep_regroup(const int32_t* counts, int G, int El, int64_t n, const bf16* in, int d, bf16* out,
+                      int32_t* offsets, int32_t* row_of, cudaStream_t st);
 
 // ------------------------------------------------------------ packing
 int launch_pack(const bf16* W1, const bf16* W3, const bf16* W2, int E, int d, int f, bf16* W13p,

@@ -263,11 +263,13 @@ def router_col_transform(wl: Workload, device="cpu"):
     """(col_scale, col_shift) applied to the router weight columns."""
     E = wl.E
     if wl.skew == "col_scale" and "scales" in wl.skew_params:
-        return torch.tensor(wl.skew_params["scales"], dtype=torch.float32, device=device), None
+        # a workload reduced to its first E experts (a profiling case) keeps their scales
+        return torch.tensor(wl.skew_params["scales"][:E], dtype=torch.float32, device=device), None
     if wl.skew == "hot_shift" and "shift" in wl.skew_params:
         shift = torch.zeros(E, dtype=torch.float32)
         for e in wl.skew_params["hot"]:
-            shift[e] = float(wl.skew_params["shift"])
+            if e < E:
+                shift[e] = float(wl.skew_params["shift"])
         return None, shift.to(device)
     return None, None
 

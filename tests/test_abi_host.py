@@ -70,8 +70,8 @@ def test_null_arguments_are_rejected_before_any_launch(lib):
     nul = None
     assert lib.moe_route(ctypes.byref(d), nul, nul, nul, nul, nul, nul, nul, nul, ws_bytes, nul) == abi.MOE_EINVAL
     assert lib.moe_permute(ctypes.byref(d), nul, nul, nul, nul, nul, nul, nul, nul, nul, nul, 0, nul) == abi.MOE_EINVAL
-    assert lib.moe_combine(ctypes.byref(d), nul, nul, nul, nul, nul) == abi.MOE_EINVAL
-    assert lib.moe_layer_forward(ctypes.byref(d), nul, nul, nul, 0.0, nul, nul, nul, nul, nul, 0, nul) == abi.MOE_EINVAL
+    assert lib.moe_combine(ctypes.byref(d), nul, nul, nul, nul, 0, nul) == abi.MOE_EINVAL
+    assert lib.moe_layer_forward(ctypes.byref(d), nul, nul, nul, 0.0, nul, nul, nul, 0, nul, nul, 0, nul) == abi.MOE_EINVAL
     assert lib.moe_bias_update(ctypes.byref(d), nul, 0.001, nul, nul) == abi.MOE_EINVAL
     assert lib.moe_pack_weights(None, nul, nul, nul, nul, nul, nul) == abi.MOE_EINVAL
 
@@ -154,15 +154,15 @@ def test_chunked_workspace_and_host_checks(lib):
     # a capacity is defined over the whole batch: rejected before any launch
     d = abi.Dims(1000, 128, 256, 8, 2, 1.0).c()
     fake = ctypes.c_void_p(0x10000)   # never dereferenced
-    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 256, fake, fake, None, 0.0, fake, fake, fake, None,
+    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 256, fake, fake, None, 0.0, fake, fake, fake, 0, None,
                                        fake, 1 << 30, None)
     assert st == abi.MOE_EUNSUPPORTED
     d = abi.Dims(1000, 128, 256, 8, 2).c()
-    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 0, fake, fake, None, 0.0, fake, fake, fake, None,
+    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 0, fake, fake, None, 0.0, fake, fake, fake, 0, None,
                                        fake, 1 << 30, None)
     assert st == abi.MOE_EINVAL
     n = abi.moe_chunked_workspace_size(abi.Dims(1000, 128, 256, 8, 2), 256)
-    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 256, fake, fake, None, 0.0, fake, fake, fake, None,
+    st = lib.moe_layer_forward_chunked(ctypes.byref(d), 256, fake, fake, None, 0.0, fake, fake, fake, 0, None,
                                        fake, n - 1, None)
     assert st == abi.MOE_EWORKSPACE
 

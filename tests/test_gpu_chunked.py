@@ -71,3 +71,15 @@ def test_chunked_matches_whole_batch_and_oracle(name, T, chunk, ntok):
     rows = rows[~unc[rows]]
     assert len(rows) >= len(tokens) - 1
     assert_close_y(yb[rows], ref["y"][rows], Y_MAX_ABS, Y_REL_L2, "y (chunked)")
+
+
+def test_chunked_bf16_output_is_rne_of_fp32():
+    inp = LayerInputs(synth.get_workload("mixtral_decode"), T=300)
+    T, d = inp.T, inp.wl.d_model
+    ws = abi.alloc_chunked_workspace(inp.dims, 128)
+    y32 = torch.empty(T, d, dtype=torch.float32, device=dev())
+    y16 = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
+    abi.moe_layer_forward_chunked(inp.dims, 128, inp.x, inp.Wr, None, 0.0, inp.W13p, inp.W2p, y32, ws)
+    abi.moe_layer_forward_chunked(inp.dims, 128, inp.x, inp.Wr, None, 0.0, inp.W13p, inp.W2p, y16, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y16.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16))

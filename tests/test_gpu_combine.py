@@ -81,3 +81,16 @@ def test_load_stats_matches_oracle(T, E, K, with_P):
         assert abs(float(aux.item()) - aux_o) <= 1e-5 * max(1.0, aux_o)
     else:
         assert np.isnan(float(aux.item()))  # not written
+
+
+def test_combine_bf16_output_is_rne_of_fp32():
+    T, K, d = 513, 4, 1024
+    inv, w, Y, N = _combine_inputs(T, K, d, 0.2, seed=11)
+    dims = abi.Dims(T, d, 64, 8, K)
+    args = (Y.to(dev()), torch.from_numpy(inv).to(dev()), torch.from_numpy(w).to(dev()))
+    y32 = torch.empty(T, d, dtype=torch.float32, device=dev())
+    y16 = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
+    abi.moe_combine(dims, *args, y32)
+    abi.moe_combine(dims, *args, y16)
+    torch.cuda.synchronize()
+    assert torch.equal(y16.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16))

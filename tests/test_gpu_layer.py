@@ -156,3 +156,18 @@ def test_layer_full_size_sampled(name, S):
     inv = outs["inv"].cpu().numpy()
     dead = np.all(inv < 0, axis=1)
     assert np.all(yg[dead] == 0)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 64), ("mixtral_decode", 256), ("qwen_capacity", 1000),
+                                    ("deepseek_bias", 300)])
+def test_layer_bf16_output_is_rne_of_fp32(name, T):
+    """The bf16 layer output is, bit for bit, the round-to-nearest-even of the
+    fp32 output of the same call (every step is deterministic)."""
+    inp = LayerInputs(synth.get_workload(name), T=T)
+    d = dev()
+    y32 = torch.empty(T, inp.wl.d_model, dtype=torch.float32, device=d)
+    y16 = torch.empty(T, inp.wl.d_model, dtype=torch.bfloat16, device=d)
+    abi.moe_layer_forward(inp.dims, inp.x, inp.Wr, None, 0.0, inp.W13p, inp.W2p, y32, inp.ws)
+    abi.moe_layer_forward(inp.dims, inp.x, inp.Wr, None, 0.0, inp.W13p, inp.W2p, y16, inp.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y16.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16))
