@@ -375,6 +375,57 @@ def moe_layer(x, Wr, W1, W3, W2, K, capacity_factor=0.0, bias32=None, alpha=0.0,
     return out
 
 
+# ---------------------------------------------------------------------------
+# Offloaded experts: group-wise INT4 storage
+# ---------------------------------------------------------------------------
+
+INT4_GROUP = 64
+
+
+def int4_quantize(W: np.ndarray, group: int = INT4_GROUP):
+    """Group-wise symmetric 4-bit quantization of one expert matrix.
+
+    [P3] section 3.2 (experts offloaded to CPU memory are stored group-wise
+    quantized to INT4 to cut the transfer volume).
+    READING (the page gives no scheme): W is [K_red, N] with the reduction
+    axis first (W1, W3: [d_model, d_ff]; W2: [d_ff, d_model]); a group is
+    `group` consecutive elements along the reduction axis for one column.
+    Per group, in fp32: s = fl32(amax / 7) with amax = max |w| (w the fp32
+    value of each weight), q = clamp(round_half_even(fl32(w / s)), -8, 7);
+    an all-zero group has s = 0 and q = 0.  The divisions are correctly
+    rounded fp32 divisions, so the codes are fixed bit for bit.
+
+    Returns (q int8 [K_red, N], s float32 [K_red / group, N]).
+    """
+    w = np.asarray(W, dtype=np.float32)
+    Kr, N = w.shape
+    if Kr % group != 0:
+        raise ValueError("the reduction length must be a multiple of the group")
+    g = w.reshape(Kr // group, group, N)
+    amax = np.max(np.abs(g), axis=1)                                  # [Kr/group, N] fp32
+    s = (amax / np.float32(7.0)).astype(np.float32)
+    q = np.zeros_like(g, dtype=np.int8)
+    for b in range(Kr // group):
+        for n in range(N):
+            sb = s[b, n]
+            if sb == 0:
+                continue
+            for i in range(group):
+                r = np.float32(g[b, i, n] / sb)                      # fp32 division
+                q[b, i, n] = int(min(7, max(-8, np.rint(r))))         # rint: ties to even
+    return q.reshape(Kr, N), s
+
+
+def int4_dequantize(q: np.ndarray, s: np.ndarray, group: int = INT4_GROUP) -> np.ndarray:
+    """w' = bf16(fl32(q * s)): the fp32 product rounded to bf16 (nearest
+    even), widened to fp64.  The weight value the expert GEMM then uses."""
+    q = np.asarray(q)
+    Kr, N = q.shape
+    srep = np.repeat(np.asarray(s, dtype=np.float32), group, axis=0)  # [Kr, N]
+    prod = (q.astype(np.float32) * srep).astype(np.float32)
+    return bf16_round(prod)
+
+
 def dot_error_bound(x: np.ndarray, Wr: np.ndarray) -> np.ndarray:
     """Rigorous bound on |fp32-accumulated dot product - exact| per logit,
     before the final result is stored.

@@ -433,3 +433,70 @@ def test_capacity_uses_exact_value_of_the_double():
     # 0.8 is stored as 0.8000000000000000444..., so 0.8*30*2/3 is just above 16
     assert O.capacity(30, 2, 3, 0.8) == 17
     assert O.capacity(30, 2, 3, 0.75) == 15
+
+
+# ---------------------------------------------------------------------------
+# group-wise INT4 storage of offloaded experts
+# ---------------------------------------------------------------------------
+
+def test_int4_exact_round_trip_on_the_code_grid():
+    """Weights already on the grid q * 2^-7 with |q| reaching 7 in every
+    group: s is exactly 2^-7, the codes come back unchanged and the
+    dequantized weights equal the originals."""
+    rng = np.random.default_rng(0)
+    q0 = rng.integers(-7, 8, size=(128, 5))
+    q0[0::64, :] = 7            # every group holds a 7
+    W = q0 * 2.0 ** -7
+    q, s = O.int4_quantize(W)
+    assert s.shape == (2, 5) and np.all(s == np.float32(2.0 ** -7))
+    assert np.array_equal(q, q0)
+    assert np.array_equal(O.int4_dequantize(q, s), W)
+
+
+def test_int4_groups_run_along_the_reduction_axis():
+    """Scales are the per-(64-row block, column) maxima / 7, computed here by
+    plain loops; a group with a large weight does not affect its neighbours."""
+    rng = np.random.default_rng(1)
+    W = (rng.standard_normal((192, 3)) * 0.02).astype(np.float32).astype(np.float64)
+    W[70, 1] = 5.0
+    q, s = O.int4_quantize(W)
+    for b in range(3):
+        for n in range(3):
+            amax = max(abs(float(np.float32(W[b * 64 + i, n]))) for i in range(64))
+            assert s[b, n] == np.float32(np.float32(amax) / np.float32(7.0))
+    assert s[1, 1] == np.float32(np.float32(5.0) / np.float32(7.0))
+    assert s[1, 0] < 0.1 and s[0, 1] < 0.1 and s[2, 1] < 0.1
+
+
+def test_int4_codes_are_nearest_with_the_extreme_at_seven():
+    rng = np.random.default_rng(2)
+    W = rng.standard_normal((256, 7)) * 0.05
+    W[:64, 3] = 0.0                                    # an all-zero group
+    q, s = O.int4_quantize(W)
+    assert q.dtype == np.int8 and q.min() >= -8 and q.max() <= 7
+    assert np.all(q[:64, 3] == 0) and s[0, 3] == 0
+    srep = np.repeat(s.astype(np.float64), 64, axis=0)
+    w32 = W.astype(np.float32).astype(np.float64)
+    # nearest code: within half a step (plus the fp32 division's rounding)
+    assert np.all(np.abs(w32 - q * srep) <= 0.5 * srep * (1 + 2.0 ** -20) + 1e-30)
+    # sign kept; the largest magnitude of each group maps to +-7
+    assert np.all((q == 0) | (np.sign(q) == np.sign(w32)))
+    g = np.abs(w32).reshape(4, 64, 7)
+    arg = g.argmax(axis=1)
+    for b in range(4):
+        for n in range(7):
+            if s[b, n] > 0:
+                assert abs(int(q[b * 64 + arg[b, n], n])) == 7
+    # monotone within a group
+    for n in range(7):
+        order = np.argsort(w32[64:128, n], kind="stable")
+        assert np.all(np.diff(q[64:128, n][order].astype(int)) >= 0)
+
+
+def test_int4_dequantize_rounds_the_fp32_product_to_bf16():
+    # q = 3, s = fl32(0.1): 3 s = 0.30000000447... in fp32, 1.0011001|1001.. x 2^-2,
+    # rounded up to 1.0011010 x 2^-2 = 0.30078125 in bf16
+    q = np.full((64, 1), 3, np.int8)
+    s = np.array([[0.1]], np.float32)
+    assert np.all(O.int4_dequantize(q, s) == 0.30078125)
+    assert np.all(O.int4_dequantize(-q, s) == -0.30078125)
