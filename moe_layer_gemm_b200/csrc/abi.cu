@@ -393,7 +393,7 @@ int moe_get_device_status(const void* ws, void* stream, int* status, int* detail
             cudaSuccess ||
         cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return MOE_ECUDA;
-    *status = host == 0 ? MOE_OK : (host == DEV_BAD_INDEX ? MOE_EINDEX : MOE_ETIMEOUT);
+    *status = host == 0 ? MOE_OK : (host == DEV_BAD_INDEX || host == DEV_BAD_SLOT ? MOE_EINDEX : MOE_ETIMEOUT);
     if (detail) *detail = host;
     return MOE_OK;
 }
@@ -481,6 +481,70 @@ int moe_expert_ffn(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* 
         MOE_TRY(map_launch(launch_reduce_splits(yout, L.nsplit, dims->T * dims->K * dims->d_model, offsets, dims->E,
                                                 dims->d_model, y_perm, st)));
     return MOE_OK;
+}
+
+int moe_expert_ffn_slots(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets,
+                         const int32_t* expert_slot, int n_slots, const moe_bf16* W13c, const moe_bf16* W2c,
+                         moe_bf16* h, float* y_perm, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!x_perm || !offsets || !expert_slot || !W13c || !W2c || !h || !y_perm || n_slots < 1) return MOE_EINVAL;
+    if (!aligned16(x_perm) || !aligned16(W13c) || !aligned16(W2c) || !aligned16(h) || !aligned16(y_perm))
+        return MOE_EUNSUPPORTED;
+    MOE_TRY(check_ws(dims, ws, ws_bytes));
+    const Layout L = layout_of(dims);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* yout = L.nsplit > 1 ? at<float>(ws, L.yperm) : y_perm;
+    if (cudaMemsetAsync(at<int>(ws, L.sched_ffn), 0, gemm_sched_bytes(dims->E), st) != cudaSuccess) return MOE_ECUDA;
+    GemmLaunch g = ffn_launch(dims, L, reinterpret_cast<const bf16*>(x_perm), offsets,
+                              reinterpret_cast<const bf16*>(W13c), reinterpret_cast<const bf16*>(W2c),
+                              reinterpret_cast<bf16*>(h), yout, L.nsplit, ws);
+    g.w_slot = expert_slot;
+    g.w_slots = n_slots;
+    if (ffn_uses_pair(dims, L, g)) {
+        MOE_TRY(map_launch(launch_grouped_gemm_2sm(g, st)));
+    } else {
+        if (L.swap == 2) g.swap_max_rows = 0;
+        MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
+    }
+    if (L.nsplit > 1)
+        MOE_TRY(map_launch(launch_reduce_splits(yout, L.nsplit, dims->T * dims->K * dims->d_model, offsets, dims->E,
+                                                dims->d_model, y_perm, st)));
+    return MOE_OK;
+}
+
+int moe_int4_bytes(const moe_dims* dims, size_t* q13_bytes, size_t* s13_bytes, size_t* q2_bytes, size_t* s2_bytes) {
+    MOE_TRY(check_dims(dims));
+    if (!q13_bytes || !s13_bytes || !q2_bytes || !s2_bytes) return MOE_EINVAL;
+    int4_sizes(dims->E, dims->d_model, dims->d_ff, q13_bytes, s13_bytes, q2_bytes, s2_bytes);
+    return MOE_OK;
+}
+
+int moe_int4_pack(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2, uint8_t* q13,
+                  float* s13, uint8_t* q2, float* s2, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (!W1 || !W3 || !W2 || !q13 || !s13 || !q2 || !s2) return MOE_EINVAL;
+    if (dims->d_model % 64 != 0 || dims->d_ff % 64 != 0) return MOE_EUNSUPPORTED;  // whole 64-element groups
+    if (!aligned16(q13) || !aligned16(q2) || !aligned16(s13) || !aligned16(s2)) return MOE_EUNSUPPORTED;
+    return map_launch(launch_int4_pack(reinterpret_cast<const bf16*>(W1), reinterpret_cast<const bf16*>(W3),
+                                       reinterpret_cast<const bf16*>(W2), dims->E, dims->d_model, dims->d_ff, q13, s13,
+                                       q2, s2, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_int4_unpack(const moe_dims* dims, int n_jobs, const int32_t* job_expert, const int32_t* job_slot,
+                    const uint8_t* q13, const float* s13, const uint8_t* q2, const float* s2, int n_slots,
+                    moe_bf16* W13c, moe_bf16* W2c, void* stream) {
+    MOE_TRY(check_dims(dims));
+    if (n_jobs < 0 || n_slots < 1) return MOE_EINVAL;
+    if (n_jobs == 0) return MOE_OK;
+    if (!job_expert || !job_slot || !q13 || !s13 || !q2 || !s2 || !W13c || !W2c) return MOE_EINVAL;
+    if (dims->d_model % 64 != 0 || dims->d_ff % 64 != 0) return MOE_EUNSUPPORTED;
+    if (!aligned16(q13) || !aligned16(q2) || !aligned16(W13c) || !aligned16(W2c)) return MOE_EUNSUPPORTED;
+    for (int j = 0; j < n_jobs; ++j)
+        if (job_expert[j] < 0 || job_expert[j] >= dims->E || job_slot[j] < 0 || job_slot[j] >= n_slots)
+            return MOE_EINVAL;
+    return map_launch(launch_int4_unpack(n_jobs, job_expert, job_slot, dims->d_model, dims->d_ff, q13, s13, q2, s2,
+                                         reinterpret_cast<bf16*>(W13c), reinterpret_cast<bf16*>(W2c),
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 int moe_permute_noalloc(const moe_dims* dims, const int32_t* topk_idx, const moe_bf16* x, int32_t* counts,

@@ -79,6 +79,8 @@ struct DevArgs {
     uint32_t wait_limit;      // polls of a bounded mbarrier or drain wait
     uint32_t dep_wait_limit;  // polls of the phase-1 readiness wait
     int dep_extra;            // added to the phase-1 readiness target (0; a test makes it unreachable)
+    const int32_t* w_slot;    // group -> weight matrix (expert cache slot), or nullptr
+    int w_slots;
 };
 
 struct Maps {
@@ -317,6 +319,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                     fence_proxy_async_global();
                     if (!ok) break;
                 }
+                const int wg = weight_slot(a.w_slot, a.w_slots, t.g, a.status);
                 const int nb = t.swap ? (t.rows + 31) / 32 : 0;
                 const uint32_t wbytes = t.swap ? 16384u : static_cast<uint32_t>(pa.BN) * 128u;
                 const uint32_t xbytes = t.swap ? static_cast<uint32_t>(nb) * 4096u : kTileABytes;
@@ -331,7 +334,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                     const int kx = kb * kBK;
                     if (t.swap) {
                         // weights (M side): one contiguous 16 KB tile, streamed once
-                        bulk_load(dW, weight_rows(pa, t.g, t.n0, kb), 16384u, &full[s], pol_first);
+                        bulk_load(dW, weight_rows(pa, wg, t.n0, kb), 16384u, &full[s], pol_first);
                         for (int j = 0; j < nb; ++j)
                             tma_load_2d(&maps.tokB[t.phase], dX + j * 4096, &full[s], kx,
                                         static_cast<int32_t>(t.row0 + 32 * j), pol_last);
@@ -342,10 +345,10 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                         tma_load_2d(&maps.tokA[t.phase], dX, &full[s], kx, static_cast<int32_t>(t.row0), pol_last);
                         if (pa.BN >= 128) {
                             for (int j = 0; j < pa.BN / 128; ++j)
-                                bulk_load(dW + j * 16384, weight_rows(pa, t.g, t.n0 + 128 * j, kb), 16384u, &full[s],
+                                bulk_load(dW + j * 16384, weight_rows(pa, wg, t.n0 + 128 * j, kb), 16384u, &full[s],
                                           pol_first);
                         } else {
-                            bulk_load(dW, weight_rows(pa, t.g, t.n0, kb), wbytes, &full[s], pol_first);
+                            bulk_load(dW, weight_rows(pa, wg, t.n0, kb), wbytes, &full[s], pol_first);
                         }
                     }
                     issued_mask |= 1u << s;
@@ -571,6 +574,9 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
     a.wait_limit = L.wait_limit ? L.wait_limit : kWaitLimit;
     a.dep_wait_limit = L.dep_wait_limit ? L.dep_wait_limit : kWaitLimit;
     a.dep_extra = L.dep_extra;
+    a.w_slot = L.w_slot;
+    a.w_slots = L.w_slots;
+    if (L.w_slot && L.w_slots < 1) return -2;
     const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
     a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
     {

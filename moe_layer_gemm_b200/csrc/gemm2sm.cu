@@ -96,6 +96,8 @@ struct Args2 {
     uint32_t dep_wait_limit;  // polls of the phase-1 readiness wait
     int dep_extra;            // added to the phase-1 readiness target (0; a test makes it unreachable)
     int prefetch_kb;          // k-blocks of the first-round weight tiles pulled into L2 before the wait (0: none)
+    const int32_t* w_slot;    // group -> weight matrix (expert cache slot), or nullptr
+    int w_slots;
 };
 
 constexpr int kMaxStages = 16;
@@ -428,7 +430,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     if (!ok) break;
                 }
                 // this CTA's 128-row weight block of (sub-)tile j: rows n0 + 256 j + 128 rank
-                const int64_t wblk0 = static_cast<int64_t>(t.g) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
+                const int wg = weight_slot(a.w_slot, a.w_slots, t.g, a.status);
+                const int64_t wblk0 = static_cast<int64_t>(wg) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
                 // weight-major: the MMA's N is the tile's tokens rounded up to 16;
                 // this CTA holds N / 2 of them (a multiple of 8), loaded in 16-row boxes
                 const int half = t.swap ? ((t.rows + 15) / 16) * 8 : 0;
@@ -716,6 +719,9 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     a.wait_limit = L.wait_limit ? L.wait_limit : kWaitLimit;
     a.dep_wait_limit = L.dep_wait_limit ? L.dep_wait_limit : kWaitLimit;
     a.dep_extra = L.dep_extra;
+    a.w_slot = L.w_slot;
+    a.w_slots = L.w_slots;
+    if (L.w_slot && L.w_slots < 1) return -2;
     const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
     a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
     // weight-major tiles take up to 128 tokens, or 256 when the launch asks
@@ -760,7 +766,8 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
         if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
         if (!map2(&maps.tok16[p], g.tok, trows, g.Kdim, 16u, true)) return -3;
-        const uint64_t wrows = static_cast<uint64_t>(L.G) * ph.nb * ph.k_blocks * 128;
+        const uint64_t wmats = static_cast<uint64_t>(L.w_slot ? L.w_slots : L.G);
+        const uint64_t wrows = wmats * ph.nb * ph.k_blocks * 128;
         if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
     }
     const size_t fixed = 1024 + static_cast<size_t>(2 * kMaxStages + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
@@ -772,7 +779,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     a.xoff = static_cast<uint32_t>(wt_max) * kHalf;
     // decode-sized launches (weight-major tiles for groups of <= 128 rows):
     // prefetch up to 16 k-blocks of each first-round weight tile
-    a.prefetch_kb = (weight_major_possible && a.swap_max_rows <= 128 && a.BNs <= 128)
+    a.prefetch_kb = (weight_major_possible && a.swap_max_rows <= 128 && a.BNs <= 128 && L.w_slot == nullptr)
                         ? (a.ph[0].k_blocks < 16 ? a.ph[0].k_blocks : 16) : 0;
     uint32_t stage_bytes = token_major_possible ? 2u * kHalf : 0u;
     if (weight_major_possible) {

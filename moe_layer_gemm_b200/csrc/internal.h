@@ -86,6 +86,10 @@ struct GemmLaunch {
     uint32_t wait_limit = 0;
     uint32_t dep_wait_limit = 0;
     int dep_extra = 0;
+    // Expert cache: group g's weights are matrix w_slot[g] of the phase's
+    // buffer, which holds w_slots matrices (nullptr: matrix g of G).
+    const int32_t* w_slot = nullptr;
+    int w_slots = 0;
 };
 
 // Test-only settings of the expert-GEMM launches (see moe_test_set_wait_limits
@@ -175,6 +179,14 @@ int launch_bias_update(const int32_t* counts, int64_t T, int E, int K, float alp
 int ep_regroup_max_blocks();
 int launch_ep_regroup(const int32_t* counts, int G, int El, int64_t n, const bf16* in, int d, bf16* out,
                       int32_t* offsets, int32_t* row_of, cudaStream_t st);
+
+// ------------------------------------------------------------ offloaded experts (INT4)
+void int4_sizes(int E, int d, int f, size_t* q13, size_t* s13, size_t* q2, size_t* s2);
+int launch_int4_pack(const bf16* W1, const bf16* W3, const bf16* W2, int E, int d, int f, uint8_t* q13, float* s13,
+                     uint8_t* q2, float* s2, cudaStream_t st);
+int launch_int4_unpack(int n_jobs, const int32_t* job_expert, const int32_t* job_slot, int d, int f,
+                       const uint8_t* q13, const float* s13, const uint8_t* q2, const float* s2, bf16* W13c,
+                       bf16* W2c, cudaStream_t st);
 
 // ------------------------------------------------------------ packing
 int launch_pack(const bf16* W1, const bf16* W3, const bf16* W2, int E, int d, int f, bf16* W13p,

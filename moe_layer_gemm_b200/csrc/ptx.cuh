@@ -19,7 +19,19 @@ enum : int {
     DEV_TIMEOUT_DRAIN = 5,
     DEV_TIMEOUT_DEPENDENCY = 6,
     DEV_BAD_INDEX = 7,  // a dispatch input named an expert outside [0, E); the slot was skipped
+    DEV_BAD_SLOT = 8,   // an expert with rows had no valid cache slot; slot 0 was read instead
 };
+
+// Weight matrix of group g: g itself, or its cache slot from `slot_of`
+// (nullptr: none).  A slot outside [0, n_slots) is never used as an address:
+// the status records DEV_BAD_SLOT and slot 0 is read instead.
+__device__ __forceinline__ int weight_slot(const int32_t* slot_of, int n_slots, int g, int* status) {
+    if (slot_of == nullptr) return g;
+    const int s = slot_of[g];
+    if (static_cast<unsigned>(s) < static_cast<unsigned>(n_slots)) return s;
+    atomicCAS(status, 0, DEV_BAD_SLOT);
+    return 0;
+}
 
 // Default poll limit of a bounded wait: about a few seconds on a B200
 // before it gives up.  Launches pass their limit to the kernels (a test can

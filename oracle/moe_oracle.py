@@ -426,6 +426,103 @@ def int4_dequantize(q: np.ndarray, s: np.ndarray, group: int = INT4_GROUP) -> np
     return bf16_round(prod)
 
 
+def lru_expert_cache(needed_per_step, n_slots: int, prefetch_per_step=None):
+    """The LRU expert cache of [P3] section 3.2, step by step.
+
+    [P3] section 3.2: keep the frequently used experts in a cache in GPU
+    memory (LRU), and load the experts predicted for the next batch ahead of
+    time.  READING (the page gives no algorithm):
+      - before step t's expert computation every needed expert is resident;
+        a hit refreshes its slot's last use to t;
+      - misses, in ascending expert order, each take the slot with the
+        smallest (last use, slot index) among the slots that hold no expert
+        needed at step t; an empty slot has last use -1;
+      - after step t, the experts of prefetch_per_step[t] (the prediction for
+        step t + 1, in order) that are not resident are loaded the same way,
+        into slots holding no expert used at step t, with last use t;
+      - a step needing more experts than there are slots is an error.
+    Returns one dict per step: hits (resident before the step and not loaded
+    by the previous step's prefetch), prefetch_hits (loaded by that
+    prefetch), misses (loaded on demand) as sorted expert lists, loads and
+    prefetch_loads as [(expert, slot)], and slot_of {expert: slot} after the
+    step's demand loads.
+    """
+    expert_of = [-1] * n_slots
+    last_use = [-1] * n_slots
+    slot_of = {}
+    prefetched = set()
+    out = []
+    for t, needed in enumerate(needed_per_step):
+        need = sorted(set(int(e) for e in needed))
+        if len(need) > n_slots:
+            raise ValueError(f"step {t} needs {len(need)} experts, the cache has {n_slots} slots")
+        hits = [e for e in need if e in slot_of and e not in prefetched]
+        phits = [e for e in need if e in slot_of and e in prefetched]
+        misses = [e for e in need if e not in slot_of]
+        for e in need:
+            if e in slot_of:
+                last_use[slot_of[e]] = t
+        loads = []
+        needset = set(need)
+
+        def take(t_use, protect):
+            cands = [(last_use[sl], sl) for sl in range(n_slots) if expert_of[sl] not in protect]
+            return min(cands)[1] if cands else None
+
+        for e in misses:
+            sl = take(t, needset)
+            old = expert_of[sl]
+            if old >= 0:
+                del slot_of[old]
+            expert_of[sl] = e
+            slot_of[e] = sl
+            last_use[sl] = t
+            loads.append((e, sl))
+        snapshot = dict(slot_of)
+        ploads = []
+        prefetched = set()
+        if prefetch_per_step is not None:
+            for e in prefetch_per_step[t]:
+                e = int(e)
+                if e in slot_of:
+                    continue
+                sl = take(t, needset)
+                if sl is None:
+                    break
+                old = expert_of[sl]
+                if old >= 0:
+                    del slot_of[old]
+                expert_of[sl] = e
+                slot_of[e] = sl
+                last_use[sl] = t
+                ploads.append((e, sl))
+                prefetched.add(e)
+        out.append(dict(hits=hits, prefetch_hits=phits, misses=misses, loads=loads, prefetch_loads=ploads,
+                        slot_of=snapshot))
+    return out
+
+
+def routing_history_prediction(counts_per_step, width: int, beta: float = 0.75):
+    """Experts predicted for the next step from the routing history.
+
+    [P3] section 3.2 (predict from the routing history which experts the next
+    batch needs, and load them ahead of time).  READING: a per-expert
+    exponential moving average of the routed token counts, in fp32:
+    c_e <- fl32(fl32(beta * c_e) + n_e(t)) with c_e = 0 before step 0; the
+    prediction after step t is the `width` experts with the largest c_e
+    (equal values: lower expert index first), in that order.
+    """
+    c = None
+    b = np.float32(beta)
+    preds = []
+    for n in counts_per_step:
+        n = np.asarray(n, dtype=np.float32)
+        c = n.copy() if c is None else (b * c + n).astype(np.float32)
+        order = np.argsort(-c, kind="stable")
+        preds.append([int(e) for e in order[:width]])
+    return preds
+
+
 def dot_error_bound(x: np.ndarray, Wr: np.ndarray) -> np.ndarray:
     """Rigorous bound on |fp32-accumulated dot product - exact| per logit,
     before the final result is stored.
