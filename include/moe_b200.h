@@ -119,7 +119,8 @@ MOE_API int moe_reset_device_status(void* ws, void* stream);
  * *status = MOE_OK; MOE_ETIMEOUT with *detail naming the wait that ran out
  * (a small integer, 1..6); or MOE_EINDEX (*detail = 7) when a dispatch input
  * named an expert outside [0, E).  The first failure recorded wins; the
- * flag stays set until moe_reset_device_status. */
+ * flag stays set until moe_reset_device_status.  MOE_EINDEX with detail 8
+ * means an expert with rows had no valid cache slot (moe_expert_ffn_slots). */
 MOE_API int moe_get_device_status(const void* ws, void* stream, int* status, int* detail);
 
 /* Bytes of the packed expert weights moe_pack_weights writes for these dims:
@@ -373,6 +374,52 @@ MOE_API int moe_layer_forward_chunked(const moe_dims* dims, int64_t chunk_tokens
 MOE_API int moe_ep_regroup(int n_ranks, int E_local, const int32_t* recv_counts, int64_t n_rows, int d_model,
                            const moe_bf16* rows_in, moe_bf16* rows_out, int32_t* offsets, int32_t* row_of,
                            void* stream);
+
+/* Expert offloading ([P3] section 3.2: when the experts do not all fit in
+ * GPU memory, keep some in host memory, group-wise quantized to INT4 to cut
+ * the transfer volume, with an LRU cache of experts in GPU memory and
+ * prefetching predicted from the routing history).  The cache's bookkeeping
+ * (which expert sits in which slot) is the caller's; these calls move and
+ * use the weights.
+ *
+ * INT4 format.  Codes follow the packed weight layout of moe_pack_weights:
+ * for every 128-row x 64-column tile of an expert's packed matrix, 4096
+ * bytes of 4-bit two's-complement codes (tile element i, in the tile's own
+ * swizzled order, in the low nibble of byte i / 2 for even i, the high
+ * nibble for odd i) and 128 fp32 scales, one per tile row.  A tile row's 64
+ * elements form one group: 64 consecutive weights along the reduction axis
+ * of one output column.  Per group, in fp32: s = amax / 7, q =
+ * clamp(round_half_even(w / s), -8, 7) (correctly rounded divisions); an
+ * all-zero group has s = 0.  The weight a GEMM uses is bf16(q * s), the
+ * fp32 product rounded to nearest even.  Requires d_model % 64 == 0 and
+ * d_ff % 64 == 0.
+ *
+ * moe_int4_bytes: sizes of the codes and scales of all E experts (host only).
+ * moe_int4_pack: quantize W1, W3 [E, d_model, d_ff] and W2 [E, d_ff, d_model]
+ *   (bf16, device) into q13/s13 and q2/s2 (device); a load-time step.
+ * moe_int4_unpack: for each job j, expand expert job_expert[j]'s codes into
+ *   cache slot job_slot[j] of W13c / W2c (each n_slots experts of packed
+ *   weights, moe_packed_weight_bytes / E bytes per slot).  job_expert and
+ *   job_slot are HOST arrays of n_jobs entries, checked against E and
+ *   n_slots before any launch.  q13, s13, q2, s2 may be device memory or
+ *   page-locked host memory mapped into the device's address space (read
+ *   directly by the kernel over the host link: no staging copy); other host
+ *   memory is refused with MOE_EUNSUPPORTED before any launch.
+ * moe_expert_ffn_slots: moe_expert_ffn with the weights of expert e read
+ *   from slot expert_slot[e] ([E] int32, device) of W13c / W2c.  An expert
+ *   with rows whose slot lies outside [0, n_slots) is never used as an
+ *   address: slot 0 is read instead and the workspace status flag records
+ *   MOE_EINDEX (detail 8). */
+MOE_API int moe_int4_bytes(const moe_dims* dims, size_t* q13_bytes, size_t* s13_bytes, size_t* q2_bytes,
+                           size_t* s2_bytes);
+MOE_API int moe_int4_pack(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                          uint8_t* q13, float* s13, uint8_t* q2, float* s2, void* stream);
+MOE_API int moe_int4_unpack(const moe_dims* dims, int n_jobs, const int32_t* job_expert, const int32_t* job_slot,
+                            const uint8_t* q13, const float* s13, const uint8_t* q2, const float* s2, int n_slots,
+                            moe_bf16* W13c, moe_bf16* W2c, void* stream);
+MOE_API int moe_expert_ffn_slots(const moe_dims* dims, const moe_bf16* x_perm, const int32_t* offsets,
+                                 const int32_t* expert_slot, int n_slots, const moe_bf16* W13c, const moe_bf16* W2c,
+                                 moe_bf16* h, float* y_perm, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -34,7 +34,8 @@ EXPORTED = [
     "moe_expert_ffn", "moe_combine", "moe_load_stats", "moe_bias_update", "moe_layer_forward",
     "moe_layer_launch_count", "moe_packed_weight_bytes", "moe_permute_noalloc", "moe_ffn_kernel",
     "moe_chunked_workspace_size", "moe_layer_forward_chunked", "moe_layer_chunked_launch_count",
-    "moe_test_set_wait_limits", "moe_ep_regroup",
+    "moe_test_set_wait_limits", "moe_ep_regroup", "moe_int4_bytes", "moe_int4_pack", "moe_int4_unpack",
+    "moe_expert_ffn_slots",
 ]
 NUM_STAGE_EVENTS = 6
 
@@ -95,6 +96,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                           ctypes.POINTER(moe_layer_outputs), P, SZ, P]),
         "moe_test_set_wait_limits": (I, [ctypes.c_int64, ctypes.c_int64, I]),
         "moe_ep_regroup": (I, [I, I, P, I64, I, P, P, P, P, P]),
+        "moe_int4_bytes": (I, [dims_p, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ),
+                               ctypes.POINTER(SZ)]),
+        "moe_int4_pack": (I, [dims_p, P, P, P, P, P, P, P, P]),
+        "moe_int4_unpack": (I, [dims_p, I, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                P, P, P, P, I, P, P, P]),
+        "moe_expert_ffn_slots": (I, [dims_p, P, P, P, I, P, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -353,6 +360,53 @@ def moe_ep_regroup(n_ranks: int, E_local: int, recv_counts, rows_in, rows_out, o
         int(n_ranks), int(E_local), _ptr(recv_counts, I32, "recv_counts"), ctypes.c_int64(n), d,
         _ptr(rows_in, BF16, "rows_in") if n else None, _ptr(rows_out, BF16, "rows_out") if n else None,
         _ptr(offsets, I32, "offsets"), _ptr(row_of, I32, "row_of") if n else None, _stream(stream)))
+
+
+def moe_int4_bytes(dims):
+    """(q13, s13, q2, s2) byte counts of all experts' INT4 codes and scales."""
+    v = [ctypes.c_size_t(0) for _ in range(4)]
+    _check("moe_int4_bytes", load().moe_int4_bytes(ctypes.byref(_dims(dims)), *[ctypes.byref(x) for x in v]))
+    return tuple(int(x.value) for x in v)
+
+
+def _any_ptr(t, dtype, name):
+    """Pointer of a device tensor or of a page-locked host tensor."""
+    if t.device.type == "cpu":
+        if not t.is_pinned():
+            raise ValueError(f"{name}: a host tensor must be page-locked (pin_memory)")
+        if t.dtype != dtype or not t.is_contiguous():
+            raise TypeError(f"{name}: expected a contiguous {dtype} tensor")
+        return t.data_ptr()
+    return _ptr(t, dtype, name)
+
+
+def moe_int4_pack(dims, W1, W3, W2, q13, s13, q2, s2, stream=None):
+    _check("moe_int4_pack", load().moe_int4_pack(
+        ctypes.byref(_dims(dims)), _ptr(W1, BF16, "W1"), _ptr(W3, BF16, "W3"), _ptr(W2, BF16, "W2"),
+        _ptr(q13, torch.uint8, "q13"), _ptr(s13, F32, "s13"), _ptr(q2, torch.uint8, "q2"), _ptr(s2, F32, "s2"),
+        _stream(stream)))
+
+
+def moe_int4_unpack(dims, experts, slots, q13, s13, q2, s2, n_slots: int, W13c, W2c, stream=None):
+    """Expand experts[j]'s INT4 codes into cache slot slots[j] (host lists)."""
+    n = len(experts)
+    if n != len(slots):
+        raise ValueError("experts and slots differ in length")
+    if n == 0:
+        return
+    je = (ctypes.c_int32 * n)(*[int(e) for e in experts])
+    js = (ctypes.c_int32 * n)(*[int(s) for s in slots])
+    _check("moe_int4_unpack", load().moe_int4_unpack(
+        ctypes.byref(_dims(dims)), n, je, js, _any_ptr(q13, torch.uint8, "q13"), _any_ptr(s13, F32, "s13"),
+        _any_ptr(q2, torch.uint8, "q2"), _any_ptr(s2, F32, "s2"), int(n_slots), _ptr(W13c, BF16, "W13c"),
+        _ptr(W2c, BF16, "W2c"), _stream(stream)))
+
+
+def moe_expert_ffn_slots(dims, x_perm, offsets, expert_slot, n_slots: int, W13c, W2c, h, y_perm, ws, stream=None):
+    _check("moe_expert_ffn_slots", load().moe_expert_ffn_slots(
+        ctypes.byref(_dims(dims)), _ptr(x_perm, BF16, "x_perm"), _ptr(offsets, I32, "offsets"),
+        _ptr(expert_slot, I32, "expert_slot"), int(n_slots), _ptr(W13c, BF16, "W13c"), _ptr(W2c, BF16, "W2c"),
+        _ptr(h, BF16, "h"), _ptr(y_perm, F32, "y_perm"), _ptr(ws, None, "ws"), ws.numel(), _stream(stream)))
 
 
 # ---------------------------------------------------------------- helpers

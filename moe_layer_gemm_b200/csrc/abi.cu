@@ -530,6 +530,27 @@ int moe_int4_pack(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3, 
                                        q2, s2, static_cast<cudaStream_t>(stream)));
 }
 
+// The address a kernel may use for `p`: device (or managed) memory as is,
+// page-locked host memory through its mapped device pointer.  Anything else
+// (pageable host memory, an unmapped registration) is refused, so no kernel
+// is handed an address it cannot reach.
+int device_view(const void* p, const void** out) {
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_EUNSUPPORTED;
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+        *out = p;
+        return MOE_OK;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
+        *out = at.devicePointer;
+        return MOE_OK;
+    }
+    return MOE_EUNSUPPORTED;
+}
+
 int moe_int4_unpack(const moe_dims* dims, int n_jobs, const int32_t* job_expert, const int32_t* job_slot,
                     const uint8_t* q13, const float* s13, const uint8_t* q2, const float* s2, int n_slots,
                     moe_bf16* W13c, moe_bf16* W2c, void* stream) {
@@ -542,7 +563,15 @@ int moe_int4_unpack(const moe_dims* dims, int n_jobs, const int32_t* job_expert,
     for (int j = 0; j < n_jobs; ++j)
         if (job_expert[j] < 0 || job_expert[j] >= dims->E || job_slot[j] < 0 || job_slot[j] >= n_slots)
             return MOE_EINVAL;
-    return map_launch(launch_int4_unpack(n_jobs, job_expert, job_slot, dims->d_model, dims->d_ff, q13, s13, q2, s2,
+    const void *dq13 = nullptr, *ds13 = nullptr, *dq2 = nullptr, *ds2 = nullptr;
+    MOE_TRY(device_view(q13, &dq13));
+    MOE_TRY(device_view(s13, &ds13));
+    MOE_TRY(device_view(q2, &dq2));
+    MOE_TRY(device_view(s2, &ds2));
+    if (!aligned16(dq13) || !aligned16(dq2)) return MOE_EUNSUPPORTED;
+    return map_launch(launch_int4_unpack(n_jobs, job_expert, job_slot, dims->d_model, dims->d_ff,
+                                         static_cast<const uint8_t*>(dq13), static_cast<const float*>(ds13),
+                                         static_cast<const uint8_t*>(dq2), static_cast<const float*>(ds2),
                                          reinterpret_cast<bf16*>(W13c), reinterpret_cast<bf16*>(W2c),
                                          static_cast<cudaStream_t>(stream)));
 }

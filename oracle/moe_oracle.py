@@ -403,16 +403,11 @@ def int4_quantize(W: np.ndarray, group: int = INT4_GROUP):
         raise ValueError("the reduction length must be a multiple of the group")
     g = w.reshape(Kr // group, group, N)
     amax = np.max(np.abs(g), axis=1)                                  # [Kr/group, N] fp32
-    s = (amax / np.float32(7.0)).astype(np.float32)
-    q = np.zeros_like(g, dtype=np.int8)
-    for b in range(Kr // group):
-        for n in range(N):
-            sb = s[b, n]
-            if sb == 0:
-                continue
-            for i in range(group):
-                r = np.float32(g[b, i, n] / sb)                      # fp32 division
-                q[b, i, n] = int(min(7, max(-8, np.rint(r))))         # rint: ties to even
+    s = (amax / np.float32(7.0)).astype(np.float32)                   # fp32 division
+    safe = np.where(s > 0, s, np.float32(1.0))[:, None, :]
+    r = (g / safe).astype(np.float32)                                 # fp32 division per weight
+    q = np.clip(np.rint(r), -8, 7).astype(np.int8)                    # rint: ties to even
+    q = np.where((s > 0)[:, None, :], q, np.int8(0))
     return q.reshape(Kr, N), s
 
 
