@@ -471,14 +471,21 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 for (int c = 0; c < nb; ++c) {
                     tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
                     if (pa.epi == EPI_SWIGLU_BF16) {
+                        // lane l < 16 holds gate row f0 + l and lane l + 16 the up
+                        // row of the same f, each for 32 tokens.  The half-warps
+                        // split the tokens: lane l finishes token j, lane l + 16
+                        // token j + 16, after one exchange per token pair, so each
+                        // lane computes 16 SiLUs and every store writes for both.
+                        const bool hi = lane >= 16;
                         const int f = t.n0 / 2 + q * 16 + (lane & 15);
-                        bf16* H = static_cast<bf16*>(pa.out);
+                        const int tok0 = c * 32 + (hi ? 16 : 0);
+                        bf16* H = static_cast<bf16*>(pa.out) + (t.row0 + tok0) * pa.ldo + f;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float u = __shfl_xor_sync(0xffffffffu, v[j], 16);
-                            const int tok = c * 32 + j;
-                            if (lane < 16 && tok < t.rows)
-                                H[(t.row0 + tok) * pa.ldo + f] = __float2bfloat16_rn(silu_f(v[j]) * u);
+                        for (int j = 0; j < 16; ++j) {
+                            const float other = __shfl_xor_sync(0xffffffffu, hi ? v[j] : v[j + 16], 16);
+                            const float g = hi ? other : v[j];
+                            const float u = hi ? v[j + 16] : other;
+                            if (tok0 + j < t.rows) H[static_cast<int64_t>(j) * pa.ldo] = __float2bfloat16_rn(silu_f(g) * u);
                         }
                     } else {
                         float* Y = static_cast<float*>(pa.out) + static_cast<int64_t>(t.split) * pa.split_stride;

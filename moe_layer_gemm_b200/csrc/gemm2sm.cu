@@ -113,6 +113,7 @@ struct PeerReport {
 struct Maps2 {
     CUtensorMap tok[2];  // token rows, box 128, 128-byte swizzle
     CUtensorMap tok16[2];  // token rows, box 16, 128-byte swizzle (weight-major halves)
+    CUtensorMap tok64[2];  // token rows, box 64, 128-byte swizzle (weight-major halves of >= 64 rows)
     CUtensorMap w[2];    // tiled weights as [rows, 64], box 128, no swizzle (tiles are pre-swizzled)
 };
 
@@ -301,6 +302,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
         for (int p = 0; p < a.nphase; ++p) {
             tma_prefetch_desc(&maps.tok[p]);
             tma_prefetch_desc(&maps.tok16[p]);
+            tma_prefetch_desc(&maps.tok64[p]);
             tma_prefetch_desc(&maps.w[p]);
         }
     if (warp == 1) {
@@ -433,12 +435,17 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 const int wg = weight_slot(a.w_slot, a.w_slots, t.g, a.status);
                 const int64_t wblk0 = static_cast<int64_t>(wg) * pa.nb + (t.n0 + 128 * static_cast<int>(rank)) / 128;
                 // weight-major: the MMA's N is the tile's tokens rounded up to 16;
-                // this CTA holds N / 2 of them (a multiple of 8), loaded in 16-row boxes
+                // this CTA holds N / 2 of them (a multiple of 8), loaded in 64-row
+                // boxes and the rest in 16-row boxes (fewer copies to issue; a
+                // box at a 1 KB boundary lays rows out as the 16-row boxes would)
                 const int half = t.swap ? ((t.rows + 15) / 16) * 8 : 0;
-                const int nb16 = (half + 15) / 16;
+                const int n64 = half / 64;
+                const int nb16 = (half - 64 * n64 + 15) / 16;
                 // each CTA loads exactly half of the pair's bytes
                 const uint32_t pair_bytes =
-                    t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(nb16) * 2048u) : 4u * kHalf;
+                    t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(n64) * 8192u +
+                                   static_cast<uint32_t>(nb16) * 2048u)
+                           : 4u * kHalf;
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!pwait(&empty[s], ph ^ 1u, a, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, peer_abort)) {
                         ok = false;
@@ -457,9 +464,12 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                             tma_load_pair(&maps.w[t.phase], stage + j * kHalf, bar, 0,
                                           static_cast<int32_t>(((wblk0 + 2 * j) * pa.k_blocks + kb) * 128), pol_first);
                         const int64_t trow = t.row0 + static_cast<int64_t>(rank) * half;
+                        for (int j = 0; j < n64; ++j)
+                            tma_load_pair(&maps.tok64[t.phase], stage + a.xoff + j * 8192, bar, kb * kBK,
+                                          static_cast<int32_t>(trow + 64 * j), pol_last);
                         for (int j = 0; j < nb16; ++j)
-                            tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + j * 2048, bar, kb * kBK,
-                                          static_cast<int32_t>(trow + 16 * j), pol_last);
+                            tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + n64 * 8192 + j * 2048, bar, kb * kBK,
+                                          static_cast<int32_t>(trow + 64 * n64 + 16 * j), pol_last);
                     }
                     use_bytes[s] = leader ? pair_bytes : pair_bytes / 2u;
                     ++uses;
@@ -627,14 +637,21 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     const int nwr = t.n0 + 256 * sub + 128 * static_cast<int>(rank);
                     tmem_ld32(taddr + static_cast<uint32_t>(128 * sub + c * 32), v);
                     if (pa.epi == EPI_SWIGLU_BF16) {
+                        // lane l < 16 holds gate row f0 + l and lane l + 16 the up
+                        // row of the same f, each for 32 tokens.  The half-warps
+                        // split the tokens: lane l finishes token j, lane l + 16
+                        // token j + 16, after one exchange per token pair, so each
+                        // lane computes 16 SiLUs and every store writes for both.
+                        const bool hi = lane >= 16;
                         const int f = nwr / 2 + q * 16 + (lane & 15);
-                        bf16* H = static_cast<bf16*>(pa.out);
+                        const int tok0 = c * 32 + (hi ? 16 : 0);
+                        bf16* H = static_cast<bf16*>(pa.out) + (t.row0 + tok0) * pa.ldo + f;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float u = __shfl_xor_sync(0xffffffffu, v[j], 16);
-                            const int tok = c * 32 + j;
-                            if (lane < 16 && tok < t.rows)
-                                H[(t.row0 + tok) * pa.ldo + f] = __float2bfloat16_rn(silu2(v[j]) * u);
+                        for (int j = 0; j < 16; ++j) {
+                            const float other = __shfl_xor_sync(0xffffffffu, hi ? v[j] : v[j + 16], 16);
+                            const float g = hi ? other : v[j];
+                            const float u = hi ? v[j + 16] : other;
+                            if (tok0 + j < t.rows) H[static_cast<int64_t>(j) * pa.ldo] = __float2bfloat16_rn(silu2(g) * u);
                         }
                     } else {
                         float* Y = static_cast<float*>(pa.out) + static_cast<int64_t>(t.split) * pa.split_stride;
@@ -766,6 +783,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
         if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
         if (!map2(&maps.tok16[p], g.tok, trows, g.Kdim, 16u, true)) return -3;
+        if (!map2(&maps.tok64[p], g.tok, trows, g.Kdim, 64u, true)) return -3;
         const uint64_t wmats = static_cast<uint64_t>(L.w_slot ? L.w_slots : L.G);
         const uint64_t wrows = wmats * ph.nb * ph.k_blocks * 128;
         if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
