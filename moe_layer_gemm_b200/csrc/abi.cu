@@ -85,21 +85,15 @@ struct Layout {
 // padding and the weight stream dominates.
 constexpr int kSwapMaxRows = 128;
 
-// Tile policy by the mean group (T K / E assignments per expert):
-//   1  decode-sized (mean <= 256 rows; skewed routing then also leaves many
-//      small groups): groups of <= 128 rows take weight-major tiles
-//   2  mid-sized (mean <= 2048 rows, e.g. a capacity-limited layer): every
-//      group takes weight-major CTA-pair tiles of up to 256 tokens, so a
-//      group's ragged tail is padded to 16 tokens instead of a 128- or
-//      256-row token tile (only when the CTA-pair kernel takes the shape;
-//      otherwise no weight-major tiles)
-//   0  large groups: token-major tiles
+// Weight-major tiles are enabled when groups of decode size are expected:
+// a mean group of at most 256 rows (skewed routing then also leaves many
+// small groups).  (Weight-major CTA-pair tiles of up to 256 tokens for
+// mid-sized groups were measured slower than single-CTA token-major tiles at
+// the Qwen-like shape, 0.573 vs 0.450 ms: the orientation's epilogue and
+// token loads cost more where the tiles are compute-bound.)
 int choose_swap(const moe_dims* d) {
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
-    if (d->d_model % 128 != 0 || (2 * d->d_ff) % 128 != 0) return 0;
-    if (avg <= 256) return 1;
-    if (avg <= 2048 && d->d_model % 256 == 0 && (2 * d->d_ff) % 256 == 0) return 2;
-    return 0;
+    return (avg <= 256 && d->d_model % 128 == 0 && (2 * d->d_ff) % 128 == 0) ? 1 : 0;
 }
 
 // Reduction split of the down projection when groups are decode-sized:
@@ -108,7 +102,7 @@ int choose_swap(const moe_dims* d) {
 // and there are tiles enough for the CTA-pair kernel to give each weight-
 // major tile two weight sub-tiles (half the token reads).
 int choose_nsplit(const moe_dims* d, int swap) {
-    if (swap != 1) return 1;
+    if (!swap) return 1;
     const int64_t avg = (d->T * d->K + d->E - 1) / d->E;
     if (avg > kSwapMaxRows) return 1;
     int ks = static_cast<int>((d->d_ff + d->d_model - 1) / d->d_model);
@@ -279,8 +273,7 @@ GemmLaunch ffn_launch(const moe_dims* d, const Layout& L, const bf16* xperm, con
     g.group_off = offsets;
     g.dense_rows = 0;
     g.max_group_rows = maxrows;
-    g.swap_max_rows = L.swap == 1 ? kSwapMaxRows : (L.swap == 2 ? (1 << 30) : 0);
-    g.swap_tokens_max = L.swap == 2 ? 256 : 128;
+    g.swap_max_rows = L.swap ? kSwapMaxRows : 0;
     g.small_groups = (d->T * d->K) < static_cast<int64_t>(d->E) * 128;
     g.nphase = 2;
     GemmPhase& p0 = g.ph[0];
@@ -317,9 +310,8 @@ GemmLaunch ffn_launch(const moe_dims* d, const Layout& L, const bf16* xperm, con
 }
 
 // CTA-pair tiles: token-major pairs are 256 token rows, worth it when groups
-// are large; weight-major pairs halve the token traffic of decode-sized
-// groups and, up to 256 tokens wide, cover mid-sized groups with tails
-// padded to 16 tokens.
+// are large (ragged 256-row tails of mid-sized groups cost more than they
+// save); weight-major pairs halve the token traffic of decode-sized groups.
 bool ffn_uses_pair(const moe_dims* d, const Layout& L, const GemmLaunch& g) {
     const bool large_groups = d->T * d->K >= static_cast<int64_t>(d->E) * 1024;
     return (large_groups || L.swap) && gemm_2sm_supported(g);
@@ -330,9 +322,8 @@ bool ffn_uses_pair(const moe_dims* d, const Layout& L, const GemmLaunch& g) {
 // entry point clears them with a memset).
 int do_ffn(const moe_dims* d, const Layout& L, const bf16* xperm, const int32_t* offsets, const bf16* W13p,
            const bf16* W2p, bf16* h, float* yout, int nsplit, void* ws, cudaStream_t st) {
-    GemmLaunch g = ffn_launch(d, L, xperm, offsets, W13p, W2p, h, yout, nsplit, ws);
+    const GemmLaunch g = ffn_launch(d, L, xperm, offsets, W13p, W2p, h, yout, nsplit, ws);
     if (ffn_uses_pair(d, L, g)) return map_launch(launch_grouped_gemm_2sm(g, st));
-    if (L.swap == 2) g.swap_max_rows = 0;  // wide weight-major tiles are a CTA-pair form
     return map_launch(launch_grouped_gemm(g, st));
 }
 
@@ -503,7 +494,6 @@ int moe_expert_ffn_slots(const moe_dims* dims, const moe_bf16* x_perm, const int
     if (ffn_uses_pair(dims, L, g)) {
         MOE_TRY(map_launch(launch_grouped_gemm_2sm(g, st)));
     } else {
-        if (L.swap == 2) g.swap_max_rows = 0;
         MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
     }
     if (L.nsplit > 1)

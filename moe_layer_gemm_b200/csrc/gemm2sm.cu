@@ -85,7 +85,7 @@ struct Args2 {
     int nphase;
     int dep;
     int swap_max_rows;  // groups with at most this many rows take weight-major pair tiles
-    int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 256; <= 128 with two sub-tiles)
+    int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 128)
     Phase2 ph[2];
     int stages;
     uint32_t stage_bytes;  // per stage and CTA
@@ -741,13 +741,9 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     if (L.w_slot && L.w_slots < 1) return -2;
     const int64_t mx = L.max_group_rows < 1 ? 1 : L.max_group_rows;
     a.swap_max_rows = L.swap_max_rows < 0 ? 0 : L.swap_max_rows;
-    // weight-major tiles take up to 128 tokens, or 256 when the launch asks
-    // for wide ones (then each tile has one 256-row weight sub-tile: both
-    // fill the 256 TMEM columns of an accumulator buffer)
-    const int bns_cap = L.swap_tokens_max == 256 ? 256 : 128;
     {
         const int64_t lim = mx < a.swap_max_rows ? mx : a.swap_max_rows;
-        a.BNs = static_cast<int>(lim >= bns_cap ? bns_cap : ((lim + 31) / 32) * 32);
+        a.BNs = static_cast<int>(lim >= 128 ? 128 : ((lim + 31) / 32) * 32);
         if (a.BNs < 32) a.BNs = 32;
     }
     const bool token_major_possible = mx > a.swap_max_rows;
@@ -778,7 +774,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         // last, to shorten the final tiles, measured slower at the Mixtral
         // decode shape: their extra token reads cost more than the shorter
         // tail saved.)
-        ph.wt = (weight_major_possible && a.BNs <= 128 && g.N % 512 == 0 &&
+        ph.wt = (weight_major_possible && g.N % 512 == 0 &&
                  static_cast<int64_t>(L.G) * (g.N / 512) * ph.ksplit >= 3LL * clusters) ? 2 : 1;
         const uint64_t trows = static_cast<uint64_t>(g.tok_rows);
         if (!map2(&maps.tok[p], g.tok, trows, g.Kdim, 128u, true)) return -3;
@@ -797,7 +793,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     a.xoff = static_cast<uint32_t>(wt_max) * kHalf;
     // decode-sized launches (weight-major tiles for groups of <= 128 rows):
     // prefetch up to 16 k-blocks of each first-round weight tile
-    a.prefetch_kb = (weight_major_possible && a.swap_max_rows <= 128 && a.BNs <= 128 && L.w_slot == nullptr)
+    a.prefetch_kb = (weight_major_possible && L.w_slot == nullptr)
                         ? (a.ph[0].k_blocks < 16 ? a.ph[0].k_blocks : 16) : 0;
     uint32_t stage_bytes = token_major_possible ? 2u * kHalf : 0u;
     if (weight_major_possible) {

@@ -73,7 +73,6 @@ struct GemmLaunch {
     int64_t dense_rows;
     int64_t max_group_rows;  // host-known upper bound on any group's rows
     int swap_max_rows;       // groups with at most this many rows use weight-major tiles
-    int swap_tokens_max = 128;  // CTA-pair kernel: tokens per weight-major tile, 128 or 256
     bool small_groups;       // mean group below 128 rows: keep token-major tiles narrow
     int bn_max;              // cap on token-major BN (0 = none)
     int nphase;              // 1, or 2: phase 1 of group g starts after phase 0 of g

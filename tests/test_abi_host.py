@@ -108,10 +108,8 @@ def test_ffn_kernel_choice_by_shape(lib):
     assert abi.moe_ffn_kernel(abi.Dims(256, 4096, 14336, 8, 2)) == "grouped_gemm_2sm_kernel"
     # prefill-sized groups: token-major CTA pairs
     assert abi.moe_ffn_kernel(abi.Dims(16384, 4096, 14336, 8, 2)) == "grouped_gemm_2sm_kernel"
-    # mid-sized groups (mean 546 rows) with 256-multiple widths: weight-major CTA pairs of up to 256 tokens
-    assert abi.moe_ffn_kernel(abi.Dims(8192, 2048, 1408, 60, 4, 1.0)) == "grouped_gemm_2sm_kernel"
-    # the same groups with widths that are not multiples of 256: single-CTA token-major tiles
-    assert abi.moe_ffn_kernel(abi.Dims(8192, 2048, 1392, 60, 4, 1.0)) == "grouped_gemm_kernel"
+    # mid-sized groups (mean 546 rows) keep single-CTA tiles
+    assert abi.moe_ffn_kernel(abi.Dims(8192, 2048, 1408, 60, 4, 1.0)) == "grouped_gemm_kernel"
     # widths that are not multiples of 256 cannot take 256-wide pair tiles
     assert abi.moe_ffn_kernel(abi.Dims(64, 128, 256, 8, 2)) == "grouped_gemm_kernel"
     bad = abi.Dims(0, 4096, 14336, 8, 2)

@@ -65,8 +65,8 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (2000, 256, 320, 4, 2, 0.0),      # large groups: token-major tiles, ragged m tail
     (1500, 384, 704, 12, 3, 1.5),     # skewed: empty groups possible
     (130, 128, 128, 1, 1, 0.0),       # single expert = dense FFN
-    (2100, 512, 256, 4, 2, 0.0),      # mean group 1050 rows, widths x256: wide weight-major CTA-pair tiles
-    (6200, 256, 384, 6, 1, 1.5),      # the same with skewed groups (the smallest may be tiny)
+    (2100, 512, 256, 4, 2, 0.0),      # mean group >= 1024 rows, widths x256: CTA-pair tiles, ragged tail
+    (6200, 256, 384, 6, 1, 1.5),      # CTA-pair tiles with skewed groups (the smallest may be tiny)
     (256, 256, 1024, 8, 2, 1.5),      # decode-like CTA pairs, 4-way split, one group > 128 rows (token-major)
     (256, 256, 1408, 8, 2, 0.0),      # decode-like CTA pairs, 6-way split of 22 k-blocks (4, 4, 4, 4, 4, 2)
     (256, 384, 1536, 8, 2, 1.5),      # single-CTA, 4-way split, one group > 128 rows (token-major)
@@ -75,16 +75,16 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (600, 256, 256, 16, 4, 1.2),      # CTA pairs, weight- and token-major groups in one launch
     (512, 256, 2560, 64, 4, 0.0),     # CTA pairs, gate/up tiles of two 256-row weight sub-tiles, 8-way split
     (1024, 1024, 1024, 256, 8, 1.1),  # CTA pairs, two weight sub-tiles in both phases, skewed small groups
-    (2000, 256, 256, 1, 1, 0.0),      # one expert (dense FFN) on wide weight-major CTA-pair tiles, ragged tail
+    (2000, 256, 256, 1, 1, 0.0),      # one expert (dense FFN) on CTA-pair token-major tiles, ragged tail
     (1, 256, 512, 8, 2, 0.0),         # a single token: two one-row groups on CTA-pair weight-major tiles
-    # mean group 257..2048 rows with widths x256: weight-major CTA-pair tiles of up to 256 tokens for every group
-    (3000, 256, 384, 12, 2, 0.5),     # ragged 256-token chunks, tails padded to 16 tokens
-    (4000, 512, 256, 8, 1, 1.2),      # skewed: groups from tens to ~1500 rows (several chunks)
-    (2048, 256, 256, 2, 1, 0.0),      # chunks of exactly 256 tokens
-    (700, 256, 768, 2, 1, 0.0),       # mean group 350 rows
-    # mean group above 2048 rows: token-major 256 x 256 CTA-pair tiles
+    # mid-sized groups: single-CTA token-major tiles with ragged 128-row tails
+    (3000, 256, 384, 12, 2, 0.5),
+    (4000, 512, 256, 8, 1, 1.2),      # skewed: groups from tens to ~1500 rows
+    (700, 256, 768, 2, 1, 0.0),
+    # CTA-pair token-major tiles: exact 256-row tiles, and skewed groups with one under a tile
+    (2048, 256, 256, 2, 1, 0.0),
     (5000, 256, 256, 2, 1, 0.0),
-    (9000, 256, 512, 4, 1, 1.0),      # skewed: the smallest group under one tile
+    (9000, 256, 512, 4, 1, 1.0),
 ])
 def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
     # weight scale shrinks with the width so |y| stays O(1), the scale the
