@@ -17,6 +17,8 @@ settled) and, on one GPU, a ``workloads`` entry for each other layer shape of
 the metric: Mixtral prefill (T = 16384, tensor-bound), the Qwen-like layer
 with capacity, and the DeepSeek-like layer whose steps update the bias in
 place and draw fresh tokens (step j takes the tokens of seed step j mod 10).
+A last entry runs the DeepSeek-shaped layer with its experts offloaded to
+host memory as INT4 and an LRU cache on the GPU (16-token decode steps).
 
 ``--impl reference`` times the CPU oracle (the plain fp64 implementation the
 tests check against) on the host cores on a bounded token sample per step;
@@ -441,6 +443,66 @@ def stage_dict(stage_ms):
 
 EXTRA_WORKLOADS = ("mixtral_prefill", "qwen_capacity", "deepseek_bias")
 
+# Expert offloading: the DeepSeek-shaped layer at a decode batch of 16 tokens
+# (about 65 distinct experts a step), 160 of its 256 experts cached on the GPU
+OFFLOAD_TOKENS = 16
+OFFLOAD_SLOTS = 160
+OFFLOAD_PREFETCH = 32
+
+
+def run_offload_entry(dev, steps: int, warmup: int, barrier, clock_index: int):
+    """The DeepSeek-shaped layer at a decode batch with its experts offloaded:
+    all 256 experts in page-locked host memory as group-wise INT4, a cache of
+    OFFLOAD_SLOTS experts on the GPU, OFFLOAD_PREFETCH predicted experts
+    loaded ahead after each step; every step draws fresh tokens."""
+    from moe_layer_gemm_b200 import abi
+    from moe_layer_gemm_b200.offload import OffloadedLayer, quantize_experts_to_host
+    wl = synth.get_workload("deepseek_bias")
+    T = OFFLOAD_TOKENS
+    dims = abi.Dims(T, wl.d_model, wl.d_ff, wl.E, wl.K)
+    Wr = synth.make_router(wl, device=dev)
+    W1, W3, W2 = synth.make_expert_weights(wl, device=dev)
+    q = quantize_experts_to_host(dims, W1, W3, W2)
+    del W1, W3, W2
+    torch.cuda.empty_cache()
+    layer = OffloadedLayer(dims, Wr, *q, n_slots=OFFLOAD_SLOTS, prefetch=OFFLOAD_PREFETCH)
+    xs = [synth.normal_bf16((T, wl.d_model), 7000 + j, synth.STREAM_X, wl.x_std, dev) for j in range(warmup + steps)]
+    y = torch.empty(T, wl.d_model, dtype=torch.float32, device=dev)
+    for j in range(warmup):
+        layer.forward(xs[j], y)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s = torch.cuda.current_stream()
+    clocks = ClockSampler(clock_index)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    start.record(s)
+    for j in range(steps):
+        layer.forward(xs[warmup + j], y)
+    end.record(s)
+    torch.cuda.synchronize()
+    wall = (time.perf_counter() - t0) * 1e3 / steps
+    clk = clocks.stop()
+    ms = start.elapsed_time(end) / steps
+    recs = layer.log[warmup:]
+    need = sum(len(r["needed"]) for r in recs)
+    hits = sum(len(r["hits"]) for r in recs)
+    phits = sum(len(r["prefetch_hits"]) for r in recs)
+    miss = sum(len(r["misses"]) for r in recs)
+    host_bytes = sum(r["unpacked_bytes"] for r in recs) / steps
+    return {"value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps, "warmup": warmup,
+            "config": {"T": T, "d_model": wl.d_model, "d_ff": wl.d_ff, "E": wl.E, "K": wl.K, "cache_slots": OFFLOAD_SLOTS,
+                       "prefetch": OFFLOAD_PREFETCH, "int4_bytes_per_expert": layer.bytes_per_expert,
+                       "bf16_bytes_per_expert": 3 * wl.d_model * wl.d_ff * 2, "fresh_tokens_per_step": True},
+            "cache": {"needed_per_step": need / steps, "hit_rate": (hits + phits) / max(need, 1),
+                      "resident_hit_rate": hits / max(need, 1), "prefetch_hit_rate": phits / max(need, 1),
+                      "misses_per_step": miss / steps},
+            "host_link": {"bytes_per_step": host_bytes, "GB_per_s": host_bytes / (ms * 1e-3) / 1e9},
+            "host_ms_per_step": wall, "clocks": clk}
+
+
 
 def run_ours(args):
     from moe_layer_gemm_b200 import abi
@@ -595,6 +657,9 @@ def run_ours(args):
                             "routing": rt, "clocks": rx["clocks"], "gpu_launches_per_step": lx.launches()}
             del lx
             torch.cuda.empty_cache()
+        extras["deepseek_offload"] = run_offload_entry(dev, max(1, min(K, 20)), max(3, min(args.warmup, 5)), barrier,
+                                                       local)
+        torch.cuda.empty_cache()
 
     if pg:
         torch.distributed.destroy_process_group()

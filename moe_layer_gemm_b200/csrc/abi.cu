@@ -77,8 +77,27 @@ struct Layout {
     size_t status, sched_ffn, sched_router, idx, w, logits, counts, kept, offsets, ndrop, prob_part, prob_mean, f,
         aux, block_hist, inv, src, xperm, h, yperm, wrt, total;
     int route_nb, perm_nb, nsplit, E_pad, swap;
+    int router_bn, router_split;  // logits GEMM: weight rows per tile, reduction split
     bool fused_router;
 };
+
+// The logits GEMM (tensor-core router, E > 32): tiles as wide as E allows
+// (up to 256 columns: narrow MMAs are slow), and a split of the reduction so
+// the 128-row x BN tiles cover the SMs; the top-K kernel sums the partial
+// slices in slice order.
+void router_tiling(const moe_dims* d, int E_pad, int* bn, int* split) {
+    int b = 32;
+    for (int c : {256, 128, 64, 32})
+        if (E_pad % c == 0) { b = c; break; }
+    const int64_t tiles = ((d->T + 127) / 128) * (E_pad / b);
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    const int kb = (d->d_model + 63) / 64;
+    int s = static_cast<int>(tiles >= sms ? 1 : sms / tiles);
+    if (s > 8) s = 8;
+    while (s > 1 && kb / s < 8) --s;  // at least 8 k-blocks per slice
+    *bn = b;
+    *split = s < 1 ? 1 : s;
+}
 
 // Groups of at most this many token rows put the weight rows on the MMA M
 // side (weight-major tiles): small groups then waste no tensor-core rows on
@@ -119,6 +138,8 @@ Layout layout_of(const moe_dims* d) {
     L.perm_nb = permute_blocks(T);
     L.fused_router = route_fused_supported(d->d_model, d->E) != 0;
     L.E_pad = static_cast<int>(((E + 31) / 32) * 32);
+    router_tiling(d, L.E_pad, &L.router_bn, &L.router_split);
+    if (L.fused_router) L.router_split = 1;
     L.swap = choose_swap(d);
     L.nsplit = choose_nsplit(d, L.swap);
     size_t o = 0;
@@ -132,7 +153,7 @@ Layout layout_of(const moe_dims* d) {
     L.sched_router = take(gemm_sched_bytes(1));
     L.idx = take(A * 4);
     L.w = take(A * 4);
-    L.logits = take(T * E * 4);
+    L.logits = take(static_cast<size_t>(L.router_split) * T * E * 4);  // partial slices of the logits GEMM
     L.counts = take(E * 4);
     L.kept = take(E * 4);
     L.offsets = take((E + 1) * 4);
@@ -196,7 +217,7 @@ ChunkLayout chunk_layout_of(const moe_dims* d, int64_t chunk) {
     W.sched_router = take(gemm_sched_bytes(1));
     W.idx = take(static_cast<size_t>(T * K) * 4);
     W.w = take(static_cast<size_t>(T * K) * 4);
-    W.logits = W.fused_router ? 0 : take(static_cast<size_t>(T * E) * 4);
+    W.logits = W.fused_router ? 0 : take(static_cast<size_t>(W.router_split) * T * E * 4);
     W.prob_part = take(static_cast<size_t>(W.route_nb) * (2 * E + 1) * 4);
     W.prob_mean = take(E * 4);
     W.wrt = W.fused_router ? 0 : take(static_cast<size_t>((W.E_pad + 127) / 128) * 128 * ((d->d_model + 63) / 64) * 64 * 2);
@@ -224,7 +245,7 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
         MOE_TRY(map_launch(launch_route_fused(x, Wr, bias, d->T, d->d_model, d->E, d->K, logits, idx, w, part,
                                               L.route_nb, st)));
     } else {
-        float* lg = logits ? logits : at<float>(ws, L.logits);
+        float* lg = at<float>(ws, L.logits);  // [router_split][T][E] partial logits
         bf16* wrt = at<bf16>(ws, L.wrt);
         MOE_TRY(map_launch(launch_transpose_router(Wr, d->d_model, d->E, L.E_pad, wrt, st)));
         GemmLaunch g{};
@@ -233,11 +254,7 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
         g.dense_rows = d->T;
         g.max_group_rows = d->T;
         g.swap_max_rows = 0;
-        // narrow tiles: more CTAs share the logits GEMM (N = E_pad is small);
-        // 32-wide when 64-wide tiles would leave over half the SMs idle
-        const int64_t row_tiles = (d->T + 127) / 128;
-        const int sms = num_sms() > 0 ? num_sms() : 148;
-        g.bn_max = row_tiles * (L.E_pad / 64) < sms / 2 ? 32 : 64;
+        g.bn_max = L.router_bn;
         g.nphase = 1;
         g.ph[0].tok = x;
         g.ph[0].tok_rows = d->T;
@@ -245,16 +262,17 @@ int do_route(const moe_dims* d, const Layout& L, const bf16* x, const bf16* Wr, 
         g.ph[0].N = L.E_pad;
         g.ph[0].N_store = d->E;
         g.ph[0].Kdim = d->d_model;
-        g.ph[0].ksplit = 1;
+        g.ph[0].ksplit = L.router_split;
         g.ph[0].epi = EPI_F32;
         g.ph[0].out = lg;
         g.ph[0].ldo = d->E;
-        g.ph[0].split_stride = 0;
+        g.ph[0].split_stride = d->T * d->E;
         g.status = at<int>(ws, L.status);
         g.sched = at<int>(ws, L.sched_router);
         if (cudaMemsetAsync(g.sched, 0, gemm_sched_bytes(1), st) != cudaSuccess) return MOE_ECUDA;
         MOE_TRY(map_launch(launch_grouped_gemm(g, st)));
-        MOE_TRY(map_launch(launch_topk_from_logits(lg, bias, d->T, d->E, d->K, idx, w, part, L.route_nb, st)));
+        MOE_TRY(map_launch(launch_topk_from_logits(lg, L.router_split, d->T * d->E, logits, bias, d->T, d->E, d->K,
+                                                   idx, w, part, L.route_nb, st)));
     }
     if (prob_mean && finalize)
         MOE_TRY(map_launch(launch_prob_finalize(part, L.route_nb, d->E, d->T, prob_mean, st)));
@@ -428,7 +446,7 @@ int moe_route_from_logits(const moe_dims* dims, const float* logits, const float
     const Layout L = layout_of(dims);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* part = prob_mean ? at<float>(ws, L.prob_part) : nullptr;
-    MOE_TRY(map_launch(launch_topk_from_logits(logits, bias, dims->T, dims->E, dims->K, topk_idx, topk_w, part,
+    MOE_TRY(map_launch(launch_topk_from_logits(logits, 1, 0, nullptr, bias, dims->T, dims->E, dims->K, topk_idx, topk_w, part,
                                                L.route_nb, st)));
     if (prob_mean) MOE_TRY(map_launch(launch_prob_finalize(part, L.route_nb, dims->E, dims->T, prob_mean, st)));
     return MOE_OK;

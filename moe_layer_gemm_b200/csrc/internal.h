@@ -113,8 +113,11 @@ int launch_route_fused(const bf16* x, const bf16* Wr, const float* bias, int64_t
                        cudaStream_t st);
 int route_fused_supported(int d, int E);
 int route_blocks(int64_t T);
-int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, int E, int K,
-                            int32_t* idx, float* w, float* prob_part, int nblocks, cudaStream_t st);
+// Top-K from the sum of nsplit partial logits slices [nsplit][T][E] (slice
+// order); logits_out (or nullptr) receives the sums.
+int launch_topk_from_logits(const float* logits, int nsplit, int64_t split_stride, float* logits_out,
+                            const float* bias, int64_t T, int E, int K, int32_t* idx, float* w, float* prob_part,
+                            int nblocks, cudaStream_t st);
 // WrT: the router weight as a K-major [E_pad, d] matrix in 128 x 64 swizzled tiles.
 int launch_transpose_router(const bf16* Wr, int d, int E, int E_pad, bf16* WrT, cudaStream_t st);
 int launch_prob_finalize(const float* prob_part, int nblocks, int E, int64_t T, float* prob_mean,

@@ -101,7 +101,12 @@ hist_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int K, int32_t* _
 }
 
 // One block of 1024 threads.  block_hist is rewritten in place with each
-// block's rank base.
+// block's rank base: per expert, an exclusive scan over the blocks.  Warp w
+// takes experts w, w + 32, .. (up to 8 at once); its lanes take 32 blocks at
+// a time, all loads issued before the warp scans, so a column of blocks costs
+// one round of memory latency per 32 blocks instead of one per block.
+constexpr int kScanExpertsPerWarp = kMaxE / 32;
+
 __global__ void __launch_bounds__(1024)
 scan_kernel(int32_t* __restrict__ block_hist, int nblocks, int E, int64_t C, int32_t* __restrict__ counts,
             int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
@@ -109,19 +114,44 @@ scan_kernel(int32_t* __restrict__ block_hist, int nblocks, int E, int64_t C, int
     for (int i = threadIdx.x; i < zero_count; i += blockDim.x) zero_out[i] = 0;  // next kernel's scheduler words
     __shared__ int32_t sk[kMaxE];
     __shared__ int32_t sdrop[kMaxE];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t run = 0;
-        for (int b = 0; b < nblocks; ++b) {
-            const int64_t i = static_cast<int64_t>(b) * E + e;
-            const int32_t c = block_hist[i];
-            block_hist[i] = run;
-            run += c;
+    {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+        int carry[kScanExpertsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kScanExpertsPerWarp; ++i) carry[i] = 0;
+        for (int b0 = 0; b0 < nblocks; b0 += 32) {
+            const int b = b0 + lane;
+            int v[kScanExpertsPerWarp];
+#pragma unroll
+            for (int i = 0; i < kScanExpertsPerWarp; ++i) {
+                const int e = warp + nw * i;
+                v[i] = (e < E && b < nblocks) ? block_hist[static_cast<int64_t>(b) * E + e] : 0;
+            }
+#pragma unroll
+            for (int i = 0; i < kScanExpertsPerWarp; ++i) {
+                const int e = warp + nw * i;
+                int incl = v[i];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += u;
+                }
+                if (e < E && b < nblocks) block_hist[static_cast<int64_t>(b) * E + e] = carry[i] + incl - v[i];
+                carry[i] += __shfl_sync(0xffffffffu, incl, 31);
+            }
         }
-        const int32_t kp = (C >= 0 && run > C) ? static_cast<int32_t>(C) : run;
-        counts[e] = run;
-        kept[e] = kp;
-        sk[e] = kp;
-        sdrop[e] = run - kp;
+        if (lane == 0)
+#pragma unroll
+            for (int i = 0; i < kScanExpertsPerWarp; ++i) {
+                const int e = warp + nw * i;
+                if (e >= E) continue;
+                const int32_t run = carry[i];
+                const int32_t kp = (C >= 0 && run > C) ? static_cast<int32_t>(C) : run;
+                counts[e] = run;
+                kept[e] = kp;
+                sk[e] = kp;
+                sdrop[e] = run - kp;
+            }
     }
     __syncthreads();
     if (threadIdx.x < 32) {  // warp-level exclusive scan over E <= 256 (8 per lane)

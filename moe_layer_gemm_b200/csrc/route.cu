@@ -401,9 +401,12 @@ route_split_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
     }
 }
 
+// The logits are the sum of nsplit partial slices (a split reduction of the
+// logits GEMM), added in slice order; with logits_out the sums are stored.
 template <int J>
 __global__ void __launch_bounds__(kRouteWarps * 32)
-topk_from_logits_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int64_t T, int E,
+topk_from_logits_kernel(const float* __restrict__ logits, int nsplit, int64_t split_stride,
+                        float* __restrict__ logits_out, const float* __restrict__ bias, int64_t T, int E,
                         int K, int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ prob_part) {
     pdl_trigger();
     pdl_wait();
@@ -420,7 +423,13 @@ topk_from_logits_kernel(const float* __restrict__ logits, const float* __restric
         for (int j = 0; j < J; ++j) {
             const int e = lane + 32 * j;
             valid[j] = e < E;
-            l[j] = valid[j] ? logits[t * E + e] : -FLT_MAX;
+            float v = -FLT_MAX;
+            if (valid[j]) {
+                v = logits[t * E + e];
+                for (int sp = 1; sp < nsplit; ++sp) v += logits[sp * split_stride + t * E + e];
+                if (logits_out != nullptr) logits_out[t * E + e] = v;
+            }
+            l[j] = v;
         }
         finish_token<J>(l, valid, bias, t, K, lane, idx, w, psum, tsum, zsum, want_prob);
     }
@@ -509,17 +518,23 @@ int launch_route_fused(const bf16* x, const bf16* Wr, const float* bias, int64_t
     return launch_fused_ev<4>(x, Wr, bias, T, d, E, K, logits, idx, w, prob_part, nblocks, st);
 }
 
-int launch_topk_from_logits(const float* logits, const float* bias, int64_t T, int E, int K, int32_t* idx,
-                            float* w, float* prob_part, int nblocks, cudaStream_t st) {
+int launch_topk_from_logits(const float* logits, int nsplit, int64_t split_stride, float* logits_out,
+                            const float* bias, int64_t T, int E, int K, int32_t* idx, float* w, float* prob_part,
+                            int nblocks, cudaStream_t st) {
     const int th = kRouteWarps * 32;
+    if (nsplit < 1) return -2;
     if (E <= 32)
-        (void)launch_pdl(topk_from_logits_kernel<1>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<1>, dim3(nblocks), dim3(th), 0, st, logits, nsplit, split_stride,
+                         logits_out, bias, T, E, K, idx, w, prob_part);
     else if (E <= 64)
-        (void)launch_pdl(topk_from_logits_kernel<2>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<2>, dim3(nblocks), dim3(th), 0, st, logits, nsplit, split_stride,
+                         logits_out, bias, T, E, K, idx, w, prob_part);
     else if (E <= 128)
-        (void)launch_pdl(topk_from_logits_kernel<4>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<4>, dim3(nblocks), dim3(th), 0, st, logits, nsplit, split_stride,
+                         logits_out, bias, T, E, K, idx, w, prob_part);
     else if (E <= 256)
-        (void)launch_pdl(topk_from_logits_kernel<8>, dim3(nblocks), dim3(th), 0, st, logits, bias, T, E, K, idx, w, prob_part);
+        (void)launch_pdl(topk_from_logits_kernel<8>, dim3(nblocks), dim3(th), 0, st, logits, nsplit, split_stride,
+                         logits_out, bias, T, E, K, idx, w, prob_part);
     else
         return -2;
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
