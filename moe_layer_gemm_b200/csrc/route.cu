@@ -423,14 +423,21 @@ topk_from_logits_kernel(const float* __restrict__ logits, int nsplit, int64_t sp
         for (int j = 0; j < J; ++j) {
             const int e = lane + 32 * j;
             valid[j] = e < E;
-            float v = -FLT_MAX;
-            if (valid[j]) {
-                v = logits[t * E + e];
-                for (int sp = 1; sp < nsplit; ++sp) v += logits[sp * split_stride + t * E + e];
-                if (logits_out != nullptr) logits_out[t * E + e] = v;
-            }
-            l[j] = v;
+            l[j] = valid[j] ? logits[t * E + e] : -FLT_MAX;
         }
+        // slice by slice, so the J loads of a slice are in flight together
+        for (int sp = 1; sp < nsplit; ++sp) {
+            const float* ls = logits + sp * split_stride + t * E;
+            float u[J];
+#pragma unroll
+            for (int j = 0; j < J; ++j) u[j] = valid[j] ? ls[lane + 32 * j] : 0.f;
+#pragma unroll
+            for (int j = 0; j < J; ++j) l[j] += u[j];
+        }
+        if (logits_out != nullptr)
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+                if (valid[j]) logits_out[t * E + lane + 32 * j] = l[j];
         finish_token<J>(l, valid, bias, t, K, lane, idx, w, psum, tsum, zsum, want_prob);
     }
     if (want_prob) write_prob_partials<J>(psum, tsum, zsum, E, prob_part);
