@@ -11,14 +11,21 @@
 // phase order, and a phase-1 tile of expert g waits (bounded) until every
 // phase-0 tile of g has stored its H rows, so the down projection of early
 // experts overlaps the gate/up projection of late ones and there is one
-// tail instead of two.  Roles per CTA (192 threads):
-//   warp 0        scheduler + producer (one elected thread): claims tiles,
-//                 broadcasts them through a shared-memory ring and fills a
-//                 multi-stage operand ring: token rows by TMA tile loads,
-//                 weight tiles by contiguous 16 KB bulk copies of the
-//                 pre-tiled, pre-swizzled packed weights
+// tail instead of two.  Roles per CTA (224 threads):
+//   warp 0        scheduler + producer 0 (one elected thread): claims tiles
+//                 and broadcasts them through a shared-memory ring
+//   warps 0, 6    producers (one elected thread each): fill a multi-stage
+//                 operand ring, alternating stage uses (producer k issues
+//                 the uses u with u % 2 == k, so it owns the stages of that
+//                 parity): token rows by TMA tile loads, weight tiles by
+//                 contiguous 16 KB bulk copies of the pre-tiled,
+//                 pre-swizzled packed weights
 //   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2..5    epilogue: TMEM -> registers -> SwiGLU / fp32 -> global
+// Two producers: the copies one thread issues after a barrier wait are
+// serviced one stage at a time (a measured property of the copy engine:
+// about 0.4 us per stage and issuing thread, whatever the ring depth), so a
+// second issuing thread doubles the stage rate.
 // The accumulator is double-buffered in TMEM (2 x 256 fp32 columns).
 //
 // Tile orientation is chosen per group:
@@ -42,7 +49,8 @@ namespace moe {
 namespace {
 
 constexpr int kBK = 64;                        // reduction elements per stage (one 128 B swizzle row)
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
+constexpr int kProducer1Warp = 6;
 constexpr uint32_t kTileABytes = 128u * 128u;  // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = 256;
@@ -223,7 +231,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         }
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&rfull[r], 1);
-            mbar_init(&rempty[r], 5);  // MMA thread + 4 epilogue warps
+            mbar_init(&rempty[r], 6);  // producer 1 + MMA thread + 4 epilogue warps
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -275,26 +283,38 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
     const uint32_t tmem_base = *tmem_slot;
     const int total = tstart[(a.nphase - 1) * (G + 1) + G];
 
-    if (warp == 0) {
+    if (warp == 0 || warp == kProducer1Warp) {
         if (lane == 0) {
-            // ------------------------------------------- scheduler + producer
+            // ------------------------------------- scheduler + producers
+            const uint32_t me = warp == 0 ? 0u : 1u;
             const uint64_t pol_first = policy_evict_first();
             const uint64_t pol_last = policy_evict_last();
-            uint32_t s = 0, ph = 0, r = 0, rph = 0;
+            uint32_t s = 0, ph = 0, r = 0, rph = 0, u = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool ok = true;
             // claims run one tile ahead so the atomic's round trip overlaps
             // the loads of the current tile
-            int next = atomicAdd(&a.sched[0], 1);
+            int next = me == 0 ? atomicAdd(&a.sched[0], 1) : 0;
             while (ok) {
-                const int tile = next < total ? next : -1;
-                if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
-                if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, a.wait_limit)) {
-                    ok = false;
-                    break;
+                int tile;
+                if (me == 0) {
+                    tile = next < total ? next : -1;
+                    if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
+                    if (!mbar_wait(&rempty[r], rph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag,
+                                   a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    ring[r] = tile;
+                    mbar_arrive(&rfull[r]);
+                } else {
+                    if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tile = ring[r];
+                    mbar_arrive(&rempty[r]);
                 }
-                ring[r] = tile;
-                mbar_arrive(&rfull[r]);
                 if (++r == kRing) { r = 0; rph ^= 1u; }
                 if (tile < 0) break;  // the end marker
                 const Tile t = decode_tile(a, tile, tstart, off);
@@ -323,44 +343,48 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 const int nb = t.swap ? (t.rows + 31) / 32 : 0;
                 const uint32_t wbytes = t.swap ? 16384u : static_cast<uint32_t>(pa.BN) * 128u;
                 const uint32_t xbytes = t.swap ? static_cast<uint32_t>(nb) * 4096u : kTileABytes;
-                for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, a.wait_limit)) {
+                for (int kb = t.kb0; kb < t.kb1; ++kb, ++u) {
+                    const uint32_t cs = s, cph = ph;  // this use's stage and phase
+                    if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
+                    if ((u & 1u) != me) continue;     // the other producer's use
+                    if (!mbar_wait(&empty[cs], cph ^ 1u, a.status, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag,
+                                   a.wait_limit)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], wbytes + xbytes);
-                    uint8_t* dW = sW + static_cast<size_t>(s) * a.wslot;
-                    uint8_t* dX = sX + static_cast<size_t>(s) * a.xslot;
+                    mbar_arrive_expect_tx(&full[cs], wbytes + xbytes);
+                    uint8_t* dW = sW + static_cast<size_t>(cs) * a.wslot;
+                    uint8_t* dX = sX + static_cast<size_t>(cs) * a.xslot;
                     const int kx = kb * kBK;
                     if (t.swap) {
                         // weights (M side): one contiguous 16 KB tile, streamed once
-                        bulk_load(dW, weight_rows(pa, wg, t.n0, kb), 16384u, &full[s], pol_first);
+                        bulk_load(dW, weight_rows(pa, wg, t.n0, kb), 16384u, &full[cs], pol_first);
                         for (int j = 0; j < nb; ++j)
-                            tma_load_2d(&maps.tokB[t.phase], dX + j * 4096, &full[s], kx,
+                            tma_load_2d(&maps.tokB[t.phase], dX + j * 4096, &full[cs], kx,
                                         static_cast<int32_t>(t.row0 + 32 * j), pol_last);
                     } else {
                         // tokens (M side): 128 rows, kept in L2 for the group's other
                         // weight tiles; weights: BN rows, marked first to leave L2
                         // once the group's row tiles (running together) have read them
-                        tma_load_2d(&maps.tokA[t.phase], dX, &full[s], kx, static_cast<int32_t>(t.row0), pol_last);
+                        tma_load_2d(&maps.tokA[t.phase], dX, &full[cs], kx, static_cast<int32_t>(t.row0), pol_last);
                         if (pa.BN >= 128) {
                             for (int j = 0; j < pa.BN / 128; ++j)
-                                bulk_load(dW + j * 16384, weight_rows(pa, wg, t.n0 + 128 * j, kb), 16384u, &full[s],
+                                bulk_load(dW + j * 16384, weight_rows(pa, wg, t.n0 + 128 * j, kb), 16384u, &full[cs],
                                           pol_first);
                         } else {
-                            bulk_load(dW, weight_rows(pa, wg, t.n0, kb), wbytes, &full[s], pol_first);
+                            bulk_load(dW, weight_rows(pa, wg, t.n0, kb), wbytes, &full[cs], pol_first);
                         }
                     }
-                    issued_mask |= 1u << s;
-                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-                    if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
+                    issued_mask |= 1u << cs;
+                    issued_ph = (issued_ph & ~(1u << cs)) | (cph << cs);
                 }
             }
             // Leaving without the end marker means a wait failed and raised the
             // abort flag, which every consumer's wait watches, so none needs it.
-            // Drain: every issued copy has landed before the CTA may exit.  A
-            // stage is armed and its copies issued together, so each armed
-            // stage's last phase completes once those copies land.
+            // Drain: every copy this producer issued has landed before the CTA
+            // may exit.  A stage is armed and its copies issued together, and
+            // only this producer uses its stages (the ring depth is even), so
+            // each of them completes its last armed phase once those land.
             for (int i = 0; i < S; ++i)
                 if (issued_mask & (1u << i)) mbar_drain(&full[i], (issued_ph >> i) & 1u, a.status, DEV_TIMEOUT_DRAIN, a.wait_limit);
         }
@@ -410,7 +434,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             umma_commit(drain);
             mbar_drain(drain, 0, a.status, DEV_TIMEOUT_DRAIN, a.wait_limit);
         }
-    } else {
+    } else if (warp != kProducer1Warp) {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         uint32_t r = 0, rph = 0;
@@ -638,6 +662,7 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
     const size_t budget = 227 * 1024 - fixed;
     int stages = static_cast<int>(budget / (wslot + xslot));
     if (stages > 16) stages = 16;
+    stages &= ~1;  // even: each of the two producers owns the stages of one parity
     if (stages < 2) return -2;
     a.stages = stages;
     const size_t smem = fixed + static_cast<size_t>(stages) * (wslot + xslot);
