@@ -23,9 +23,10 @@
 // MMAs into two TMEM accumulators, which halves the token traffic again.
 // The down projection's reduction can be split as in gemm.cu.
 //
-// Stage layout (per CTA): token-major tiles put their 128 token rows at 0
-// and their 128 weight rows at 16 KB; weight-major tiles put weight
-// sub-tile j at 16 KB j and their token rows at xoff.
+// Stage layout (per CTA and k-block): token-major tiles put their 128 token
+// rows at 0 and their 128 weight rows at 16 KB; weight-major tiles put
+// weight sub-tile j at 16 KB j and their token rows at xoff.  A stage holds
+// one or two such k-blocks (kpb) that complete on one barrier phase.
 //
 // Pair protocol (barriers live in each CTA; "leader" means rank 0's copy):
 //   full[s]    leader only: the leader registers the pair's bytes, both CTAs'
@@ -88,7 +89,8 @@ struct Args2 {
     int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 128)
     Phase2 ph[2];
     int stages;
-    uint32_t stage_bytes;  // per stage and CTA
+    uint32_t stage_bytes;  // per k-block and CTA
+    int kpb;               // k-blocks per stage (1 or 2)
     uint32_t xoff;         // weight-major tiles: offset of the token rows in a stage
     int* status;
     int* sched;
@@ -259,7 +261,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int S = a.stages;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * a.stage_bytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * a.kpb * a.stage_bytes);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
@@ -446,32 +448,36 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(n64) * 8192u +
                                    static_cast<uint32_t>(nb16) * 2048u)
                            : 4u * kHalf;
-                for (int kb = t.kb0; kb < t.kb1; ++kb) {
+                for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += a.kpb) {
+                    const int nk = min(a.kpb, t.kb1 - kb0);
                     if (!pwait(&empty[s], ph ^ 1u, a, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, peer_abort)) {
                         ok = false;
                         break;
                     }
-                    if (leader) mbar_arrive_expect_tx(&full[s], pair_bytes);
+                    if (leader) mbar_arrive_expect_tx(&full[s], pair_bytes * static_cast<uint32_t>(nk));
                     const uint32_t bar = leader_full0 + 8u * s;
-                    uint8_t* stage = smem + static_cast<size_t>(s) * a.stage_bytes;
-                    if (!t.swap) {
-                        tma_load_pair(&maps.tok[t.phase], stage, bar, kb * kBK,
-                                      static_cast<int32_t>(t.row0 + 128 * rank), pol_last);
-                        tma_load_pair(&maps.w[t.phase], stage + kHalf, bar, 0,
-                                      static_cast<int32_t>((wblk0 * pa.k_blocks + kb) * 128), pol_first);
-                    } else {
-                        for (int j = 0; j < t.wt; ++j)
-                            tma_load_pair(&maps.w[t.phase], stage + j * kHalf, bar, 0,
-                                          static_cast<int32_t>(((wblk0 + 2 * j) * pa.k_blocks + kb) * 128), pol_first);
-                        const int64_t trow = t.row0 + static_cast<int64_t>(rank) * half;
-                        for (int j = 0; j < n64; ++j)
-                            tma_load_pair(&maps.tok64[t.phase], stage + a.xoff + j * 8192, bar, kb * kBK,
-                                          static_cast<int32_t>(trow + 64 * j), pol_last);
-                        for (int j = 0; j < nb16; ++j)
-                            tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + n64 * 8192 + j * 2048, bar, kb * kBK,
-                                          static_cast<int32_t>(trow + 64 * n64 + 16 * j), pol_last);
+                    for (int h = 0; h < nk; ++h) {
+                        const int kb = kb0 + h;
+                        uint8_t* stage = smem + (static_cast<size_t>(s) * a.kpb + h) * a.stage_bytes;
+                        if (!t.swap) {
+                            tma_load_pair(&maps.tok[t.phase], stage, bar, kb * kBK,
+                                          static_cast<int32_t>(t.row0 + 128 * rank), pol_last);
+                            tma_load_pair(&maps.w[t.phase], stage + kHalf, bar, 0,
+                                          static_cast<int32_t>((wblk0 * pa.k_blocks + kb) * 128), pol_first);
+                        } else {
+                            for (int j = 0; j < t.wt; ++j)
+                                tma_load_pair(&maps.w[t.phase], stage + j * kHalf, bar, 0,
+                                              static_cast<int32_t>(((wblk0 + 2 * j) * pa.k_blocks + kb) * 128), pol_first);
+                            const int64_t trow = t.row0 + static_cast<int64_t>(rank) * half;
+                            for (int j = 0; j < n64; ++j)
+                                tma_load_pair(&maps.tok64[t.phase], stage + a.xoff + j * 8192, bar, kb * kBK,
+                                              static_cast<int32_t>(trow + 64 * j), pol_last);
+                            for (int j = 0; j < nb16; ++j)
+                                tma_load_pair(&maps.tok16[t.phase], stage + a.xoff + n64 * 8192 + j * 2048, bar, kb * kBK,
+                                              static_cast<int32_t>(trow + 64 * n64 + 16 * j), pol_last);
+                        }
                     }
-                    use_bytes[s] = leader ? pair_bytes : pair_bytes / 2u;
+                    use_bytes[s] = (leader ? pair_bytes : pair_bytes / 2u) * static_cast<uint32_t>(nk);
                     ++uses;
                     if (++s == static_cast<uint32_t>(S)) { s = 0; ph ^= 1u; }
                 }
@@ -551,26 +557,30 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
                 const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 15) / 16) * 16u : 256u;
                 const uint32_t idesc = umma_idesc_bf16(256, n_mma);
-                for (int kb = t.kb0; kb < t.kb1; ++kb) {
+                for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += a.kpb) {
+                    const int nk = min(a.kpb, t.kb1 - kb0);
                     if (!pwait(&full[s], ph, a, DEV_TIMEOUT_MMA_FULL, abort_flag, peer_abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t stage = smem_u32(smem + static_cast<size_t>(s) * a.stage_bytes);
-                    if (!t.swap) {
-#pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk)
-                            umma_pair(d_tmem, umma_desc_sw128(stage + kk * 32), umma_desc_sw128(stage + kHalf + kk * 32),
-                                      idesc, (kb > t.kb0 || kk > 0) ? 1u : 0u);
-                    } else {
-                        // sub-tile j accumulates into columns 128 j .. of the buffer
-                        for (int j = 0; j < t.wt; ++j) {
+                    for (int h = 0; h < nk; ++h) {
+                        const int kb = kb0 + h;
+                        const uint32_t stage = smem_u32(smem + (static_cast<size_t>(s) * a.kpb + h) * a.stage_bytes);
+                        if (!t.swap) {
 #pragma unroll
                             for (int kk = 0; kk < kBK / 16; ++kk)
-                                umma_pair(d_tmem + 128u * j, umma_desc_sw128(stage + j * kHalf + kk * 32),
-                                          umma_desc_sw128(stage + a.xoff + kk * 32), idesc,
-                                          (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                                umma_pair(d_tmem, umma_desc_sw128(stage + kk * 32), umma_desc_sw128(stage + kHalf + kk * 32),
+                                          idesc, (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                        } else {
+                            // sub-tile j accumulates into columns 128 j .. of the buffer
+                            for (int j = 0; j < t.wt; ++j) {
+#pragma unroll
+                                for (int kk = 0; kk < kBK / 16; ++kk)
+                                    umma_pair(d_tmem + 128u * j, umma_desc_sw128(stage + j * kHalf + kk * 32),
+                                              umma_desc_sw128(stage + a.xoff + kk * 32), idesc,
+                                              (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                            }
                         }
                     }
                     umma_commit_pair(&empty[s]);
@@ -801,11 +811,18 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         stage_bytes = wm > stage_bytes ? wm : stage_bytes;
     }
     a.stage_bytes = stage_bytes;
-    int stages = static_cast<int>((227 * 1024 - fixed) / stage_bytes);
+    // Two k-blocks per stage where three such stages fit (token-major-only
+    // launches): a producer thread's copies issued after a barrier wait are
+    // serviced about one stage at a time, so fewer, larger stages move more
+    // bytes per stage cycle (prefill-sized layer: expert GEMMs 3-6 % faster).
+    // Launches with weight-major tiles keep one k-block per stage and a
+    // deeper ring (two k-blocks there measured slower).
+    a.kpb = (227 * 1024 - fixed) / (2 * static_cast<size_t>(stage_bytes)) >= 3 ? 2 : 1;
+    int stages = static_cast<int>((227 * 1024 - fixed) / (a.kpb * static_cast<size_t>(stage_bytes)));
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return -2;
     a.stages = stages;
-    const size_t smem = fixed + static_cast<size_t>(stages) * stage_bytes;
+    const size_t smem = fixed + static_cast<size_t>(stages) * a.kpb * stage_bytes;
     static std::atomic<unsigned long long> attr_done{0};
     if (smem_attr_once(reinterpret_cast<const void*>(grouped_gemm_2sm_kernel), 227 * 1024, attr_done) != 0) return -3;
     cudaLaunchConfig_t cfg{};
