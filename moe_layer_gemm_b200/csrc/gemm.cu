@@ -587,7 +587,9 @@ int num_sms() {
     return n;
 }
 
-size_t gemm_sched_bytes(int G) { return static_cast<size_t>(G + 1) * sizeof(int); }
+// Scheduler words: a tile counter, one readiness counter per group, and the
+// CTA-pair kernel's second (weight-major) tile counter.
+size_t gemm_sched_bytes(int G) { return static_cast<size_t>(G + 2) * sizeof(int); }
 
 // Returns 0 on success, -2 for an unsupported shape, -3 for a CUDA failure.
 // L.sched must point at gemm_sched_bytes(G) bytes that are zero when the

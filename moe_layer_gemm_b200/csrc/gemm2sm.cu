@@ -23,6 +23,18 @@
 // MMAs into two TMEM accumulators, which halves the token traffic again.
 // The down projection's reduction can be split as in gemm.cu.
 //
+// Two tile queues.  Token-major tiles (large groups) and weight-major tiles
+// (small groups) are numbered in separate queues, each phase 0 then phase 1
+// in group order, with a tile counter each.  At kernel start every CTA
+// computes both queues' tiles and the same split of the pairs between them
+// (split_pairs: in proportion to the queues' work); a pair serves one queue
+// with a ring shaped for it: token-major pairs put two k-blocks in each of
+// three stages, weight-major pairs one k-block in each of five or more.  So
+// the tensor-bound and the stream-bound tiles of a mixed launch run side by
+// side, each kind with its better ring (DeepSeek-shaped layer: expert GEMMs
+// 5.13-5.17 -> 4.90-4.94 ms on one box).  A launch with one kind of tile
+// puts every pair on its queue.
+//
 // Stage layout (per CTA and k-block): token-major tiles put their 128 token
 // rows at 0 and their 128 weight rows at 16 KB; weight-major tiles put
 // weight sub-tile j at 16 KB j and their token rows at xoff.  A stage holds
@@ -88,12 +100,14 @@ struct Args2 {
     int swap_max_rows;  // groups with at most this many rows take weight-major pair tiles
     int BNs;            // weight-major: tokens per pair tile (multiple of 32, <= 128)
     Phase2 ph[2];
-    int stages;
-    uint32_t stage_bytes;  // per k-block and CTA
-    int kpb;               // k-blocks per stage (1 or 2)
-    uint32_t xoff;         // weight-major tiles: offset of the token rows in a stage
+    // Ring of a pair serving the token-major queue [0] or the weight-major queue [1]
+    int stages[2];
+    uint32_t stage_bytes[2];  // per k-block and CTA
+    int kpb[2];               // k-blocks per stage (1 or 2)
+    size_t ring_bytes;        // shared memory of the larger ring
+    uint32_t xoff;            // weight-major tiles: offset of the token rows in a k-block
     int* status;
-    int* sched;
+    int* sched;  // [0] token-major tile counter, [1 + g] phase-0 stores of group g, [G + 1] weight-major tile counter
     uint32_t wait_limit;      // polls of a bounded mbarrier or drain wait
     uint32_t dep_wait_limit;  // polls of the phase-1 readiness wait
     int dep_extra;            // added to the phase-1 readiness target (0; a test makes it unreachable)
@@ -202,6 +216,39 @@ __device__ __forceinline__ int tiles_of2(const Args2& a, int p, int64_t rows) {
     return static_cast<int>(((rows + a.BNs - 1) / a.BNs) * (ph.N / (256 * ph.wt)) * ph.ksplit);
 }
 
+// Tiles of a group of `rows` rows in queue q (0: token-major, 1: weight-major).
+__device__ __forceinline__ int tiles_in_queue(const Args2& a, int q, int p, int64_t rows) {
+    return (swaps2(a, rows) ? 1 : 0) == q ? tiles_of2(a, p, rows) : 0;
+}
+
+// Cost of a token-major k-block relative to a weight-major k-block of one
+// 256-row weight sub-tile when the two kinds run side by side on separate
+// pairs (DeepSeek-shaped layer, clock-counter instrumentation: 813 against
+// 600 cycles; the token-major loads then wait behind the weight stream).
+constexpr float kTokenMajorCost = 1.35f;
+
+// Pairs serving the token-major queue.  Token-major tiles are bound by the
+// tensor pipe, weight-major tiles by the weight stream, and the two kinds run
+// side by side on separate pairs, each with its own ring (token-major pairs
+// use two k-blocks per stage).  The pairs are split in proportion to the
+// queues' work: k-blocks per 256-row weight (sub-)tile, token-major ones
+// weighted by kTokenMajorCost.  An empty queue gets no pair.
+__device__ __forceinline__ int split_pairs(const Args2& a, const int* tstart_all, int npairs) {
+    const int G = a.G;
+    float w[2] = {0.f, 0.f};
+    for (int q = 0; q < 2; ++q)
+        for (int p = 0; p < a.nphase; ++p) {
+            const int* ts = tstart_all + (2 * q + p) * (G + 1);
+            const float tiles = static_cast<float>(ts[G] - ts[0]);
+            w[q] += tiles * static_cast<float>(a.ph[p].kb_per_split) * static_cast<float>(q == 1 ? a.ph[p].wt : 1);
+        }
+    w[0] *= kTokenMajorCost;
+    if (w[0] <= 0.f) return 0;
+    if (w[1] <= 0.f || npairs < 2) return npairs;
+    int x = __float2int_rn(static_cast<float>(npairs) * w[0] / (w[0] + w[1]));
+    return x < 1 ? 1 : (x > npairs - 1 ? npairs - 1 : x);
+}
+
 __device__ __forceinline__ Tile2 decode2(const Args2& a, int tile, const int* tstart, const int64_t* off) {
     Tile2 t;
     const int G = a.G;
@@ -260,10 +307,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    const int S = a.stages;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * a.kpb * a.stage_bytes);
-    uint64_t* empty = full + S;
-    uint64_t* tfull = empty + S;
+    const int Smax = a.stages[0] > a.stages[1] ? a.stages[0] : a.stages[1];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.ring_bytes);
+    uint64_t* empty = full + Smax;
+    uint64_t* tfull = empty + Smax;
     uint64_t* tempty = tfull + 2;
     uint64_t* rfull = tempty + 2;
     uint64_t* rempty = rfull + kRing;
@@ -272,8 +319,9 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + kRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int64_t* off = reinterpret_cast<int64_t*>(tmem_slot + 2);
-    int* tstart = reinterpret_cast<int*>(off + a.G + 1);
-    PeerReport* report = reinterpret_cast<PeerReport*>(tstart + 2 * (a.G + 1));
+    int* tstart_all = reinterpret_cast<int*>(off + a.G + 1);  // [queue][phase][G + 1]
+    int* role_split = tstart_all + 4 * (a.G + 1);            // pairs serving the token-major queue
+    PeerReport* report = reinterpret_cast<PeerReport*>(role_split + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -282,7 +330,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < Smax; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -342,35 +390,49 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
     __syncthreads();
     if (warp == 0) {
+        // Tile numbering per queue (0: token-major groups, 1: weight-major
+        // groups), phase 0 then phase 1, groups in order; each lane scans a
+        // contiguous span of groups.
         const int span = (G + 31) / 32;
         const int g0 = min(G, lane * span), g1 = min(G, g0 + span);
-        int carry = 0;
-        for (int p = 0; p < a.nphase; ++p) {
-            int sum = 0;
-            for (int g = g0; g < g1; ++g) sum += tiles_of2(a, p, off[g + 1] - off[g]);
-            int incl = sum;
+        for (int q = 0; q < 2; ++q) {
+            int carry = 0;
+            for (int p = 0; p < a.nphase; ++p) {
+                int sum = 0;
+                for (int g = g0; g < g1; ++g) sum += tiles_in_queue(a, q, p, off[g + 1] - off[g]);
+                int incl = sum;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                int run = carry + incl - sum;
+                int* ts = tstart_all + (2 * q + p) * (G + 1);
+                for (int g = g0; g < g1; ++g) {
+                    ts[g] = run;
+                    run += tiles_in_queue(a, q, p, off[g + 1] - off[g]);
+                }
+                const int tot = __shfl_sync(0xffffffffu, incl, 31);
+                if (lane == 0) ts[G] = carry + tot;
+                carry += tot;
             }
-            int run = carry + incl - sum;
-            int* ts = tstart + p * (G + 1);
-            for (int g = g0; g < g1; ++g) {
-                ts[g] = run;
-                run += tiles_of2(a, p, off[g + 1] - off[g]);
-            }
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            if (lane == 0) ts[G] = carry + tot;
-            carry += tot;
         }
+        __syncwarp();
+        if (lane == 0) *role_split = split_pairs(a, tstart_all, static_cast<int>(gridDim.x >> 1));
     }
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // this pair's queue and ring (both CTAs of a pair compute the same)
+    const int queue = static_cast<int>(blockIdx.x >> 1) < *role_split ? 0 : 1;
+    const int S = a.stages[queue];
+    const int kpb = a.kpb[queue];
+    const uint32_t sbytes = a.stage_bytes[queue];
+    const int* tstart = tstart_all + 2 * queue * (G + 1);
     const int total = tstart[(a.nphase - 1) * (G + 1) + G];
+    int* const counter = a.sched + (queue == 0 ? 0 : G + 1);
     const uint32_t leader_rempty0 = mapa_shared(smem_u32(rempty), 0);
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(tempty), 0);
     const uint32_t leader_full0 = mapa_shared(smem_u32(full), 0);
@@ -385,14 +447,14 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             bool ok = true;
             uint32_t uses = 0;                 // stage uses this CTA issued (armed, on the leader)
             uint32_t use_bytes[kMaxStages];    // bytes of the pair's (leader) or own (peer) last use per stage
-            int next = leader ? atomicAdd(&a.sched[0], 1) : 0;
+            int next = leader ? atomicAdd(counter, 1) : 0;
             const uint32_t peer_ring = mapa_shared(smem_u32(ring), 1);
             const uint32_t peer_rfull = mapa_shared(smem_u32(rfull), 1);
             while (ok) {
                 int tile;
                 if (leader) {
                     tile = next < total ? next : -1;
-                    if (tile >= 0) next = atomicAdd(&a.sched[0], 1);
+                    if (tile >= 0) next = atomicAdd(counter, 1);
                     if (!pwait(&rempty[r], rph ^ 1u, a, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, peer_abort)) {
                         ok = false;
                         break;
@@ -448,8 +510,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     t.swap ? 2u * (static_cast<uint32_t>(t.wt) * kHalf + static_cast<uint32_t>(n64) * 8192u +
                                    static_cast<uint32_t>(nb16) * 2048u)
                            : 4u * kHalf;
-                for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += a.kpb) {
-                    const int nk = min(a.kpb, t.kb1 - kb0);
+                for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += kpb) {
+                    const int nk = min(kpb, t.kb1 - kb0);
                     if (!pwait(&empty[s], ph ^ 1u, a, DEV_TIMEOUT_PRODUCER_EMPTY, abort_flag, peer_abort)) {
                         ok = false;
                         break;
@@ -458,7 +520,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     const uint32_t bar = leader_full0 + 8u * s;
                     for (int h = 0; h < nk; ++h) {
                         const int kb = kb0 + h;
-                        uint8_t* stage = smem + (static_cast<size_t>(s) * a.kpb + h) * a.stage_bytes;
+                        uint8_t* stage = smem + (static_cast<size_t>(s) * kpb + h) * sbytes;
                         if (!t.swap) {
                             tma_load_pair(&maps.tok[t.phase], stage, bar, kb * kBK,
                                           static_cast<int32_t>(t.row0 + 128 * rank), pol_last);
@@ -557,8 +619,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * 256u;
                 const uint32_t n_mma = t.swap ? static_cast<uint32_t>((t.rows + 15) / 16) * 16u : 256u;
                 const uint32_t idesc = umma_idesc_bf16(256, n_mma);
-                for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += a.kpb) {
-                    const int nk = min(a.kpb, t.kb1 - kb0);
+                for (int kb0 = t.kb0; kb0 < t.kb1; kb0 += kpb) {
+                    const int nk = min(kpb, t.kb1 - kb0);
                     if (!pwait(&full[s], ph, a, DEV_TIMEOUT_MMA_FULL, abort_flag, peer_abort)) {
                         ok = false;
                         break;
@@ -566,7 +628,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     tc_fence_after();
                     for (int h = 0; h < nk; ++h) {
                         const int kb = kb0 + h;
-                        const uint32_t stage = smem_u32(smem + (static_cast<size_t>(s) * a.kpb + h) * a.stage_bytes);
+                        const uint32_t stage = smem_u32(smem + (static_cast<size_t>(s) * kpb + h) * sbytes);
                         if (!t.swap) {
 #pragma unroll
                             for (int kk = 0; kk < kBK / 16; ++kk)
@@ -756,11 +818,11 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         a.BNs = static_cast<int>(lim >= 128 ? 128 : ((lim + 31) / 32) * 32);
         if (a.BNs < 32) a.BNs = 32;
     }
-    const bool token_major_possible = mx > a.swap_max_rows;
     const bool weight_major_possible = a.swap_max_rows > 0;
     const int sms = num_sms();
     if (sms <= 1) return -3;
     const int clusters = sms / 2;
+    if (clusters < 2) return -2;  // the two tile queues need a pair each
     Maps2 maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int p = 0; p < L.nphase; ++p) {
@@ -795,7 +857,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
     }
     const size_t fixed = 1024 + static_cast<size_t>(2 * kMaxStages + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
-                         static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + sizeof(PeerReport) + 64;
+                         static_cast<size_t>(L.G + 1) * (8 + 4 * 4) + 4 + sizeof(PeerReport) + 64;
     // stage: token-major tiles need 2 x 16 KB; weight-major tiles wt x 16 KB
     // of weights and BNs / 2 token rows
     int wt_max = 1;
@@ -805,24 +867,29 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     // prefetch up to 16 k-blocks of each first-round weight tile
     a.prefetch_kb = (weight_major_possible && L.w_slot == nullptr)
                         ? (a.ph[0].k_blocks < 16 ? a.ph[0].k_blocks : 16) : 0;
-    uint32_t stage_bytes = token_major_possible ? 2u * kHalf : 0u;
-    if (weight_major_possible) {
-        const uint32_t wm = a.xoff + static_cast<uint32_t>(a.BNs) * 64u;
-        stage_bytes = wm > stage_bytes ? wm : stage_bytes;
+    // Rings.  Token-major pairs: 32 KB per k-block and CTA, two k-blocks per
+    // stage where three such stages fit (a producer thread's copies issued
+    // after a barrier wait are serviced about one stage at a time, so fewer,
+    // larger stages move more bytes per stage cycle: prefill-sized layer,
+    // expert GEMMs 3-6 % faster).  Weight-major pairs: wt weight sub-tiles and
+    // BNs / 2 token rows per k-block, one k-block per stage and a deeper ring
+    // (two k-blocks there measured slower).  Both rings are always set up;
+    // the kernel splits the pairs between the queues at run time.
+    const size_t avail = 227 * 1024 - fixed;
+    a.stage_bytes[0] = 2u * kHalf;
+    a.stage_bytes[1] = a.xoff + static_cast<uint32_t>(a.BNs) * 64u;
+    size_t ring = 0;
+    for (int q = 0; q < 2; ++q) {
+        a.kpb[q] = (q == 0 && avail / (2 * static_cast<size_t>(a.stage_bytes[0])) >= 3) ? 2 : 1;
+        int stages = static_cast<int>(avail / (a.kpb[q] * static_cast<size_t>(a.stage_bytes[q])));
+        if (stages > kMaxStages) stages = kMaxStages;
+        if (stages < 2) return -2;
+        a.stages[q] = stages;
+        const size_t bytes = static_cast<size_t>(stages) * a.kpb[q] * a.stage_bytes[q];
+        ring = bytes > ring ? bytes : ring;
     }
-    a.stage_bytes = stage_bytes;
-    // Two k-blocks per stage where three such stages fit (token-major-only
-    // launches): a producer thread's copies issued after a barrier wait are
-    // serviced about one stage at a time, so fewer, larger stages move more
-    // bytes per stage cycle (prefill-sized layer: expert GEMMs 3-6 % faster).
-    // Launches with weight-major tiles keep one k-block per stage and a
-    // deeper ring (two k-blocks there measured slower).
-    a.kpb = (227 * 1024 - fixed) / (2 * static_cast<size_t>(stage_bytes)) >= 3 ? 2 : 1;
-    int stages = static_cast<int>((227 * 1024 - fixed) / (a.kpb * static_cast<size_t>(stage_bytes)));
-    if (stages > kMaxStages) stages = kMaxStages;
-    if (stages < 2) return -2;
-    a.stages = stages;
-    const size_t smem = fixed + static_cast<size_t>(stages) * a.kpb * stage_bytes;
+    a.ring_bytes = ring;
+    const size_t smem = fixed + ring;
     static std::atomic<unsigned long long> attr_done{0};
     if (smem_attr_once(reinterpret_cast<const void*>(grouped_gemm_2sm_kernel), 227 * 1024, attr_done) != 0) return -3;
     cudaLaunchConfig_t cfg{};
