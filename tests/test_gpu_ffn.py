@@ -72,6 +72,7 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (256, 384, 1536, 8, 2, 1.5),      # single-CTA, 4-way split, one group > 128 rows (token-major)
     (256, 128, 1024, 8, 2, 0.0),      # single-CTA, 8-way split
     (512, 512, 512, 16, 4, 1.5),      # CTA pairs, both tile queues: skewed groups above and below 128 rows
+    (256, 512, 1664, 8, 2, 1.5),      # CTA pairs, both queues, down split of 26 k-blocks as 7,7,7,5 (odd two-k-block tails)
     (40, 256, 1024, 8, 2, 0.0),       # CTA pairs, groups under 16 rows, 4-way split
     (600, 256, 256, 16, 4, 1.2),      # CTA pairs, weight- and token-major groups in one launch
     (512, 256, 2560, 64, 4, 0.0),     # CTA pairs, gate/up tiles of two 256-row weight sub-tiles, 8-way split
