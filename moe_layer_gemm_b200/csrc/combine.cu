@@ -187,6 +187,68 @@ combine_kernel(const float* __restrict__ yp, int nsplit, int64_t split_stride, c
     }
 }
 
+// One reduction slice (no split): a warp per token, no block barriers.  Lane
+// k < K reads the slot's row and weight, shuffled to all lanes; each lane
+// then sums columns lane, lane + 32, ... of the K rows, two 16-byte columns
+// at a time with all their loads issued together, slots in slot order, as
+// combine_kernel does (the same fp32 operations in the same order, so the
+// output is bit-identical).  With a statistics tail the last CTA does only that.
+template <typename OutT>
+__global__ void __launch_bounds__(256, 4)
+combine_warp_kernel(const float* __restrict__ yp, const int32_t* __restrict__ inv, const float* __restrict__ w,
+                    int64_t T, int d, int K, OutT* __restrict__ y, const StatsTail tail) {
+    pdl_trigger();
+    pdl_wait();
+    const int ntok_blocks = static_cast<int>(gridDim.x) - (tail.counts ? 1 : 0);
+    if (tail.counts && static_cast<int>(blockIdx.x) == ntok_blocks) {
+        stats_tail(tail, tail.T > 0 ? tail.T : T, K);
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(ntok_blocks) * (blockDim.x >> 5);
+    const int nvec = d / 4;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+        const int32_t my_row = lane < K ? inv[t * K + lane] : -1;
+        const float my_w = lane < K ? w[t * K + lane] : 0.f;
+        for (int c0 = lane; c0 < nvec; c0 += 64) {
+            const int c1 = c0 + 32;
+            const bool two = c1 < nvec;
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+            // slots in groups of 4: both columns' loads of a group in flight together
+            for (int k0 = 0; k0 < K; k0 += 4) {
+                float4 v0[4], v1[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = k0 + j;
+                    const int r = __shfl_sync(0xffffffffu, my_row, k < K ? k : 0);
+                    const bool live = k < K && r >= 0;
+                    const float4* base = reinterpret_cast<const float4*>(yp + static_cast<int64_t>(live ? r : 0) * d);
+                    v0[j] = live ? __ldg(base + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v1[j] = (live && two) ? __ldg(base + c1) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = k0 + j;
+                    const int r = __shfl_sync(0xffffffffu, my_row, k < K ? k : 0);
+                    const float wk = __shfl_sync(0xffffffffu, my_w, k < K ? k : 0);
+                    if (k < K && r >= 0) {
+                        a0.x = fmaf(wk, v0[j].x, a0.x);
+                        a0.y = fmaf(wk, v0[j].y, a0.y);
+                        a0.z = fmaf(wk, v0[j].z, a0.z);
+                        a0.w = fmaf(wk, v0[j].w, a0.w);
+                        a1.x = fmaf(wk, v1[j].x, a1.x);
+                        a1.y = fmaf(wk, v1[j].y, a1.y);
+                        a1.z = fmaf(wk, v1[j].z, a1.z);
+                        a1.w = fmaf(wk, v1[j].w, a1.w);
+                    }
+                }
+            }
+            store4(y + t * d, c0, a0);
+            if (two) store4(y + t * d, c1, a1);
+        }
+    }
+}
+
 // y_perm[r] = sum over slices s of part[s][r], rows r < offsets[E].
 __global__ void __launch_bounds__(256)
 reduce_splits_kernel(const float* __restrict__ part, int nsplit, int64_t split_stride,
@@ -324,6 +386,21 @@ int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const 
         tail = *tail_in;
         if (tail.part && !tail.P) return -2;
         ++grid;  // one extra CTA for the tail
+    }
+    if (nsplit == 1 && K <= 32 && d >= 128) {
+        // a warp per token: 8 tokens per CTA, the grid capped at 4 CTAs per SM
+        int64_t gw = (T + 7) / 8;
+        const int64_t cap = static_cast<int64_t>(sms) * 4;
+        if (gw > cap) gw = cap;
+        if (gw < 1) gw = 1;
+        if (tail.counts) ++gw;
+        if (y_bf16)
+            (void)launch_pdl(combine_warp_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(gw)), dim3(256), 0, st, y_perm,
+                             inv, w, T, d, K, static_cast<__nv_bfloat16*>(y), tail);
+        else
+            (void)launch_pdl(combine_warp_kernel<float>, dim3(static_cast<unsigned>(gw)), dim3(256), 0, st, y_perm, inv, w,
+                             T, d, K, static_cast<float*>(y), tail);
+        return cudaGetLastError() == cudaSuccess ? 0 : -3;
     }
     const int g = static_cast<int>(grid);
     if (y_bf16)
