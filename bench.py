@@ -278,7 +278,7 @@ def run_reference(args):
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{S} of {wl.T} tokens per step (routing, counts and capacity over all "
                                    f"{wl.T}); {steps} steps after {warm} warm-up (of {args.steps}/{args.warmup} "
-                                   f"asked, bounded to minutes)"},
+                                   f"asked, bounded to minutes); numpy fp64 with the BLAS threads given in cores"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
