@@ -406,10 +406,14 @@ MOE_API int moe_ep_regroup(int n_ranks, int E_local, const int32_t* recv_counts,
  *   directly by the kernel over the host link: no staging copy); other host
  *   memory is refused with MOE_EUNSUPPORTED before any launch.
  * moe_expert_ffn_slots: moe_expert_ffn with the weights of expert e read
- *   from slot expert_slot[e] ([E] int32, device) of W13c / W2c.  An expert
- *   with rows whose slot lies outside [0, n_slots) is never used as an
+ *   from slot expert_slot[e] ([E] int32, device) of W13c / W2c.  The slot
+ *   MOE_SLOT_SKIP skips expert e: its rows of h and y_perm are left as they
+ *   are (a second call with the complementary table fills them, so the
+ *   resident experts can run while the others are still loading).  Any other
+ *   slot outside [0, n_slots) of an expert with rows is never used as an
  *   address: slot 0 is read instead and the workspace status flag records
  *   MOE_EINDEX (detail 8). */
+#define MOE_SLOT_SKIP (-2)
 MOE_API int moe_int4_bytes(const moe_dims* dims, size_t* q13_bytes, size_t* s13_bytes, size_t* q2_bytes,
                            size_t* s2_bytes);
 MOE_API int moe_int4_pack(const moe_dims* dims, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,

@@ -27,6 +27,7 @@ MOE_EWORKSPACE = -4
 MOE_ETIMEOUT = -5
 MOE_ESCRATCH = -6
 MOE_EINDEX = -7
+MOE_SLOT_SKIP = -2  # slot table entry that leaves an expert out of moe_expert_ffn_slots
 
 EXPORTED = [
     "moe_status_str", "moe_version", "moe_capacity", "moe_workspace_size", "moe_reset_device_status",

@@ -252,6 +252,8 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
     for (int g = threadIdx.x; g <= G; g += blockDim.x)
         off[g] = a.group_off ? static_cast<int64_t>(a.group_off[g]) : (g == 0 ? 0 : a.dense_rows);
     __syncthreads();
+    // rows of group g in this launch (0 for a group the slot table skips)
+    auto rows_of = [&](int g) -> int64_t { return group_skipped(a.w_slot, g) ? 0 : off[g + 1] - off[g]; };
     if (warp == 0) {
         // tile prefix over (phase, group): each lane scans a contiguous span of groups
         const int span = (G + 31) / 32;
@@ -259,7 +261,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         int carry = 0;
         for (int p = 0; p < a.nphase; ++p) {
             int sum = 0;
-            for (int g = g0; g < g1; ++g) sum += tiles_of(a, p, off[g + 1] - off[g]);
+            for (int g = g0; g < g1; ++g) sum += tiles_of(a, p, rows_of(g));
             int incl = sum;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -270,7 +272,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
             int* ts = tstart + p * (G + 1);
             for (int g = g0; g < g1; ++g) {
                 ts[g] = run;
-                run += tiles_of(a, p, off[g + 1] - off[g]);
+                run += tiles_of(a, p, rows_of(g));
             }
             const int tot = __shfl_sync(0xffffffffu, incl, 31);
             if (lane == 0) ts[G] = carry + tot;

@@ -389,6 +389,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     pdl_trigger();
     for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
     __syncthreads();
+    // rows of group g in this launch (0 for a group the slot table skips)
+    auto rows_of = [&](int g) -> int64_t { return group_skipped(a.w_slot, g) ? 0 : off[g + 1] - off[g]; };
     if (warp == 0) {
         // Tile numbering per queue (0: token-major groups, 1: weight-major
         // groups), phase 0 then phase 1, groups in order; each lane scans a
@@ -399,7 +401,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
             int carry = 0;
             for (int p = 0; p < a.nphase; ++p) {
                 int sum = 0;
-                for (int g = g0; g < g1; ++g) sum += tiles_in_queue(a, q, p, off[g + 1] - off[g]);
+                for (int g = g0; g < g1; ++g) sum += tiles_in_queue(a, q, p, rows_of(g));
                 int incl = sum;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -410,7 +412,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 int* ts = tstart_all + (2 * q + p) * (G + 1);
                 for (int g = g0; g < g1; ++g) {
                     ts[g] = run;
-                    run += tiles_in_queue(a, q, p, off[g + 1] - off[g]);
+                    run += tiles_in_queue(a, q, p, rows_of(g));
                 }
                 const int tot = __shfl_sync(0xffffffffu, incl, 31);
                 if (lane == 0) ts[G] = carry + tot;

@@ -25,6 +25,12 @@ enum : int {
 // Weight matrix of group g: g itself, or its cache slot from `slot_of`
 // (nullptr: none).  A slot outside [0, n_slots) is never used as an address:
 // the status records DEV_BAD_SLOT and slot 0 is read instead.
+// Slot value that leaves group g out of a launch (its tiles are not counted).
+constexpr int32_t kSlotSkip = -2;
+__device__ __forceinline__ bool group_skipped(const int32_t* slot_of, int g) {
+    return slot_of != nullptr && slot_of[g] == kSlotSkip;
+}
+
 __device__ __forceinline__ int weight_slot(const int32_t* slot_of, int n_slots, int g, int* status) {
     if (slot_of == nullptr) return g;
     const int s = slot_of[g];

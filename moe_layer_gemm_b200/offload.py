@@ -9,18 +9,21 @@ cache of the frequently used experts on the GPU; predict from the routing
 history which experts the next batch needs and load them ahead of time; store
 the offloaded experts group-wise quantized to INT4 to cut the transfer volume.
 
-One step of OffloadedLayer (the main stream, plus a side stream for the
-prefetch):
+One step of OffloadedLayer (the main stream; a copy stream and an unpack
+stream for the experts that miss; a side stream for the prefetch):
   1 route and dispatch the batch (moe_route, moe_permute)
   2 read the per-expert kept counts on the host: the step's one host
     synchronisation, since which experts to load is decided here
   3 the cache plan (ExpertCache): hits refresh their slot; each miss, in
     ascending expert order, takes the least recently used slot holding no
     expert this step needs (equal last use: the lower slot)
-  4 expand the missed experts' INT4 codes from page-locked host memory into
-    their slots (moe_int4_unpack reads host memory directly: no staging copy)
-  5 the expert GEMMs reading each expert from its slot (moe_expert_ffn_slots),
-    then the combine (moe_combine)
+  4 each missed expert's INT4 codes are copied from page-locked host memory
+    into a device staging buffer by the copy engine (the host link's full
+    rate, no SM time), and expanded into its slot (moe_int4_unpack) as soon
+    as its copy has landed
+  5 meanwhile the expert GEMMs of the resident experts run
+    (moe_expert_ffn_slots with the missed experts skipped); then those of
+    the missed experts (the complementary table), then the combine
   6 update the prediction (HistoryPredictor: a per-expert fp32 moving average
     of routed counts) and expand the predicted experts that are not resident,
     on the side stream, into slots holding no expert of this step; the next
@@ -185,17 +188,58 @@ class OffloadedLayer:
         self.x_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=self.dev)
         self.h = torch.empty(T * K, f, dtype=torch.bfloat16, device=self.dev)
         self.y_perm = torch.empty(T * K, d, dtype=torch.float32, device=self.dev)
-        self.slot_dev = torch.full((E,), -1, **i32)
-        self.slot_host = torch.empty(E, dtype=torch.int32, pin_memory=True)
+        # slot tables: [0] the resident experts (misses skipped), [1] the misses
+        self.slot_dev = [torch.full((E,), abi.MOE_SLOT_SKIP, **i32) for _ in range(2)]
+        self.slot_host = [torch.empty(E, dtype=torch.int32, pin_memory=True) for _ in range(2)]
         self.counts_host = torch.empty(2 * E, dtype=torch.int32, pin_memory=True)
         self.side = torch.cuda.Stream(self.dev)
+        self.copy = torch.cuda.Stream(self.dev)
+        self.unpack_stream = torch.cuda.Stream(self.dev)
         self.dispatched = torch.cuda.Event()
+        self.unpacked = torch.cuda.Event()
+        # per-expert views of the host codes, and device staging buffers for the misses
+        self.host_views = tuple(t.view(E, -1) for t in (q13, s13, q2, s2))
+        self.stage = None
         self.log: List[dict] = []
 
     def _unpack(self, loads, stream):
+        """Expand experts straight from page-locked host memory (the prefetch)."""
         if loads:
             abi.moe_int4_unpack(self.dims, [e for e, _ in loads], [s for _, s in loads], self.q13, self.s13,
                                 self.q2, self.s2, self.n_slots, self.W13c, self.W2c, stream)
+
+    def _stage(self, n: int):
+        """Device staging buffers for n missed experts (grown on need)."""
+        if self.stage is None or self.stage[0].shape[0] < n:
+            self.stage = tuple(torch.empty((n, v.shape[1]), dtype=v.dtype, device=self.dev) for v in self.host_views)
+        return self.stage
+
+    def _load_misses(self, loads):
+        """Copy each missed expert's codes to the device on the copy stream and
+        expand it into its slot on the unpack stream once its copy has landed;
+        self.unpacked marks the end."""
+        stage = self._stage(len(loads))
+        unpack = self.unpack_stream
+        for j, (e, sl) in enumerate(loads):
+            copied = torch.cuda.Event()
+            with torch.cuda.stream(self.copy):
+                for dst, src in zip(stage, self.host_views):
+                    dst[j].copy_(src[e], non_blocking=True)
+                copied.record(self.copy)
+            unpack.wait_event(copied)
+            flat = tuple(t.view(-1) for t in stage)
+            abi.moe_int4_unpack(self.dims, [j], [sl], *flat, self.n_slots, self.W13c, self.W2c, unpack)
+        self.unpacked.record(unpack)
+
+    def _ffn(self, table: int, which: np.ndarray):
+        """Expert GEMMs of the experts with which[e] set (the others skipped)."""
+        dims = self.dims
+        slots = self.cache.slot_table(dims.E)
+        t = np.where(which, slots, abi.MOE_SLOT_SKIP).astype(np.int32)
+        self.slot_host[table].copy_(torch.from_numpy(t))
+        self.slot_dev[table].copy_(self.slot_host[table], non_blocking=True)
+        abi.moe_expert_ffn_slots(dims, self.x_perm, self.offsets, self.slot_dev[table], self.n_slots, self.W13c,
+                                 self.W2c, self.h, self.y_perm, self.ws)
 
     def forward(self, x, y):
         dims, E = self.dims, self.dims.E
@@ -212,11 +256,19 @@ class OffloadedLayer:
         needed = [int(e) for e in np.nonzero(kept)[0]]
         hits, phits, misses, loads = self.cache.plan(needed)
         main.wait_stream(self.side)                           # the last prefetch has landed
-        self._unpack(loads, main)
-        self.slot_host.copy_(torch.from_numpy(self.cache.slot_table(E)))
-        self.slot_dev.copy_(self.slot_host, non_blocking=True)
-        abi.moe_expert_ffn_slots(dims, self.x_perm, self.offsets, self.slot_dev, self.n_slots, self.W13c, self.W2c,
-                                 self.h, self.y_perm, self.ws)
+        missed = np.zeros(E, dtype=bool)
+        missed[misses] = True
+        resident = (kept > 0) & ~missed
+        if loads:
+            # the copies start after the prefetch (its slots) and the last step's reads of the slots
+            self.copy.wait_stream(main)
+            self.unpack_stream.wait_stream(main)
+            self._load_misses(loads)
+        if resident.any():
+            self._ffn(0, resident)                            # overlaps the copies of the misses
+        if loads:
+            main.wait_event(self.unpacked)
+            self._ffn(1, missed)
         abi.moe_combine(dims, self.y_perm, self.inv, self.w, y)
         ploads = []
         if self.predictor is not None:

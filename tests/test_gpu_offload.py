@@ -120,6 +120,46 @@ def test_slot_indirected_ffn_equals_ffn(T, d, f, E, K):
     assert torch.equal(y1[:n].view(torch.int32), y2[:n].view(torch.int32))
 
 
+@pytest.mark.parametrize("T,d,f,E,K", [(300, 256, 192, 16, 4), (512, 512, 512, 16, 4), (256, 512, 512, 8, 2)])
+def test_skipped_experts_then_complement_equal_one_call(T, d, f, E, K):
+    """Two calls with complementary slot tables (MOE_SLOT_SKIP for the experts
+    the other call covers) write the same h and y_perm as one call with all
+    experts: a skipped expert's rows are left alone, the others are computed
+    exactly as before."""
+    dv = dev()
+    dims = abi.Dims(T, d, f, E, K)
+    W1, W3, W2 = _weights(E, d, f, 21)
+    W13p, W2p = abi.pack_weights(dims, W1, W3, W2)
+    idx = synth.distinct_choices(T, E, K, seed=T + 1, weights=torch.tensor([(r + 1.0) ** -1.2 for r in range(E)])).to(dv)
+    x = synth.normal_bf16((T, d), 6, synth.STREAM_X, 1.0, dv)
+    ws = abi.alloc_workspace(dims)
+    i32 = dict(dtype=torch.int32, device=dv)
+    A = T * K
+    counts, kept, offsets = torch.empty(E, **i32), torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    inv, src = torch.empty(T, K, **i32), torch.empty(A, **i32)
+    xp = torch.zeros(A, d, dtype=torch.bfloat16, device=dv)
+    abi.moe_permute(dims, idx, x, counts, kept, offsets, inv, src, xp, None, ws)
+    ident = torch.arange(E, **i32)
+    h1, h2 = (torch.zeros(A, f, dtype=torch.bfloat16, device=dv) for _ in range(2))
+    y1, y2 = (torch.zeros(A, d, dtype=torch.float32, device=dv) for _ in range(2))
+    abi.moe_expert_ffn_slots(dims, xp, offsets, ident, E, W13p, W2p, h1, y1, ws)
+    odd = torch.arange(E, device=dv) % 2 == 1
+    first = torch.where(odd, torch.full_like(ident, abi.MOE_SLOT_SKIP), ident)
+    second = torch.where(odd, ident, torch.full_like(ident, abi.MOE_SLOT_SKIP))
+    abi.moe_expert_ffn_slots(dims, xp, offsets, first, E, W13p, W2p, h2, y2, ws)
+    torch.cuda.synchronize()
+    n = int(offsets[-1].item())
+    off = offsets.cpu().numpy()
+    # after the first call the odd experts' rows are untouched (still zero)
+    for e in range(1, E, 2):
+        assert torch.count_nonzero(y2[off[e]:off[e + 1]]) == 0
+    abi.moe_expert_ffn_slots(dims, xp, offsets, second, E, W13p, W2p, h2, y2, ws)
+    torch.cuda.synchronize()
+    assert abi.moe_get_device_status(ws)[0] == abi.MOE_OK
+    assert torch.equal(h1[:n].view(torch.int16), h2[:n].view(torch.int16))
+    assert torch.equal(y1[:n].view(torch.int32), y2[:n].view(torch.int32))
+
+
 def test_offloaded_layer_steps_match_oracle():
     """Eight decode-sized steps (fresh tokens each) with 16 experts in host
     memory and 10 cache slots, 3 predicted experts loaded ahead per step."""
