@@ -64,3 +64,9 @@ def test_timeout_cta_pair_kernel():
 def test_timeout_cta_pair_token_major_tiles():
     # groups of ~1024 rows: token-major 256 x 256 pair tiles
     _aborted_then_normal("mixtral_prefill", 4096, "grouped_gemm_2sm_kernel")
+
+
+def test_timeout_cta_pair_both_queues():
+    # skewed groups above and below 128 rows: token-major pairs (two k-blocks
+    # per stage) and weight-major pairs (one) abort and drain in one launch
+    _aborted_then_normal("deepseek_bias", 1024, "grouped_gemm_2sm_kernel")
