@@ -212,6 +212,9 @@ class OffloadedLayer:
         """Device staging buffers for n missed experts (grown on need)."""
         if self.stage is None or self.stage[0].shape[0] < n:
             self.stage = tuple(torch.empty((n, v.shape[1]), dtype=v.dtype, device=self.dev) for v in self.host_views)
+            for t in self.stage:  # used on the copy and unpack streams: the allocator must wait for them
+                t.record_stream(self.copy)
+                t.record_stream(self.unpack_stream)
         return self.stage
 
     def _load_misses(self, loads):
