@@ -21,7 +21,13 @@
 //                 contiguous 16 KB bulk copies of the pre-tiled,
 //                 pre-swizzled packed weights
 //   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..5    epilogue: TMEM -> registers -> SwiGLU / fp32 -> global
+//   warps 2..5    epilogue: TMEM -> registers -> SwiGLU / fp32 -> global.
+//                 fp32 rows of token-major tiles go through a 4 KB staging
+//                 buffer per warp and one TMA tile store per 32 x 32 block:
+//                 stored from registers, each 16-byte store touched 32 rows,
+//                 and the down projection's short tiles (reduction d_ff) could
+//                 not hide them (Qwen-like layer: expert GEMMs 0.430 ->
+//                 0.412 ms; the same layer with no fp32 stores at all, 0.39)
 // Two producers: the copies one thread issues after a barrier wait are
 // serviced one stage at a time (a measured property of the copy engine:
 // about 0.4 us per stage and issuing thread, whatever the ring depth), so a
@@ -39,6 +45,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <cstring>
 
 #include "internal.h"
@@ -69,6 +76,8 @@ struct PhaseArgs {
     void* out;
     int64_t ldo;
     int64_t split_stride;
+    int tma_out;         // fp32 token-major tiles store full 32-row slabs by TMA (Maps::out)
+    int64_t split_rows;  // rows between partial slices in the output map (split_stride / ldo)
 };
 
 struct DevArgs {
@@ -82,6 +91,7 @@ struct DevArgs {
     PhaseArgs ph[2];
     int stages;                 // operand ring depth; a stage holds one weight and one token slot
     uint32_t wslot, xslot;      // bytes per weight / token slot
+    int stg_bufs;               // 4 KB output staging buffers per epilogue warp (0: none)
     int* status;
     int* sched;         // [0] tile counter, [1..G] phase-0 tiles done per group (x4 warps)
     uint32_t wait_limit;      // polls of a bounded mbarrier or drain wait
@@ -94,6 +104,7 @@ struct DevArgs {
 struct Maps {
     CUtensorMap tokA[2];  // token rows, box 128 (token-major A)
     CUtensorMap tokB[2];  // token rows, box 32  (weight-major B)
+    CUtensorMap out[2];   // fp32 output rows, box {32 columns, 32 rows}, 128-byte swizzle (phases with tma_out)
 };
 
 struct Tile {
@@ -203,7 +214,8 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
     const int S = a.stages;
     uint8_t* sW = smem;                                               // [S][wslot]
     uint8_t* sX = smem + static_cast<size_t>(S) * a.wslot;            // [S][xslot]
-    uint64_t* full = reinterpret_cast<uint64_t*>(sX + static_cast<size_t>(S) * a.xslot);
+    uint8_t* sStg = sX + static_cast<size_t>(S) * a.xslot;           // [4 warps][stg_bufs][4 KB]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sStg + static_cast<size_t>(a.stg_bufs) * 4 * 4096);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
@@ -441,6 +453,7 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         uint32_t r = 0, rph = 0;
         int it = 0;
+        uint32_t nst = 0;  // staged tile stores this warp issued
         for (;;) {
             if (!mbar_wait(&rfull[r], rph, a.status, DEV_TIMEOUT_EPI_TFULL, abort_flag, a.wait_limit)) break;
             const int tile = ring[r];
@@ -463,8 +476,29 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 const bool valid = rr < t.rows;
                 const int64_t grow = t.row0 + rr;
                 const int nchunks = pa.BN / 32;
+                // fp32 output of a slab whose 32 rows all belong to the group: staged
+                // in shared memory and written by one TMA tile store per chunk
+                const bool staged = pa.tma_out && a.stg_bufs > 0 && q * 32 + 32 <= t.rows;
                 for (int c = 0; c < nchunks; ++c) {
                     tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                    if (staged) {
+                        uint8_t* stg = sStg + static_cast<size_t>(q * a.stg_bufs + static_cast<int>(nst % a.stg_bufs)) * 4096;
+                        if (lane == 0) {
+                            // the store that last used this buffer has read it
+                            if (a.stg_bufs > 1) bulk_wait_read<1>(); else bulk_wait_read<0>();
+                        }
+                        __syncwarp();
+                        stage_row_f32_sw128(stg, lane, v);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&maps.out[t.phase], stg, t.n0 + c * 32,
+                                         static_cast<int32_t>(t.split * pa.split_rows + t.row0 + q * 32));
+                            bulk_commit();
+                        }
+                        ++nst;
+                        continue;
+                    }
                     if (!valid) continue;
                     if (pa.epi == EPI_SWIGLU_BF16) {
                         uint32_t pk[8];
@@ -538,6 +572,8 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
         }
     }
 
+    // staged output stores complete (and stop reading shared memory) before the CTA exits
+    if (warp >= 2 && warp != kProducer1Warp && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -577,6 +613,35 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 }  // namespace
+
+// 2D fp32 map over [rows, cols] (cols contiguous, row stride ld elements)
+// with box {32, 32} and the 128-byte swizzle of the staged output tiles.
+bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
+    cuuint64_t strides[1] = {ld * 4};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Whether a phase's fp32 output can take staged TMA tile stores: full-width
+// rows (no clipped columns), 16-byte aligned rows and base, partial slices a
+// whole number of rows apart.
+bool out_map_ok(const GemmPhase& g) {
+    return g.epi == EPI_F32 && g.out != nullptr && g.N_store == g.N && g.N % 32 == 0 && g.ldo % 4 == 0 &&
+           g.ldo >= g.N && (reinterpret_cast<uintptr_t>(g.out) & 15u) == 0 &&
+           (g.ksplit <= 1 || g.split_stride % g.ldo == 0);
+}
+
+// Rows of the output map of a phase that out_map_ok accepts (every partial slice).
+uint64_t out_map_rows(const GemmPhase& g, int ksplit) {
+    const int64_t split_rows = ksplit > 1 ? g.split_stride / g.ldo : 0;
+    return static_cast<uint64_t>(static_cast<int64_t>(ksplit - 1) * split_rows + g.tok_rows);
+}
 
 int num_sms() {
     int dev = 0;
@@ -664,12 +729,21 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
     const size_t fixed = 1024 + static_cast<size_t>(2 * 16 + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
                          static_cast<size_t>(L.G + 1) * (8 + 2 * 4) + 64;
     const size_t budget = 227 * 1024 - fixed;
-    int stages = static_cast<int>(budget / (wslot + xslot));
-    if (stages > 16) stages = 16;
-    stages &= ~1;  // even: each of the two producers owns the stages of one parity
+    // even: each of the two producers owns the stages of one parity
+    auto ring_stages = [&](size_t bytes) { return std::min(static_cast<int>(bytes / (wslot + xslot)), 16) & ~1; };
+    const int stages = ring_stages(budget);
     if (stages < 2) return -2;
     a.stages = stages;
-    const size_t smem = fixed + static_cast<size_t>(stages) * (wslot + xslot);
+    // Output staging for fp32 token-major tiles (4 epilogue warps x 4 KB per
+    // buffer): two buffers per warp, else one, where the ring keeps its depth.
+    bool want_stg = false;
+    for (int p = 0; p < L.nphase; ++p) want_stg = want_stg || out_map_ok(L.ph[p]);
+    a.stg_bufs = 0;
+    for (int nb = 2; want_stg && nb >= 1 && a.stg_bufs == 0; --nb) {
+        const size_t stg = static_cast<size_t>(nb) * 4 * 4096;
+        if (budget > stg && ring_stages(budget - stg) == stages) a.stg_bufs = nb;
+    }
+    const size_t smem = fixed + static_cast<size_t>(stages) * (wslot + xslot) + static_cast<size_t>(a.stg_bufs) * 4 * 4096;
 
     Maps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -678,6 +752,10 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         const uint64_t tok_rows = static_cast<uint64_t>(g.tok_rows < 1 ? 1 : g.tok_rows);
         if (!make_map(&maps.tokA[p], g.tok, tok_rows, g.Kdim, 128u)) return -3;
         if (!make_map(&maps.tokB[p], g.tok, tok_rows, g.Kdim, 32u)) return -3;
+        PhaseArgs& ph = a.ph[p];
+        ph.tma_out = (a.stg_bufs > 0 && out_map_ok(g)) ? 1 : 0;
+        ph.split_rows = ph.tma_out && ph.ksplit > 1 ? g.split_stride / g.ldo : 0;
+        if (ph.tma_out && !make_out_map(&maps.out[p], g.out, out_map_rows(g, ph.ksplit), g.N, g.ldo)) return -3;
     }
 
     static std::atomic<unsigned long long> attr_done{0};

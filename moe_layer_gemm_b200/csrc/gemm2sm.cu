@@ -35,6 +35,11 @@
 // 5.13-5.17 -> 4.90-4.94 ms on one box).  A launch with one kind of tile
 // puts every pair on its queue.
 //
+// fp32 output of token-major tiles (the down projection) leaves through a
+// 4 KB staging buffer per epilogue warp and one TMA tile store per 32 x 32
+// block, as in gemm.cu; the buffers sit after the token-major ring (two per
+// warp where they fit, else one).
+//
 // Stage layout (per CTA and k-block): token-major tiles put their 128 token
 // rows at 0 and their 128 weight rows at 16 KB; weight-major tiles put
 // weight sub-tile j at 16 KB j and their token rows at xoff.  A stage holds
@@ -90,6 +95,8 @@ struct Phase2 {
     void* out;
     int64_t ldo;
     int64_t split_stride;
+    int tma_out;         // fp32 token-major tiles store full 32-row slabs by TMA (Maps2::out)
+    int64_t split_rows;  // rows between partial slices in the output map
 };
 
 struct Args2 {
@@ -104,7 +111,9 @@ struct Args2 {
     int stages[2];
     uint32_t stage_bytes[2];  // per k-block and CTA
     int kpb[2];               // k-blocks per stage (1 or 2)
-    size_t ring_bytes;        // shared memory of the larger ring
+    size_t ring_bytes;        // shared memory of the larger ring (token-major: with its output staging)
+    int stg_bufs;             // token-major pairs: 4 KB output staging buffers per epilogue warp (0: none)
+    uint32_t stg_off;         // offset of the staging buffers (after the token-major ring)
     uint32_t xoff;            // weight-major tiles: offset of the token rows in a k-block
     int* status;
     int* sched;  // [0] token-major tile counter, [1 + g] phase-0 stores of group g, [G + 1] weight-major tile counter
@@ -131,6 +140,7 @@ struct Maps2 {
     CUtensorMap tok16[2];  // token rows, box 16, 128-byte swizzle (weight-major halves)
     CUtensorMap tok64[2];  // token rows, box 64, 128-byte swizzle (weight-major halves of >= 64 rows)
     CUtensorMap w[2];    // tiled weights as [rows, 64], box 128, no swizzle (tiles are pre-swizzled)
+    CUtensorMap out[2];  // fp32 output rows, box {32 columns, 32 rows}, 128-byte swizzle (phases with tma_out)
 };
 
 struct Tile2 {
@@ -662,6 +672,7 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
         const int q = warp & 3;
         uint32_t r = 0, rph = 0;
         int it = 0;
+        uint32_t nst = 0;  // staged tile stores this warp issued
         for (;;) {
             if (!pwait(&rfull[r], rph, a, DEV_TIMEOUT_EPI_TFULL, abort_flag, peer_abort)) break;
             const int tile = ring[r];
@@ -682,8 +693,31 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                 const int rr = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the pair's 256
                 const bool valid = rr < t.rows;
                 const int64_t grow = t.row0 + rr;
+                // fp32 output of a slab whose 32 rows all belong to the group: staged
+                // in shared memory and written by one TMA tile store per chunk
+                const int slab0 = static_cast<int>(rank) * 128 + q * 32;
+                const bool staged = pa.tma_out && a.stg_bufs > 0 && slab0 + 32 <= t.rows;
                 for (int c = 0; c < 8; ++c) {
                     tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                    if (staged) {
+                        uint8_t* stg = smem + a.stg_off +
+                                       static_cast<size_t>(q * a.stg_bufs + static_cast<int>(nst % a.stg_bufs)) * 4096;
+                        if (lane == 0) {
+                            // the store that last used this buffer has read it
+                            if (a.stg_bufs > 1) bulk_wait_read<1>(); else bulk_wait_read<0>();
+                        }
+                        __syncwarp();
+                        stage_row_f32_sw128(stg, lane, v);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&maps.out[t.phase], stg, t.n0 + c * 32,
+                                         static_cast<int32_t>(t.split * pa.split_rows + t.row0 + slab0));
+                            bulk_commit();
+                        }
+                        ++nst;
+                        continue;
+                    }
                     if (!valid) continue;
                     if (pa.epi == EPI_SWIGLU_BF16) {
                         uint32_t pk[8];
@@ -751,6 +785,8 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
         }
     }
 
+    // staged output stores complete (and stop reading shared memory) before the CTA exits
+    if (warp >= 2 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // the peer's TMEM and shared memory stay alive until the leader is done
@@ -857,6 +893,9 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         const uint64_t wmats = static_cast<uint64_t>(L.w_slot ? L.w_slots : L.G);
         const uint64_t wrows = wmats * ph.nb * ph.k_blocks * 128;
         if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
+        ph.tma_out = out_map_ok(g) ? 1 : 0;  // cleared below if no staging fits
+        ph.split_rows = ph.tma_out && ph.ksplit > 1 ? g.split_stride / g.ldo : 0;
+        if (ph.tma_out && !make_out_map(&maps.out[p], g.out, out_map_rows(g, ph.ksplit), g.N, g.ldo)) return -3;
     }
     const size_t fixed = 1024 + static_cast<size_t>(2 * kMaxStages + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
                          static_cast<size_t>(L.G + 1) * (8 + 4 * 4) + 4 + sizeof(PeerReport) + 64;
@@ -880,16 +919,29 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     const size_t avail = 227 * 1024 - fixed;
     a.stage_bytes[0] = 2u * kHalf;
     a.stage_bytes[1] = a.xoff + static_cast<uint32_t>(a.BNs) * 64u;
-    size_t ring = 0;
+    size_t ring = 0, ring_q[2] = {0, 0};
     for (int q = 0; q < 2; ++q) {
         a.kpb[q] = (q == 0 && avail / (2 * static_cast<size_t>(a.stage_bytes[0])) >= 3) ? 2 : 1;
         int stages = static_cast<int>(avail / (a.kpb[q] * static_cast<size_t>(a.stage_bytes[q])));
         if (stages > kMaxStages) stages = kMaxStages;
         if (stages < 2) return -2;
         a.stages[q] = stages;
-        const size_t bytes = static_cast<size_t>(stages) * a.kpb[q] * a.stage_bytes[q];
-        ring = bytes > ring ? bytes : ring;
+        ring_q[q] = static_cast<size_t>(stages) * a.kpb[q] * a.stage_bytes[q];
     }
+    // Output staging of token-major pairs (4 epilogue warps x 4 KB per buffer)
+    // after their ring: two buffers per warp, else one, in the room the ring
+    // leaves.  Weight-major pairs never touch it (their epilogue stores
+    // columns of 32 tokens, already whole rows), so it may overlap their ring.
+    bool want_stg = false;
+    for (int p = 0; p < L.nphase; ++p) want_stg = want_stg || a.ph[p].tma_out;
+    a.stg_bufs = 0;
+    for (int nb = 2; want_stg && nb >= 1 && a.stg_bufs == 0; --nb)
+        if (ring_q[0] + static_cast<size_t>(nb) * 4 * 4096 <= avail) a.stg_bufs = nb;
+    if (a.stg_bufs == 0)
+        for (int p = 0; p < L.nphase; ++p) a.ph[p].tma_out = 0;
+    a.stg_off = static_cast<uint32_t>(ring_q[0]);
+    ring = ring_q[0] + static_cast<size_t>(a.stg_bufs) * 4 * 4096;
+    if (ring_q[1] > ring) ring = ring_q[1];
     a.ring_bytes = ring;
     const size_t smem = fixed + ring;
     static std::atomic<unsigned long long> attr_done{0};

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstdint>
 #include <cstddef>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -90,6 +91,12 @@ struct GemmLaunch {
     const int32_t* w_slot = nullptr;
     int w_slots = 0;
 };
+
+// Staged fp32 output stores (gemm.cu): whether a phase qualifies, the rows
+// of its output map, and the map itself (box {32, 32}, 128-byte swizzle).
+bool out_map_ok(const GemmPhase& g);
+uint64_t out_map_rows(const GemmPhase& g, int ksplit);
+bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint64_t ld);
 
 // Test-only settings of the expert-GEMM launches (see moe_test_set_wait_limits
 // in the header); all zero in production.

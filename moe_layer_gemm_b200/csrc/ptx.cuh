@@ -165,6 +165,40 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
         : "memory");
 }
 
+// ------------------------------------------------ staged fp32 tile stores
+// An epilogue warp holds 32 rows x 32 fp32 columns of an output tile, one
+// row per lane.  Stored directly, each 16-byte store instruction touches 32
+// rows; instead the warp writes them into a 4 KB staging buffer (1024-byte
+// aligned) in the 128-byte-swizzled layout of a TMA box {32 columns, 32 rows}
+// (16-byte chunk j of row r at chunk j ^ (r mod 8): each quarter-warp's
+// stores cover all 32 banks), and one lane stores the box with a TMA tile
+// store.  Column x must be a multiple of 4 (16 bytes); a store is clipped at
+// the tensor map's extent, never at a group boundary, so only fully valid
+// 32-row slabs go this way.
+__device__ __forceinline__ void stage_row_f32_sw128(uint8_t* stg, int lane, const float* v) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
+// Make this thread's shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 2D tiled store shared -> global of the box at (x, y), in this thread's
+// bulk async-group (commit with bulk_commit).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Until all of this thread's committed bulk groups are complete (writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Element offset of (row n, column k) of a K-major bf16 matrix stored as
 // 128-row x 64-column tiles (row-block-major, then column-block) with the
 // 128-byte swizzle inside each 16 KB tile: the 16-byte chunk c of row r sits
