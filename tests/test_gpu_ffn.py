@@ -79,6 +79,8 @@ def _run(T, d, f, E, K, skew=0.0, seed=11, w_std=0.05):
     (1024, 1024, 1024, 256, 8, 1.1),  # CTA pairs, two weight sub-tiles in both phases, skewed small groups
     (2000, 256, 256, 1, 1, 0.0),      # one expert (dense FFN) on CTA-pair token-major tiles, ragged tail
     (1, 256, 512, 8, 2, 0.0),         # a single token: two one-row groups on CTA-pair weight-major tiles
+    (1024, 256, 512, 16, 4, 1.2),     # CTA pairs, both queues: 128-row pair tiles for the last chunks of groups of 321-893 rows
+    (1024, 256, 512, 8, 2, 1.5),      # CTA pairs, both queues: 128-row last chunks of 17 and 43 rows
     # mid-sized groups: single-CTA token-major tiles with ragged 128-row tails
     (3000, 256, 384, 12, 2, 0.5),
     (4000, 512, 256, 8, 1, 1.2),      # skewed: groups from tens to ~1500 rows
