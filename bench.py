@@ -45,7 +45,11 @@ sys.path.insert(0, ROOT)
 from moe_layer_gemm_b200 import synth  # noqa: E402
 
 METRIC = "MoE-layer tokens/s on 1 B200 (Mixtral shape decode/prefill); % of roofline"
-STAGE_EVERY = 4  # steps between the ones that carry per-stage events
+# steps between the ones that carry per-stage events; workloads that draw
+# fresh tokens every step carry them on every step, so the stage times
+# average over all their token sets (every 4th step of 10 token sets would
+# see only half of them)
+STAGE_EVERY = 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -350,7 +354,7 @@ class Layer:
 STAGES = ("route", "dispatch", "expert_gemms", "combine_stats")
 
 
-def time_steps(layer: Layer, K: int, barrier, clock_index: int, stage_every: int = STAGE_EVERY, start_step: int = 0):
+def time_steps(layer: Layer, K: int, barrier, clock_index: int, stage_every=None, start_step: int = 0):
     """Time K layer steps with CUDA events on the launching stream (barrier
     and device synchronisation on both sides); per-stage events ride on every
     stage_every-th step (an event between two kernels keeps the second from
@@ -358,6 +362,8 @@ def time_steps(layer: Layer, K: int, barrier, clock_index: int, stage_every: int
     sampled during the region."""
     from moe_layer_gemm_b200 import abi
     nev = abi.NUM_STAGE_EVENTS
+    if stage_every is None:
+        stage_every = 1 if len(layer.xs) > 1 else STAGE_EVERY
     sampled = list(range(0, K, stage_every)) if layer.chunk == 0 and stage_every > 0 else []
     evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(nev)] for i in sampled}
     s = torch.cuda.current_stream()

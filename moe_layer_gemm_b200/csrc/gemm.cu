@@ -77,6 +77,7 @@ struct PhaseArgs {
     int64_t ldo;
     int64_t split_stride;
     int tma_out;         // fp32 token-major tiles store full 32-row slabs by TMA (Maps::out)
+    int tma_h;           // SwiGLU token-major tiles store full 32-row slabs of H by TMA (Maps::out)
     int64_t split_rows;  // rows between partial slices in the output map (split_stride / ldo)
 };
 
@@ -104,7 +105,7 @@ struct DevArgs {
 struct Maps {
     CUtensorMap tokA[2];  // token rows, box 128 (token-major A)
     CUtensorMap tokB[2];  // token rows, box 32  (weight-major B)
-    CUtensorMap out[2];   // fp32 output rows, box {32 columns, 32 rows}, 128-byte swizzle (phases with tma_out)
+    CUtensorMap out[2];   // output rows, 128-byte swizzle: fp32 box {32, 32} (tma_out) or bf16 box {64, 32} (tma_h)
 };
 
 struct Tile {
@@ -479,8 +480,40 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 // fp32 output of a slab whose 32 rows all belong to the group: staged
                 // in shared memory and written by one TMA tile store per chunk
                 const bool staged = pa.tma_out && a.stg_bufs > 0 && q * 32 + 32 <= t.rows;
+                // H of such a slab: four chunks (64 columns of H) fill one staging
+                // buffer, written by one TMA tile store
+                const bool staged_h = pa.tma_h && a.stg_bufs > 0 && q * 32 + 32 <= t.rows;
                 for (int c = 0; c < nchunks; ++c) {
                     tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+                    if (staged_h) {
+                        const int sub = c & 3;
+                        uint8_t* stg = sStg + static_cast<size_t>(q * a.stg_bufs + static_cast<int>(nst % a.stg_bufs)) * 4096;
+                        if (sub == 0) {
+                            if (lane == 0) {
+                                if (a.stg_bufs > 1) bulk_wait_read<1>(); else bulk_wait_read<0>();
+                            }
+                            __syncwarp();
+                        }
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = pack_bf16x2(silu_f(v[2 * i]) * v[16 + 2 * i],
+                                                silu_f(v[2 * i + 1]) * v[16 + 2 * i + 1]);
+                        uint8_t* row = stg + lane * 128;
+                        *reinterpret_cast<uint4*>(row + (((2 * sub) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4*>(row + (((2 * sub + 1) ^ (lane & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        if (sub == 3) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d(&maps.out[t.phase], stg, t.n0 / 2 + (c >> 2) * 64,
+                                             static_cast<int32_t>(t.row0 + q * 32));
+                                bulk_commit();
+                            }
+                            ++nst;
+                        }
+                        continue;
+                    }
                     if (staged) {
                         uint8_t* stg = sStg + static_cast<size_t>(q * a.stg_bufs + static_cast<int>(nst % a.stg_bufs)) * 4096;
                         if (lane == 0) {
@@ -564,6 +597,8 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                 mbar_arrive(&tempty[buf]);
                 if (t.phase == 0 && a.dep) {
                     // publish this warp's rows of H to the phase-1 tiles of group g
+                    // (rows written by TMA tile stores must have landed first)
+                    if (pa.tma_h) bulk_wait_all();
                     fence_proxy_async_global();
                     __threadfence();
                     atomicAdd(&a.sched[1 + t.g], 1);
@@ -614,16 +649,18 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 }  // namespace
 
-// 2D fp32 map over [rows, cols] (cols contiguous, row stride ld elements)
-// with box {32, 32} and the 128-byte swizzle of the staged output tiles.
-bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+// 2D output map over [rows, cols] (cols contiguous, row stride ld elements)
+// with a box of 32 rows x 128 bytes (32 fp32 or 64 bf16 columns) and the
+// 128-byte swizzle of the staged output tiles.
+bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint64_t ld, bool bf16_out) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows < 1 ? 1 : rows};
-    cuuint64_t strides[1] = {ld * 4};
-    cuuint32_t box[2] = {32u, 32u};
+    cuuint64_t strides[1] = {ld * (bf16_out ? 2 : 4)};
+    cuuint32_t box[2] = {bf16_out ? 64u : 32u, 32u};  // 128 bytes of a row
     cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    return enc(m, bf16_out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims,
+               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -635,6 +672,13 @@ bool out_map_ok(const GemmPhase& g) {
     return g.epi == EPI_F32 && g.out != nullptr && g.N_store == g.N && g.N % 32 == 0 && g.ldo % 4 == 0 &&
            g.ldo >= g.N && (reinterpret_cast<uintptr_t>(g.out) & 15u) == 0 &&
            (g.ksplit <= 1 || g.split_stride % g.ldo == 0);
+}
+
+// Whether a SwiGLU phase's bf16 H can take staged TMA tile stores (token-major
+// tiles of BN = 128 or 256, so four chunks make whole 64-column boxes).
+bool h_map_ok(const GemmPhase& g) {
+    return g.epi == EPI_SWIGLU_BF16 && g.out != nullptr && g.ksplit <= 1 && g.ldo % 8 == 0 && g.N % 128 == 0 &&
+           (reinterpret_cast<uintptr_t>(g.out) & 15u) == 0;
 }
 
 // Rows of the output map of a phase that out_map_ok accepts (every partial slice).
@@ -737,7 +781,7 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
     // Output staging for fp32 token-major tiles (4 epilogue warps x 4 KB per
     // buffer): two buffers per warp, else one, where the ring keeps its depth.
     bool want_stg = false;
-    for (int p = 0; p < L.nphase; ++p) want_stg = want_stg || out_map_ok(L.ph[p]);
+    for (int p = 0; p < L.nphase; ++p) want_stg = want_stg || out_map_ok(L.ph[p]) || h_map_ok(L.ph[p]);
     a.stg_bufs = 0;
     for (int nb = 2; want_stg && nb >= 1 && a.stg_bufs == 0; --nb) {
         const size_t stg = static_cast<size_t>(nb) * 4 * 4096;
@@ -754,8 +798,11 @@ int launch_grouped_gemm(const GemmLaunch& L, cudaStream_t st) {
         if (!make_map(&maps.tokB[p], g.tok, tok_rows, g.Kdim, 32u)) return -3;
         PhaseArgs& ph = a.ph[p];
         ph.tma_out = (a.stg_bufs > 0 && out_map_ok(g)) ? 1 : 0;
+        ph.tma_h = (a.stg_bufs > 0 && h_map_ok(g) && ph.BN % 128 == 0) ? 1 : 0;
         ph.split_rows = ph.tma_out && ph.ksplit > 1 ? g.split_stride / g.ldo : 0;
-        if (ph.tma_out && !make_out_map(&maps.out[p], g.out, out_map_rows(g, ph.ksplit), g.N, g.ldo)) return -3;
+        if (ph.tma_out && !make_out_map(&maps.out[p], g.out, out_map_rows(g, ph.ksplit), g.N, g.ldo, false)) return -3;
+        if (ph.tma_h && !make_out_map(&maps.out[p], g.out, static_cast<uint64_t>(g.tok_rows), g.N / 2, g.ldo, true))
+            return -3;
     }
 
     static std::atomic<unsigned long long> attr_done{0};

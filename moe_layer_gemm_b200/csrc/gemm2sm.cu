@@ -928,7 +928,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
         if (!map2(&maps.w[p], g.w, wrows, 64, 128u, false)) return -3;
         ph.tma_out = out_map_ok(g) ? 1 : 0;  // cleared below if no staging fits
         ph.split_rows = ph.tma_out && ph.ksplit > 1 ? g.split_stride / g.ldo : 0;
-        if (ph.tma_out && !make_out_map(&maps.out[p], g.out, out_map_rows(g, ph.ksplit), g.N, g.ldo)) return -3;
+        if (ph.tma_out && !make_out_map(&maps.out[p], g.out, out_map_rows(g, ph.ksplit), g.N, g.ldo, false)) return -3;
     }
     const size_t fixed = 1024 + static_cast<size_t>(2 * kMaxStages + 4 + 2 * kRing + 1) * 8 + kRing * 4 + 16 +
                          static_cast<size_t>(L.G + 1) * (8 + 4 * 4) + 4 + sizeof(PeerReport) + 64;

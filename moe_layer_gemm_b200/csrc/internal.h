@@ -96,7 +96,8 @@ struct GemmLaunch {
 // of its output map, and the map itself (box {32, 32}, 128-byte swizzle).
 bool out_map_ok(const GemmPhase& g);
 uint64_t out_map_rows(const GemmPhase& g, int ksplit);
-bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint64_t ld);
+bool h_map_ok(const GemmPhase& g);
+bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, uint64_t ld, bool bf16_out);
 
 // Test-only settings of the expert-GEMM launches (see moe_test_set_wait_limits
 // in the header); all zero in production.
