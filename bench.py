@@ -19,6 +19,9 @@ with capacity, and the DeepSeek-like layer whose steps update the bias in
 place and draw fresh tokens (step j takes the tokens of seed step j mod 10).
 A last entry runs the DeepSeek-shaped layer with its experts offloaded to
 host memory as INT4 and an LRU cache on the GPU (16-token decode steps).
+Timed regions carry no per-stage events; each is followed by as many steps
+with an event between every two stages, which give the stage split (and the
+expert-GEMM time of the roofline).
 
 ``--impl reference`` times the CPU oracle (the plain fp64 implementation the
 tests check against) on the host cores on a bounded token sample per step;
@@ -45,10 +48,9 @@ sys.path.insert(0, ROOT)
 from moe_layer_gemm_b200 import synth  # noqa: E402
 
 METRIC = "MoE-layer tokens/s on 1 B200 (Mixtral shape decode/prefill); % of roofline"
-# steps between the ones that carry per-stage events; workloads that draw
-# fresh tokens every step carry them on every step, so the stage times
-# average over all their token sets (every 4th step of 10 token sets would
-# see only half of them)
+# steps between the ones that carry per-stage events (working runs); the
+# bench's own timed regions carry none, and their stage split comes from a
+# second run with events on every step (see time_with_stages)
 STAGE_EVERY = 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -393,6 +395,20 @@ def time_steps(layer: Layer, K: int, barrier, clock_index: int, stage_every=None
                 peak_bytes=int(torch.cuda.max_memory_allocated(layer.dev)))
 
 
+def time_with_stages(layer: Layer, K: int, barrier, clock_index: int, start_step: int, n_staged: int = 0):
+    """The timed region (K steps, no per-stage events: an event between two
+    kernels costs a few microseconds per step), then n_staged (default K)
+    more steps with events on every step for the stage split, which covers
+    every token set of a workload that draws fresh tokens per step."""
+    res = time_steps(layer, K, barrier, clock_index, stage_every=0, start_step=start_step)
+    if layer.chunk == 0:
+        n = n_staged if n_staged > 0 else K
+        st = time_steps(layer, n, barrier, clock_index, stage_every=1, start_step=start_step + K)
+        res["stage_ms"] = st["stage_ms"]
+        res["staged_ms_step"] = st["ms_step"]
+    return res
+
+
 def roofline_of(layer: Layer, res: dict, peaks: dict, peak_src: str):
     """The expert-GEMM roofline (touched weight bytes or FLOPs over the
     kernel's event-timed duration) and the layer roofline of one timed run."""
@@ -552,7 +568,7 @@ def run_ours(args):
 
     # ---- timed region: K steps of the headline workload
     K = args.steps
-    res = time_steps(layer, K, barrier, local, start_step=args.warmup)
+    res = time_with_stages(layer, K, barrier, local, start_step=args.warmup)
     roof, layer_roof, routing = roofline_of(layer, res, peaks, peak_src)
     ms_step = res["ms_step"]
 
@@ -561,7 +577,7 @@ def run_ours(args):
     sustained = None
     if not args.no_sustained and chunk == 0:
         n_sus = max(K, int(np.ceil(1100.0 / max(ms_step, 1e-3))))
-        rs = time_steps(layer, n_sus, barrier, local, start_step=args.warmup + K)
+        rs = time_with_stages(layer, n_sus, barrier, local, start_step=args.warmup + 2 * K, n_staged=K)
         r2, l2, _ = roofline_of(layer, rs, peaks, peak_src)
         sustained = {"steps": n_sus, "ms_per_step": rs["ms_step"],
                      "value": job_tokens_per_s(wl.T, world, rs["ms_step"]), "timed_ms": rs["ms_total"],
@@ -652,7 +668,7 @@ def run_ours(args):
                 lx.step(i)
             torch.cuda.synchronize()
             lx.check_status(f"during warm-up ({name})")
-            rx = time_steps(lx, K, barrier, local, start_step=args.warmup)
+            rx = time_with_stages(lx, K, barrier, local, start_step=args.warmup)
             rf, lr, rt = roofline_of(lx, rx, peaks, peak_src)
             extras[name] = {"value": job_tokens_per_s(wx.T, world, rx["ms_step"]), "unit": "tokens/s",
                             "ms_per_step": rx["ms_step"], "steps": K, "warmup": args.warmup,

@@ -259,9 +259,12 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     // group offsets, scheduler words and token rows come from earlier kernels
     pdl_wait();
-    // the next kernel may launch now: its CTAs wait in their own pdl_wait
-    // until this grid completes, but no launch gap remains
-    pdl_trigger();
+    // The next kernel may launch once every CTA has run out of tiles (its
+    // producer sees the end marker, below): its CTAs then wait in their own
+    // pdl_wait while the last tiles finish.  Triggered at the start instead,
+    // the next kernel's CTAs sat resident on every SM for the whole launch
+    // (DeepSeek-like layer: 5.33 ms per step against 5.14 with the kernels
+    // serialised).
     for (int g = threadIdx.x; g <= G; g += blockDim.x)
         off[g] = a.group_off ? static_cast<int64_t>(a.group_off[g]) : (g == 0 ? 0 : a.dense_rows);
     __syncthreads();
@@ -331,7 +334,10 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
                     mbar_arrive(&rempty[r]);
                 }
                 if (++r == kRing) { r = 0; rph ^= 1u; }
-                if (tile < 0) break;  // the end marker
+                if (tile < 0) {  // the end marker
+                    pdl_trigger();
+                    break;
+                }
                 const Tile t = decode_tile(a, tile, tstart, off);
                 const PhaseArgs& pa = a.ph[t.phase];
                 if (t.phase == 1 && a.dep) {

@@ -403,9 +403,12 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     }
     // group offsets, scheduler words and token rows come from earlier kernels
     pdl_wait();
-    // the next kernel (the combine) may launch now: its CTAs wait in their own
-    // pdl_wait until this grid completes, but no launch gap remains
-    pdl_trigger();
+    // The next kernel may launch once every CTA has run out of tiles (its
+    // producer sees the end marker, below): its CTAs then wait in their own
+    // pdl_wait while the last tiles finish.  Triggered at the start instead,
+    // the next kernel's CTAs sat resident on every SM for the whole launch
+    // (DeepSeek-like layer: 5.33 ms per step against 5.14 with the kernels
+    // serialised).
     for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
     __syncthreads();
     // rows of group g in this launch (0 for a group the slot table skips)
@@ -505,7 +508,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                     remote_arrive(leader_rempty0 + 8u * r);
                 }
                 if (++r == kRing) { r = 0; rph ^= 1u; }
-                if (tile < 0) break;  // the end marker
+                if (tile < 0) {  // the end marker
+                    pdl_trigger();
+                    break;
+                }
                 const Tile2 t = decode2<kHalfTiles>(a, tile, tstart, off);
                 const Phase2& pa = a.ph[t.phase];
                 if (t.phase == 1 && a.dep) {
@@ -996,7 +1002,7 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // pdl_wait in the kernel
     attrs[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attrs;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = kProgrammaticLaunch ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, kern, maps, a) != cudaSuccess) return -3;
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
