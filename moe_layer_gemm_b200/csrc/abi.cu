@@ -104,6 +104,9 @@ void router_tiling(const moe_dims* d, int E_pad, int* bn, int* split) {
 // padding and the weight stream dominates.
 constexpr int kSwapMaxRows = 128;
 
+// Largest batch routed by the fused warp-per-token router (E <= 32).
+constexpr int64_t kFusedRouterMaxTokens = 4096;
+
 // Weight-major tiles are enabled when groups of decode size are expected:
 // a mean group of at most 256 rows (skewed routing then also leaves many
 // small groups).  (Weight-major CTA-pair tiles of up to 256 tokens for
@@ -136,7 +139,11 @@ Layout layout_of(const moe_dims* d) {
     const int64_t A = T * K;
     L.route_nb = route_blocks(T);
     L.perm_nb = permute_blocks(T);
-    L.fused_router = route_fused_supported(d->d_model, d->E) != 0;
+    // The fused router (a warp per token, W_r converted from bf16 for every
+    // token) is instruction-bound at large T; past 4096 tokens the tensor-core
+    // logits GEMM + top-K path is faster (moe_route at d = 4096, E = 8:
+    // 33 vs 34 us at T = 4096, 47 vs 43 us at 8192, 96 vs 56 us at 16384).
+    L.fused_router = route_fused_supported(d->d_model, d->E) != 0 && d->T <= kFusedRouterMaxTokens;
     L.E_pad = static_cast<int>(((E + 31) / 32) * 32);
     router_tiling(d, L.E_pad, &L.router_bn, &L.router_split);
     if (L.fused_router) L.router_split = 1;

@@ -122,8 +122,10 @@ def test_layer_launch_counts(lib):
     assert abi.moe_layer_launch_count(abi.Dims(256, 4096, 14336, 8, 2), True, False) == 4
     # statistics and the bias update add no launch
     assert abi.moe_layer_launch_count(abi.Dims(256, 4096, 14336, 8, 2), True, True) == 4
-    # prefill: fused router, hist / scan / rank + gather, GEMMs, combine
-    assert abi.moe_layer_launch_count(abi.Dims(16384, 4096, 14336, 8, 2), True, False) == 7
+    # prefill (T > 4096): transpose + logits GEMM + top-K router, hist / scan / rank + gather, GEMMs, combine
+    assert abi.moe_layer_launch_count(abi.Dims(16384, 4096, 14336, 8, 2), True, False) == 9
+    # up to 4096 tokens the fused router: one launch
+    assert abi.moe_layer_launch_count(abi.Dims(4096, 4096, 14336, 8, 2), True, False) == 7
     # E > 32: transpose + logits GEMM + top-K router; DeepSeek-like T = 4096 > 1024
     assert abi.moe_layer_launch_count(abi.Dims(4096, 7168, 2048, 256, 8), True, True) == 9
 
@@ -168,11 +170,13 @@ def test_chunked_workspace_and_host_checks(lib):
 
 
 def test_chunked_launch_counts(lib):
-    # Mixtral prefill in 4 chunks of 4096: fused router + 4 x (hist/scan/rank + gather, GEMMs, combine,
-    # counts) + the statistics CTA
+    # Mixtral prefill in 4 chunks of 4096: the router of the whole batch (16384 tokens: transpose + logits
+    # GEMM + top-K) + 4 x (hist/scan/rank + gather, GEMMs, combine, counts) + the statistics CTA
     d = abi.Dims(16384, 4096, 14336, 8, 2)
-    assert abi.moe_layer_chunked_launch_count(d, 4096, True, False) == 1 + 4 * (4 + 3) + 1
+    assert abi.moe_layer_chunked_launch_count(d, 4096, True, False) == 3 + 4 * (4 + 3) + 1
     # chunks of 1024 take the one-launch dispatch
-    assert abi.moe_layer_chunked_launch_count(d, 1024, True, False) == 1 + 16 * (1 + 3) + 1
+    assert abi.moe_layer_chunked_launch_count(d, 1024, True, False) == 3 + 16 * (1 + 3) + 1
     # no statistics, no bias: no statistics CTA
-    assert abi.moe_layer_chunked_launch_count(d, 16384, False, False) == 1 + (4 + 3)
+    assert abi.moe_layer_chunked_launch_count(d, 16384, False, False) == 3 + (4 + 3)
+    # a batch of 4096 tokens is routed by the fused router
+    assert abi.moe_layer_chunked_launch_count(abi.Dims(4096, 4096, 14336, 8, 2), 1024, True, False) == 1 + 4 * (1 + 3) + 1
