@@ -388,9 +388,11 @@ int launch_combine(const float* y_perm, int nsplit, int64_t split_stride, const 
         ++grid;  // one extra CTA for the tail
     }
     if (nsplit == 1 && K <= 32 && d >= 128) {
-        // a warp per token: 8 tokens per CTA, the grid capped at 4 CTAs per SM
+        // a warp per token: 8 tokens per CTA, the grid (with the statistics
+        // CTA) capped at 4 CTAs per SM, one resident wave; a statistics CTA
+        // beyond the wave would start only once a token CTA had finished
         int64_t gw = (T + 7) / 8;
-        const int64_t cap = static_cast<int64_t>(sms) * 4;
+        const int64_t cap = static_cast<int64_t>(sms) * 4 - (tail.counts ? 1 : 0);
         if (gw > cap) gw = cap;
         if (gw < 1) gw = 1;
         if (tail.counts) ++gw;
