@@ -22,16 +22,19 @@
 //                 pre-swizzled packed weights
 //   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2..5    epilogue: TMEM -> registers -> SwiGLU / fp32 -> global.
-//                 fp32 rows of token-major tiles go through a 4 KB staging
-//                 buffer per warp and one TMA tile store per 32 x 32 block:
-//                 stored from registers, each 16-byte store touched 32 rows,
-//                 and the down projection's short tiles (reduction d_ff) could
-//                 not hide them (Qwen-like layer: expert GEMMs 0.430 ->
-//                 0.412 ms; the same layer with no fp32 stores at all, 0.39)
-// Two producers: the copies one thread issues after a barrier wait are
-// serviced one stage at a time (a measured property of the copy engine:
-// about 0.4 us per stage and issuing thread, whatever the ring depth), so a
-// second issuing thread doubles the stage rate.
+//                 Rows of token-major tiles go through a 4 KB staging buffer
+//                 per warp and one TMA tile store per 32 x 32 fp32 block (or
+//                 32 x 64 bf16 block of H): stored from registers, each
+//                 16-byte store touched 32 rows, and the down projection's
+//                 short tiles (reduction d_ff) could not hide them (Qwen-like
+//                 layer: expert GEMMs 0.430 -> 0.411 ms; with no output
+//                 stores at all, 0.39)
+// Two producers: with 16 KB stages a probe measured one issuing thread at
+// about one stage per 0.4 us whatever the ring depth, and two threads at
+// twice that; with this kernel's 48 KB stages the probe's rate no longer
+// depends on the number of issuing threads (the copy engine's throughput,
+// about 140 GB/s per SM with every SM loading, binds), and the second
+// producer measured 2-3 % faster at the Qwen-like shape.
 // The accumulator is double-buffered in TMEM (2 x 256 fp32 columns).
 //
 // Tile orientation is chosen per group:
@@ -259,12 +262,10 @@ grouped_gemm_kernel(const __grid_constant__ Maps maps, const DevArgs a) {
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
     // group offsets, scheduler words and token rows come from earlier kernels
     pdl_wait();
-    // The next kernel may launch once every CTA has run out of tiles (its
-    // producer sees the end marker, below): its CTAs then wait in their own
-    // pdl_wait while the last tiles finish.  Triggered at the start instead,
-    // the next kernel's CTAs sat resident on every SM for the whole launch
-    // (DeepSeek-like layer: 5.33 ms per step against 5.14 with the kernels
-    // serialised).
+    // Under programmatic launch (kProgrammaticLaunch, off by default) the
+    // next kernel may launch once every CTA has run out of tiles (its
+    // producer sees the end marker, below), so its CTAs do not sit resident
+    // on the SMs through the whole launch, only through the last tiles.
     for (int g = threadIdx.x; g <= G; g += blockDim.x)
         off[g] = a.group_off ? static_cast<int64_t>(a.group_off[g]) : (g == 0 ? 0 : a.dense_rows);
     __syncthreads();

@@ -23,6 +23,13 @@
 // MMAs into two TMEM accumulators, which halves the token traffic again.
 // The down projection's reduction can be split as in gemm.cu.
 //
+// Where weight-major tiles are enabled (mixed group sizes), a token-major
+// group's last chunk of at most 128 rows takes a 128-row tile instead of a
+// 256-row one: tcgen05.mma cta_group::2 with M = 128, each CTA loading 64
+// token rows; a CTA's accumulator then holds its 64 rows in TMEM lanes 0-63
+// for output columns 0-127 and in lanes 64-127 for columns 128-255.  This is
+// the kHalfTiles instance of the kernel.
+//
 // Two tile queues.  Token-major tiles (large groups) and weight-major tiles
 // (small groups) are numbered in separate queues, each phase 0 then phase 1
 // in group order, with a tile counter each.  At kernel start every CTA
@@ -403,12 +410,10 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
     }
     // group offsets, scheduler words and token rows come from earlier kernels
     pdl_wait();
-    // The next kernel may launch once every CTA has run out of tiles (its
-    // producer sees the end marker, below): its CTAs then wait in their own
-    // pdl_wait while the last tiles finish.  Triggered at the start instead,
-    // the next kernel's CTAs sat resident on every SM for the whole launch
-    // (DeepSeek-like layer: 5.33 ms per step against 5.14 with the kernels
-    // serialised).
+    // Under programmatic launch (kProgrammaticLaunch, off by default) the
+    // next kernel may launch once every CTA has run out of tiles (its
+    // producer sees the end marker, below), so its CTAs do not sit resident
+    // on the SMs through the whole launch, only through the last tiles.
     for (int g = threadIdx.x; g <= G; g += blockDim.x) off[g] = static_cast<int64_t>(a.group_off[g]);
     __syncthreads();
     // rows of group g in this launch (0 for a group the slot table skips)
