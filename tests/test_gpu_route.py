@@ -38,6 +38,7 @@ def test_route_from_logits_bitexact(T, E, K, use_bias, tie):
 
 
 @pytest.mark.parametrize("name,T", [("tiny", 64), ("mixtral_decode", 256), ("mixtral_prefill", 3000),
+                                    ("mixtral_prefill", 5000),  # past 4096 tokens: logits GEMM + top-K at E = 8
                                     ("qwen_capacity", 1000), ("deepseek_bias", 700)])
 def test_route_fused_vs_oracle(name, T):
     d = dev()
