@@ -386,12 +386,13 @@ grouped_gemm_2sm_kernel(const __grid_constant__ Maps2 maps, const Args2 a) {
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
-    // Weight tiles depend on no earlier kernel.  While the router and the
-    // dispatch finish, pull the first k-blocks of the first round of
-    // weight-major tiles into L2: cluster c takes tile c of the first phase,
-    // as if every group had one token chunk (the decode case); whichever
-    // cluster claims that tile later finds them in L2.  A hint only: no
-    // result depends on it, and every address lies inside the packed weights.
+    // Weight tiles depend on no earlier kernel.  Under programmatic launch,
+    // while the router and the dispatch finish, pull the first k-blocks of
+    // the first round of weight-major tiles into L2: cluster c takes tile c
+    // of the first phase, as if every group had one token chunk (the decode
+    // case); whichever cluster claims that tile later finds them in L2.  A
+    // hint only: no result depends on it, and every address lies inside the
+    // packed weights.
     if (a.prefetch_kb > 0 && warp == 0 && lane == 0) {
         const Phase2& p0 = a.ph[0];
         const int tpg = (p0.N / (256 * p0.wt)) * p0.ksplit;  // tiles per group with one token chunk
@@ -948,9 +949,12 @@ int launch_grouped_gemm_2sm(const GemmLaunch& L, cudaStream_t st) {
     int wt_max = 1;
     for (int p = 0; p < L.nphase; ++p) wt_max = a.ph[p].wt > wt_max ? a.ph[p].wt : wt_max;
     a.xoff = static_cast<uint32_t>(wt_max) * kHalf;
-    // decode-sized launches (weight-major tiles for groups of <= 128 rows):
-    // prefetch up to 16 k-blocks of each first-round weight tile
-    a.prefetch_kb = (weight_major_possible && L.w_slot == nullptr)
+    // decode-sized launches (weight-major tiles for groups of <= 128 rows)
+    // under programmatic launch: prefetch up to 16 k-blocks of each
+    // first-round weight tile.  Without it the prefetch cannot overlap the
+    // earlier kernels and measured slightly slower at decode (0.488-0.490 vs
+    // 0.485-0.488 ms per step), so it is off.
+    a.prefetch_kb = (kProgrammaticLaunch && weight_major_possible && L.w_slot == nullptr)
                         ? (a.ph[0].k_blocks < 16 ? a.ph[0].k_blocks : 16) : 0;
     // Rings.  Token-major pairs: 32 KB per k-block and CTA, two k-blocks per
     // stage where three such stages fit (a producer thread's copies issued
