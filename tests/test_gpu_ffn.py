@@ -100,3 +100,50 @@ def test_expert_ffn_vs_oracle(T, d, f, E, K, skew):
     assert np.all(np.abs(Hg - H) <= np.abs(H) * 2.0 ** -8 + 1e-4)
     assert_close_y(r["yp"][:n], r["Y"][:n], Y_MAX_ABS, Y_REL_L2, "y_perm")
     assert_close_y(r["yp"][:n], r["Yr"][:n], Y_MIRROR_MAX_ABS, Y_MIRROR_REL_L2, "y_perm (H rounded)")
+
+
+# Explicit group sizes on the edges of the epilogue's and the tiles' cases:
+# 32-row slabs that are exactly full (staged TMA stores) or not (direct
+# stores), last chunks of 1, 33, 44 and 128 rows, groups of 129 and 257 rows,
+# empty groups; each case checks that the kernel it means to reach is the one
+# launched.
+@pytest.mark.parametrize("d,f,sizes,kernel", [
+    # single-CTA token-major tiles (mean group 500 rows): slabs of 128, 160 (the last exactly 32), 33, 1, 118 rows
+    (256, 384, [128, 160, 0, 33, 1, 2678], "grouped_gemm_kernel"),
+    # CTA pairs with weight-major tiles enabled: 128-row last chunks of 1, 128 and 44 rows, a 129-row group
+    (256, 256, [257, 384, 129, 0, 31, 128, 300, 100], "grouped_gemm_2sm_kernel"),
+    # CTA pairs, groups of >= 1024 rows on average: 256-row last chunks of 33 and 127 rows
+    (256, 256, [1057, 2175], "grouped_gemm_2sm_kernel"),
+    # CTA pairs with a 4-way split of the down projection and one 300-row group (256 + a 44-row chunk)
+    (256, 1024, [300, 40, 40, 40, 40, 40, 40, 40], "grouped_gemm_2sm_kernel"),
+])
+def test_expert_ffn_explicit_groups(d, f, sizes, kernel):
+    dv = dev()
+    E, T = len(sizes), sum(sizes)
+    dims = abi.Dims(T, d, f, E, 1)
+    assert abi.moe_ffn_kernel(dims) == kernel
+    seed = 21
+    w_std = 0.05 * min(1.0, (256.0 / d) ** 0.5)
+    xp = synth.normal_bf16((T, d), seed, synth.STREAM_X, 1.0, dv)
+    W1 = synth.normal_bf16((E, d, f), seed, synth.STREAM_W1, w_std, dv)
+    W3 = synth.normal_bf16((E, d, f), seed, synth.STREAM_W3, w_std, dv)
+    W2 = synth.normal_bf16((E, f, d), seed, synth.STREAM_W2, w_std, dv)
+    W13p, W2p = abi.pack_weights(dims, W1, W3, W2)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    offsets = torch.from_numpy(off).to(dv)
+    ws = abi.alloc_workspace(dims)
+    h = torch.zeros(T, f, dtype=torch.bfloat16, device=dv)
+    yp = torch.zeros(T, d, dtype=torch.float32, device=dv)
+    abi.moe_expert_ffn(dims, xp, offsets, W13p, W2p, h, yp, ws)
+    torch.cuda.synchronize()
+    st, detail = abi.moe_get_device_status(ws)
+    assert st == abi.MOE_OK, f"device wait ran out (code {detail})"
+    x64, W1h, W3h, W2h = f64(xp), f64(W1), f64(W3), f64(W2)
+    Y, Yr = np.zeros((T, d)), np.zeros((T, d))
+    for e in range(E):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if r1 > r0:
+            Y[r0:r1] = O.swiglu_ffn(x64[r0:r1], W1h[e], W3h[e], W2h[e])
+            Yr[r0:r1] = O.swiglu_ffn(x64[r0:r1], W1h[e], W3h[e], W2h[e], h_round=O.bf16_round)
+    assert_close_y(f64(yp), Y, Y_MAX_ABS, Y_REL_L2, "y_perm")
+    assert_close_y(f64(yp), Yr, Y_MIRROR_MAX_ABS, Y_MIRROR_REL_L2, "y_perm (H rounded)")
